@@ -1,0 +1,352 @@
+"""Pins of the fp64 oracle to facts fixed independently of it: hand-derived fixtures, closed forms,
+textbook reshapes, brute force on tiny inputs and invariants.  CPU only."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from conftest import read_golden
+from mate_inputs import CONFIGS, MateConfig, make_inputs
+from oracle import mate_oracle as O
+
+
+# ------------------------------------------------------------------ Rotary Major Scan
+
+def test_rms_orders_match_hand_fixture():
+    g = read_golden("rms_orders_T2_H2_W3.txt")
+    T, H, W = 2, 2, 3
+    for o in range(4):
+        pos = O.scan_positions(T, H, W, o)
+        visited = np.empty(T * H * W, dtype=np.int64)
+        for t, h, w in itertools.product(range(T), range(H), range(W)):
+            visited[pos[t, h, w]] = (t * H + h) * W + w
+        assert visited.tolist() == [int(v) for v in g[f"order{o}"]], o
+
+
+@pytest.mark.parametrize("grid", [(4, 8, 8), (3, 5, 7), (1, 1, 6), (16, 32, 32)])
+def test_rms_is_a_bijection_with_exact_inverse(grid):
+    T, H, W = grid
+    rng = np.random.default_rng(0)
+    X = rng.standard_normal((T, H, W, 3)).astype(np.float32)
+    for o in range(4):
+        pos = O.scan_positions(T, H, W, o)
+        assert np.array_equal(np.sort(pos.ravel()), np.arange(T * H * W))  # every token exactly once
+        Xp = O.rms_permute(X, o)
+        assert np.array_equal(O.rms_unpermute(Xp, o, T, H, W), X)          # bitwise round trip
+
+
+@pytest.mark.parametrize("grid", [(4, 8, 8), (3, 5, 7)])
+def test_rms_orders_equal_textbook_transposes(grid):
+    T, H, W = grid
+    X = np.random.default_rng(1).standard_normal((T, H, W, 2))
+    n = T * H * W
+    # order 0 is plain raster order; the others are axis transposes followed by a reshape
+    assert np.array_equal(O.rms_permute(X, 0), X.reshape(n, 2))
+    assert np.array_equal(O.rms_permute(X, 1), X.transpose(0, 2, 1, 3).reshape(n, 2))   # T, W, H(fastest)
+    assert np.array_equal(O.rms_permute(X, 2), X.transpose(1, 2, 0, 3).reshape(n, 2))   # H, W, T(fastest)
+    assert np.array_equal(O.rms_permute(X, 3), X.transpose(2, 1, 0, 3).reshape(n, 2))   # W, H, T(fastest)
+
+
+# ------------------------------------------------------------------ review tokens
+
+def test_review_tokens_unit_pool_is_the_scan():
+    X = np.random.default_rng(2).standard_normal((3, 4, 4, 5))
+    for o in range(4):
+        assert np.allclose(O.review_tokens(X, 48, o), O.rms_permute(X, o), atol=0, rtol=1e-15)
+
+
+@pytest.mark.parametrize("grid,R", [((4, 8, 8), 16), ((8, 8, 12), 32), ((6, 4, 8), 48)])
+def test_review_tokens_preserve_total_mass(grid, R):
+    T, H, W = grid
+    X = np.random.default_rng(3).standard_normal((T, H, W, 7))
+    _, f = O.review_grid(T, H, W, R)
+    vol = f[0] * f[1] * f[2]
+    for o in range(4):
+        Rv = O.review_tokens(X, R, o)
+        assert Rv.shape == (R, 7)
+        np.testing.assert_allclose(Rv.sum(axis=0) * vol, X.reshape(-1, 7).sum(axis=0), rtol=1e-12, atol=1e-12)
+
+
+def test_review_tokens_constant_cells():
+    # X constant on every pool cell: each review token equals its cell's constant, listed in scan order
+    T, H, W, R = 4, 8, 8, 32
+    (Tr, Hr, Wr), (ft, fh, fw) = O.review_grid(T, H, W, R)
+    cellval = np.arange(Tr * Hr * Wr, dtype=np.float64).reshape(Tr, Hr, Wr)
+    X = np.repeat(np.repeat(np.repeat(cellval, ft, 0), fh, 1), fw, 2)[..., None]
+    for o in range(4):
+        pos = O.scan_positions(Tr, Hr, Wr, o)
+        expect = np.empty(R)
+        expect[pos.ravel()] = cellval.ravel()
+        assert np.array_equal(O.review_tokens(X, R, o)[:, 0], expect)
+
+
+# ------------------------------------------------------------------ selective scan
+
+def test_ssd_hand_scalar():
+    g = read_golden("ssd_hand.txt")
+    x = np.array(g["scalar.x"])[:, None, None]
+    y = O.ssd_recurrence(x, np.array(g["scalar.B"])[:, None], np.array(g["scalar.C"])[:, None],
+                         np.array(g["scalar.delta"])[:, None], np.array(g["scalar.A"]), np.array(g["scalar.D"]))
+    np.testing.assert_allclose(y[:, 0, 0], g["scalar.y"], rtol=1e-14, atol=1e-14)
+
+
+def test_ssd_hand_orientation():
+    g = read_golden("ssd_hand.txt")
+    x = np.array(g["orient.x"])[:, None, None]
+    Bm = np.array(g["orient.B"]).reshape(2, 2)
+    Cm = np.array(g["orient.C"]).reshape(2, 2)
+    y = O.ssd_recurrence(x, Bm, Cm, np.ones((2, 1)), np.zeros(1), np.zeros(1))
+    np.testing.assert_allclose(y[:, 0, 0], g["orient.y"], atol=1e-15)
+
+
+def test_ssd_hand_bidirectional_with_prefix():
+    g = read_golden("ssd_hand.txt")
+    x = np.array(g["bidir.x"])[:, None, None]
+    ones = np.ones((3, 1))
+    y = O.ssd_bidirectional(x, ones, ones, ones, np.array([-math.log(2.0)]), np.zeros(1), R=1)
+    np.testing.assert_allclose(y[:, 0, 0], g["bidir.y_video"], rtol=1e-14)
+
+
+def _rand_ssd(L, nh, P, N, seed, long_memory=False):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((L, nh, P))
+    Bm = rng.standard_normal((L, N))
+    Cm = rng.standard_normal((L, N))
+    delta = O.softplus(rng.standard_normal((L, nh)) - (4.0 if long_memory else 0.0))
+    A = -np.exp(rng.uniform(-3 if long_memory else 0, 1, nh))
+    D = rng.standard_normal(nh)
+    return x, Bm, Cm, delta, A, D
+
+
+@pytest.mark.parametrize("long_memory", [False, True])
+def test_ssd_equals_dense_quadratic_form(long_memory):
+    # y = (Lmask o C B^T)(delta x) + D x with Lmask[i, j] = exp(sum_{k=j+1..i} delta_k A), j <= i
+    L, nh, P, N = 37, 3, 4, 5
+    x, Bm, Cm, delta, A, D = _rand_ssd(L, nh, P, N, 4, long_memory)
+    y = O.ssd_recurrence(x, Bm, Cm, delta, A, D)
+    G = Cm @ Bm.T
+    for hh in range(nh):
+        a = delta[:, hh] * A[hh]
+        Lm = np.zeros((L, L))
+        for i in range(L):
+            for j in range(i + 1):
+                Lm[i, j] = math.exp(a[j + 1:i + 1].sum())
+        yq = (Lm * G) @ (delta[:, hh:hh + 1] * x[:, hh, :]) + D[hh] * x[:, hh, :]
+        np.testing.assert_allclose(y[:, hh, :], yq, rtol=1e-11, atol=1e-11)
+
+
+def _chunked_ssd(x, Bm, Cm, delta, A, D, Q):
+    """Chunked state-space-duality evaluation (intra-chunk quadratic part + carried chunk states)."""
+    L, nh, P = x.shape
+    N = Bm.shape[1]
+    y = np.zeros_like(x)
+    for hh in range(nh):
+        Hs = np.zeros((P, N))
+        for c0 in range(0, L, Q):
+            c1 = min(c0 + Q, L)
+            a = delta[c0:c1, hh] * A[hh]
+            s = np.cumsum(a)
+            seg = s[:, None] - s[None, :]
+            Lm = np.where(np.tril(np.ones((c1 - c0, c1 - c0))) > 0, np.exp(np.minimum(seg, 0)), 0.0)
+            u = delta[c0:c1, hh:hh + 1] * x[c0:c1, hh, :]
+            yc = (Lm * (Cm[c0:c1] @ Bm[c0:c1].T)) @ u
+            yc += np.exp(s)[:, None] * (Cm[c0:c1] @ Hs.T)
+            y[c0:c1, hh, :] = yc + D[hh] * x[c0:c1, hh, :]
+            w = np.exp(s[-1] - s)
+            Hs = math.exp(s[-1]) * Hs + (w[:, None] * u).T @ Bm[c0:c1]
+    return y
+
+
+@pytest.mark.parametrize("Q", [1, 16, 64, 100])
+def test_ssd_equals_chunked_form(Q):
+    L, nh, P, N = 100, 2, 3, 6
+    for lm in (False, True):
+        args = _rand_ssd(L, nh, P, N, 5, lm)
+        np.testing.assert_allclose(O.ssd_recurrence(*args), _chunked_ssd(*args, Q), rtol=1e-11, atol=1e-11)
+
+
+def test_ssd_no_decay_is_prefix_sum():
+    # A = 0, D = 0: y_t = (sum_{s<=t} delta_s x_s B_s^T) C_t
+    L, nh, P, N = 50, 2, 3, 4
+    x, Bm, Cm, delta, _, _ = _rand_ssd(L, nh, P, N, 6)
+    y = O.ssd_recurrence(x, Bm, Cm, delta, np.zeros(nh), np.zeros(nh))
+    Hc = np.cumsum((delta[:, :, None, None] * x[:, :, :, None]) * Bm[:, None, None, :], axis=0)
+    np.testing.assert_allclose(y, np.einsum("thpn,tn->thp", Hc, Cm), rtol=1e-12, atol=1e-12)
+
+
+def test_ssd_geometric_series():
+    # P = N = 1, constant delta, B = C = x = 1: h_t = delta * (1 - q^(t+1)) / (1 - q), q = exp(delta A)
+    L, dl, A = 60, 0.3, -0.7
+    y = O.ssd_recurrence(np.ones((L, 1, 1)), np.ones((L, 1)), np.ones((L, 1)), np.full((L, 1), dl),
+                         np.array([A]), np.zeros(1))
+    q = math.exp(dl * A)
+    t = np.arange(L)
+    np.testing.assert_allclose(y[:, 0, 0], dl * (1 - q ** (t + 1)) / (1 - q), rtol=1e-13)
+
+
+def test_bidirectional_identity_without_prefix():
+    L, nh, P, N = 30, 2, 3, 4
+    x, Bm, Cm, delta, A, D = _rand_ssd(L, nh, P, N, 7)
+    y = O.ssd_bidirectional(x, Bm, Cm, delta, A, D, R=0)
+    yf = O.ssd_recurrence(x, Bm, Cm, delta, A, D)
+    yb = O.ssd_recurrence(x[::-1], Bm[::-1], Cm[::-1], delta[::-1], A, D)[::-1]
+    np.testing.assert_allclose(y, yf + yb, rtol=1e-13, atol=1e-13)
+
+
+def test_bidirectional_zero_prefix_reduces_to_no_prefix():
+    L, R, nh, P, N = 30, 5, 2, 3, 4
+    x, Bm, Cm, delta, A, D = _rand_ssd(L + R, nh, P, N, 8)
+    x[:R] = 0.0
+    Bm[:R] = 0.0
+    y_r = O.ssd_bidirectional(x, Bm, Cm, delta, A, D, R=R)
+    y_0 = O.ssd_bidirectional(x[R:], Bm[R:], Cm[R:], delta[R:], A, D, R=0)
+    np.testing.assert_allclose(y_r, y_0, rtol=1e-13, atol=1e-13)
+
+
+def test_softplus_values():
+    v = np.array([-40.0, -1.0, 0.0, 2.0, 50.0])
+    expect = [math.log1p(math.exp(t)) if t < 0 else t + math.log1p(math.exp(-t)) for t in v]
+    np.testing.assert_allclose(O.softplus(v), expect, rtol=1e-14)
+
+
+# ------------------------------------------------------------------ TEmporal Swin Attention
+
+def _tesa_hand_qkv():
+    g = read_golden("tesa_hand.txt")
+    qkv = np.stack([g["q"], g["k"], g["v"]], axis=-1).reshape(1, 1, 4, 3)
+    return g, qkv
+
+
+def test_tesa_hand_shifted_and_unshifted():
+    g, qkv = _tesa_hand_qkv()
+    out_s = O.tesa_attention(qkv, 1, 1, (1, 1, 2), (0, 0, 1), True)
+    out_u = O.tesa_attention(qkv, 1, 1, (1, 1, 2), (0, 0, 1), False)
+    np.testing.assert_allclose(out_s.ravel(), g["shifted"], rtol=1e-12)
+    np.testing.assert_allclose(out_u.ravel(), g["unshifted"], rtol=1e-12)
+
+
+def test_tesa_single_window_is_full_attention():
+    T, H, W, th, tp = 2, 3, 4, 2, 5
+    qkv = np.random.default_rng(9).standard_normal((T, H, W, 3 * th * tp))
+    out = O.tesa_attention(qkv, th, tp, (T, H, W), (1, 1, 2), False)
+    n = T * H * W
+    flat = qkv.reshape(n, 3, th, tp)
+    for hh in range(th):
+        q, k, v = flat[:, 0, hh], flat[:, 1, hh], flat[:, 2, hh]
+        s = q @ k.T / math.sqrt(tp)
+        p = np.exp(s - s.max(1, keepdims=True))
+        ref = (p / p.sum(1, keepdims=True)) @ v
+        np.testing.assert_allclose(out.reshape(n, th, tp)[:, hh], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_tesa_zero_shift_equals_unshifted():
+    qkv = np.random.default_rng(10).standard_normal((4, 8, 8, 3 * 2 * 4))
+    a = O.tesa_attention(qkv, 2, 4, (2, 4, 4), (0, 0, 0), True)
+    b = O.tesa_attention(qkv, 2, 4, (2, 4, 4), (1, 2, 2), False)
+    np.testing.assert_allclose(a, b, rtol=1e-14, atol=1e-14)
+
+
+@pytest.mark.parametrize("shifted", [False, True])
+def test_tesa_attention_support_and_row_sums(shifted):
+    # With v = one-hot of the key token, the output row of a query is its attention distribution.
+    # Its support must be: same shifted window on every axis and same wrap status (o < s) on every axis.
+    T, H, W = 4, 4, 6
+    win, sh = (2, 2, 2), (1, 1, 1)
+    n = T * H * W
+    rng = np.random.default_rng(11)
+    q = rng.standard_normal((n, 3))
+    k = rng.standard_normal((n, 3))
+    qkv = np.zeros((T, H, W, 3 + 3 + n))
+    qkv[..., :3] = q.reshape(T, H, W, 3)
+    qkv[..., 3:6] = k.reshape(T, H, W, 3)
+    # tp differs per slot here, so evaluate with a single head of size n by padding q, k with zeros
+    tp = n
+    qkv2 = np.zeros((T, H, W, 3 * tp))
+    qkv2[..., :3] = q.reshape(T, H, W, 3)
+    qkv2[..., tp:tp + 3] = k.reshape(T, H, W, 3)
+    qkv2[..., 2 * tp:] = np.eye(n).reshape(T, H, W, n)
+    att = O.tesa_attention(qkv2, 1, tp, win, sh, shifted).reshape(n, n)
+    np.testing.assert_allclose(att.sum(1), 1.0, rtol=1e-13)
+    s = sh if shifted else (0, 0, 0)
+    dims = (T, H, W)
+    coords = np.array(list(itertools.product(range(T), range(H), range(W))))
+    for i in range(n):
+        for j in range(n):
+            same = True
+            for ax in range(3):
+                oi, oj, D, w, ss = coords[i, ax], coords[j, ax], dims[ax], win[ax], s[ax]
+                same &= ((oi - ss) % D) // w == ((oj - ss) % D) // w
+                same &= (oi < ss) == (oj < ss)
+            assert (att[i, j] > 0) == same, (i, j)
+
+
+def test_tesa_interior_windows_are_translation_equivariant():
+    # Away from the wrap-around, a shifted layer is the unshifted layer applied to the rolled grid.
+    T, H, W, th, tp = 4, 8, 8, 2, 3
+    win, s = (2, 4, 4), (1, 2, 2)
+    qkv = np.random.default_rng(12).standard_normal((T, H, W, 3 * th * tp))
+    out_s = O.tesa_attention(qkv, th, tp, win, s, True)
+    rolled = np.roll(qkv, shift=(-s[0], -s[1], -s[2]), axis=(0, 1, 2))
+    out_u = np.roll(O.tesa_attention(rolled, th, tp, win, s, False), shift=s, axis=(0, 1, 2))
+    for t, h, w in itertools.product(range(T), range(H), range(W)):
+        # shifted position of the token; windows ending at the grid edge hold wrapped tokens
+        p = ((t - s[0]) % T, (h - s[1]) % H, (w - s[2]) % W)
+        if p[0] < T - win[0] and p[1] < H - win[1] and p[2] < W - win[2]:
+            np.testing.assert_allclose(out_s[t, h, w], out_u[t, h, w], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ block-level properties
+
+def _small_cfg(T=4, H=8, W=8, R=16, B=1):
+    return MateConfig("t", B, T, H, W, 16, 2, 8, 4, 64, R, 2, 8, 2, 4, 4, 1, 2, 2, "f32", 0)
+
+
+def test_work_is_linear_in_token_count():
+    per_token = []
+    for T in (4, 8, 16):
+        cfg = _small_cfg(T=T, R=4 * T)
+        w = make_inputs(cfg)
+        c = {}
+        O.mate_forward(w["X"], w, cfg, 1, counter=c)
+        per_token.append({k: v / (cfg.n + cfg.R * (k != "tesa")) for k, v in c.items()})
+    for k in per_token[0]:
+        vals = [p[k] for p in per_token]
+        assert max(vals) / min(vals) < 1.0 + 1e-9, (k, vals)
+
+
+def test_block_is_sum_of_branches():
+    cfg = _small_cfg()
+    w = make_inputs(cfg)
+    for layer in range(4):
+        full = O.mate_forward(w["X"], w, cfg, layer)
+        w_ma = dict(w, W_o=np.zeros_like(w["W_o"]))
+        w_te = dict(w, W_out=np.zeros_like(w["W_out"]))
+        np.testing.assert_allclose(full, O.mate_forward(w["X"], w_ma, cfg, layer)
+                                   + O.mate_forward(w["X"], w_te, cfg, layer), rtol=1e-12, atol=1e-12)
+
+
+def test_ma_branch_without_prefix_is_scan_of_reordered_tokens():
+    # R = 0, D = 0, W_out = identity on d_inner = d: MA(X) = unpermute(bidir-scan(in_proj(permute(X))))
+    cfg = MateConfig("t", 1, 2, 4, 4, 8, 2, 4, 3, 8, 0, 1, 8, 2, 4, 4, 1, 2, 2, "f32", 0)
+    w = make_inputs(cfg)
+    w = dict(w, W_out=np.eye(8, dtype=np.float32), D=np.zeros(2, np.float32))
+    X3 = w["X"][0]
+    for order in range(4):
+        got = O.ma_branch(X3, w, cfg, order)
+        seq = O.rms_permute(X3, order).astype(np.float64) @ w["W_in"].astype(np.float64).T
+        x = seq[:, :8].reshape(-1, 2, 4)
+        Bm, Cm, dt = seq[:, 8:11], seq[:, 11:14], seq[:, 14:]
+        delta = np.log1p(np.exp(dt))
+        A = -np.exp(w["A_log"].astype(np.float64))
+        yf = O.ssd_recurrence(x, Bm, Cm, delta, A, np.zeros(2))
+        yb = O.ssd_recurrence(x[::-1], Bm[::-1], Cm[::-1], delta[::-1], A, np.zeros(2))[::-1]
+        expect = O.rms_unpermute((yf + yb).reshape(-1, 8), order, 2, 4, 4)
+        np.testing.assert_allclose(got, expect, rtol=1e-12, atol=1e-12)
+
+
+def test_config_shapes_are_consistent():
+    for cfg in CONFIGS.values():
+        assert cfg.T % cfg.wt == 0 and cfg.H % cfg.wh == 0 and cfg.W % cfg.ww == 0
+        O.review_grid(cfg.T, cfg.H, cfg.W, cfg.R)   # pool factors integral
+        assert 0 < cfg.st < cfg.wt and 0 < cfg.sh < cfg.wh and 0 < cfg.sw < cfg.ww
