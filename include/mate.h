@@ -1,0 +1,195 @@
+/*
+ * libmate: forward pass of the LinGen MATE token-mixing block on NVIDIA B200 (sm_100a).
+ *
+ * Method sources (the pages that describe it):
+ *   [ABS]  "Towards High-Resolution Minute-Length Text-to-Video Generation with Linear Computational
+ *          Complexity", abstract: MATE replaces DiT self-attention and consists of an MA branch (a
+ *          bidirectional Mamba2 block with Rotary Major Scan and review tokens) and a TE branch
+ *          (TEmporal Swin Attention).
+ *   [NEWS] LinGen news article (weiba1314.com / xihudo.com), section "方法：线性复杂度的 MATE 模块":
+ *          RMS unrolls the T x H x W grid with W, H, T as 1st/2nd/3rd priority and swaps priorities
+ *          between adjacent layers; TESA is 3D window attention with small fixed windows that slide
+ *          between layers; review tokens write an overview of the video tensor into the Mamba hidden
+ *          state ahead of the video.
+ *   [FEAT] "LinGen：基于Mamba机制的线性复杂度高清长视频生成框架", 关键算法创新: the four RMS modes
+ *          (spatial row / spatial column / temporal row / temporal column) and TESA's alternating
+ *          normal and shifted windows.
+ *
+ * Conventions for every entry point
+ *   - Tensors are DEVICE pointers owned by the caller, contiguous, channels-last, 16-byte aligned.
+ *     Element type follows cfg->dtype (bf16 or fp32) unless the argument says float.
+ *   - Calls are stream-ordered on `stream` and never synchronise; they never allocate or free device
+ *     memory.  Scratch memory is the caller's workspace `ws` of at least the queried size.
+ *   - Host-side validation happens before any launch; a rejected call launches nothing.
+ *   - Weight matrices use the out_features x in_features layout (row r = output feature r).
+ *   - Layer behaviour is a pure function of layer_idx: scan order layer_idx mod 4, Swin shift on odd
+ *     layers.
+ *   - The grid token (t, h, w) of sample b is row b*T*H*W + (t*H + h)*W + w of a [B, T, H, W, C]
+ *     tensor.
+ */
+#ifndef MATE_H_
+#define MATE_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MATE_API __attribute__((visibility("default")))
+#else
+#define MATE_API
+#endif
+
+/* Same object as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st* mate_stream_t;
+
+typedef enum {
+  MATE_OK = 0,
+  MATE_ERR_ARG = 1,         /* null pointer, misaligned pointer, order/layer out of range */
+  MATE_ERR_SHAPE = 2,       /* inconsistent sizes: window does not divide the grid, bad review count */
+  MATE_ERR_WORKSPACE = 3,   /* ws_bytes smaller than the queried workspace size */
+  MATE_ERR_CUDA = 4,        /* a CUDA launch or copy failed (cudaGetLastError after the launch) */
+  MATE_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (reported by mate_device_status) */
+  MATE_ERR_UNSUPPORTED = 6  /* valid shape that the bf16 tensor-core kernels do not cover */
+} mate_status;
+
+typedef enum { MATE_BF16 = 0, MATE_F32 = 1 } mate_dtype;
+
+/*
+ * Block shape.  B samples of a T x H x W latent grid with d channels; Mamba2 with nh heads of size P,
+ * state size N, chunk length Q and R review tokens; TESA with th heads of size tp, window
+ * (wt, wh, ww) and Swin shift (st, sh, sw) used on odd layers.
+ * Requirements: window divides the grid; 0 <= shift < window per axis; R = 16 * Tr with Tr dividing T
+ * and 4 dividing H and W (review tokens pool onto a Tr x 4 x 4 grid), R = 0 allowed; d, nh*P, th*tp
+ * multiples of 8 elements.
+ * bf16 tensor-core path additionally: d % 64 == 0, nh % 8 == 0, P == 64, N == 128, Q == 256,
+ * tp == 128, wt*wh*ww == 256.  fp32 path (CUDA-core kernels, for small blocks): P*N <= 1024, tp <= 128.
+ * B * (T*H*W + R) < 2^31.
+ */
+typedef struct {
+  int B, T, H, W, d;
+  int nh, P, N, Q, R;
+  int th, tp;
+  int wt, wh, ww;
+  int st, sh, sw;
+  mate_dtype dtype;
+} mate_config;
+
+/* Block weights, device pointers, caller-owned.  Element type cfg->dtype except the fp32 vectors. */
+typedef struct {
+  const void* W_in;     /* [nh*P + 2N + nh, d]: output features x (head h at h*P..) | B | C | dt      */
+  const float* dt_bias; /* [nh]   delta = softplus(dt + dt_bias)                                     */
+  const float* A_log;   /* [nh]   A = -exp(A_log)                                                    */
+  const float* D;       /* [nh]   skip weight                                                        */
+  const void* W_out;    /* [d, nh*P]  MA out-projection                                              */
+  const void* W_qkv;    /* [3*th*tp, d] output features q | k | v, head-major inside each            */
+  const void* W_o;      /* [d, th*tp]  TE out-projection                                             */
+} mate_weights;
+
+/* Human-readable name of a status code (static string). */
+MATE_API const char* mate_status_str(mate_status s);
+
+/* MATE_OK if cfg describes a block this library can run, else the reason (no device work). */
+MATE_API mate_status mate_check_config(const mate_config* cfg);
+
+/* Workspace bytes needed by mate_forward / mate_forward_host for this shape (0 if cfg is invalid). */
+MATE_API size_t mate_workspace_bytes(const mate_config* cfg);
+
+/* Workspace bytes needed by ssd_scan_bidir for this shape with `prefix_len` prefix rows. */
+MATE_API size_t mate_ssd_workspace_bytes(const mate_config* cfg, int prefix_len);
+
+/*
+ * Rotary Major Scan reorder ([NEWS] RMS paragraphs; [FEAT] RMS modes).
+ *   X  [B, T, H, W, d] -> Xp [B, T*H*W, d] with Xp[b, s_o(t,h,w)] = X[b, t, h, w], where the scan
+ *   position s_o unrolls the grid with the order's first-priority axis fastest:
+ *     order 0 (spatial row):     s = (t*H + h)*W + w     (W, H, T)
+ *     order 1 (spatial column):  s = (t*W + w)*H + h     (H, W, T)
+ *     order 2 (temporal row):    s = (h*W + w)*T + t     (T, W, H)
+ *     order 3 (temporal column): s = (w*H + h)*T + t     (T, H, W)
+ * Bit copy; X and Xp must not overlap.  MATE_ERR_ARG if order is not 0..3.
+ */
+MATE_API mate_status rms_permute(const void* X, void* Xp, int order, const mate_config* cfg, mate_stream_t stream);
+
+/* Inverse of rms_permute: X[b, t, h, w] = Xp[b, s_o(t,h,w)]. */
+MATE_API mate_status rms_unpermute(const void* Xp, void* X, int order, const mate_config* cfg, mate_stream_t stream);
+
+/*
+ * Review tokens ([NEWS] review-token paragraph: an overview of the video tensor, written into the
+ * Mamba hidden state before the video tokens).  Rv [B, R, d]: the average of X over each cell of the
+ * Tr x 4 x 4 pooling grid (cells of (T/Tr) x (H/4) x (W/4) tokens), listed in scan order `order` of
+ * that grid.  fp32 accumulation.  Does nothing when R == 0.
+ */
+MATE_API mate_status review_pool(const void* X, void* Rv, int order, const mate_config* cfg, mate_stream_t stream);
+
+/*
+ * Bidirectional Mamba2 selective scan ([ABS] "bidirectional Mamba2 block").  For each sample b the
+ * sequence S has L = prefix_len + T*H*W rows: prefix rows first, then the video rows.  Per head h
+ * (A_h = -exp(A_log[h]), delta = softplus(dt + dt_bias[h]), zero initial state):
+ *     h_t = exp(delta_t A_h) h_{t-1} + delta_t x_t B_t^T,    y_t = h_t C_t + D_h x_t
+ * is run over S (forward) and over [prefix rows; video rows reversed] (backward).  The output holds
+ * the video rows only: y = y_forward + (y_backward reversed back).
+ *   x  [B, L, nh*P]    Bm, Cm [B, L, N]    dt [B, L, nh] float (raw, before softplus)
+ *   dt_bias, A_log, D  [nh] float           y [B, T*H*W, nh*P]
+ * ws: at least mate_ssd_workspace_bytes(cfg, prefix_len) bytes.  cfg->R is ignored (prefix_len is
+ * used instead); prefix_len must satisfy 0 <= prefix_len.
+ */
+MATE_API mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const float* dt, const float* dt_bias,
+                           const float* A_log, const float* D, int prefix_len, void* y, const mate_config* cfg,
+                           void* ws, size_t ws_bytes, mate_stream_t stream);
+
+/*
+ * TEmporal Swin Attention ([NEWS] TESA paragraph; [FEAT] TESA): window attention on qkv
+ * [B, T, H, W, 3*th*tp] (q | k | v, head-major) -> O [B, T, H, W, th*tp].  shifted == 0: windows
+ * (wt, wh, ww) tile the grid.  shifted != 0: the grid is rolled by -(st, sh, sw) before tiling and
+ * rolled back after; keys that wrapped around an axis and keys that did not are masked from each other.
+ * Per window and head: softmax(q k^T / sqrt(tp)) v with fp32 softmax.
+ */
+MATE_API mate_status tesa_forward(const void* qkv, void* O, int shifted, const mate_config* cfg, mate_stream_t stream);
+
+/*
+ * Tensor-core projection used by the block's in/out maps: C[M, N] = A[M, K] W[N, K]^T in bf16 with
+ * fp32 accumulation (row strides lda, ldw, ldc in elements, multiples of 8; K a multiple of 64).
+ * bf16 only (cfg is not needed); MATE_ERR_UNSUPPORTED otherwise.
+ */
+MATE_API mate_status mate_project_bf16(const void* A, int lda, long long M, int K, const void* Wt, int ldw, int N,
+                                       void* C, int ldc, mate_stream_t stream);
+
+/*
+ * The MATE block: Out = MA(X) + TE(X) for X, Out [B, T, H, W, d] (may not alias).  Layer layer_idx >= 0
+ * selects scan order layer_idx mod 4 and the Swin shift on odd layers.
+ *   MA: review tokens (pooled from X, in scan order) prefixed to the scanned sequence; in-projection
+ *       W_in; bidirectional scan; out-projection W_out of the video rows; back to grid order.
+ *   TE: qkv = X W_qkv^T; tesa; projection W_o.
+ * ws: at least mate_workspace_bytes(cfg) bytes (caller-owned, no alignment beyond 256 bytes needed).
+ */
+MATE_API mate_status mate_forward(const void* X, const mate_weights* w, int layer_idx, void* Out, const mate_config* cfg,
+                         void* ws, size_t ws_bytes, mate_stream_t stream);
+
+/*
+ * mate_forward with HOST input and output: copies X_host (B*T*H*W*d elements) to the device part of
+ * the workspace, runs the block and copies Out back to Out_host, all on `stream` (page-locked host
+ * buffers give full-speed asynchronous copies).  The host buffers must stay valid until the stream
+ * reaches the end of the call.  ws: at least mate_workspace_bytes(cfg) + 2 * B*T*H*W*d*elem bytes.
+ */
+MATE_API mate_status mate_forward_host(const void* X_host, const mate_weights* w, int layer_idx, void* Out_host,
+                              const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream);
+
+/* Workspace bytes needed by mate_forward_host. */
+MATE_API size_t mate_forward_host_workspace_bytes(const mate_config* cfg);
+
+/*
+ * Reads and clears the device status word that kernels set when a bounded wait runs out.  Synchronises
+ * `stream` first.  *flags receives the raw bits (1 = wait timed out); returns MATE_ERR_TIMEOUT if any
+ * bit was set, MATE_OK otherwise.
+ */
+MATE_API mate_status mate_device_status(mate_stream_t stream, unsigned int* flags);
+
+/* Number of kernel launches the last successful mate_forward call issued on this thread. */
+MATE_API int mate_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MATE_H_ */

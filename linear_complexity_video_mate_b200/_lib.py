@@ -1,0 +1,90 @@
+"""ctypes declarations of the C ABI in include/mate.h (argument marshalling only)."""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmate.so")
+
+MATE_OK, MATE_ERR_ARG, MATE_ERR_SHAPE, MATE_ERR_WORKSPACE, MATE_ERR_CUDA, MATE_ERR_TIMEOUT, MATE_ERR_UNSUPPORTED = range(7)
+MATE_BF16, MATE_F32 = 0, 1
+
+# every symbol include/mate.h declares
+EXPORTS = (
+    "mate_status_str", "mate_check_config", "mate_workspace_bytes", "mate_ssd_workspace_bytes", "rms_permute",
+    "rms_unpermute", "review_pool", "ssd_scan_bidir", "tesa_forward", "mate_forward", "mate_forward_host",
+    "mate_forward_host_workspace_bytes", "mate_device_status", "mate_last_launch_count", "mate_project_bf16",
+)
+
+_CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp", "wt", "wh", "ww", "st", "sh", "sw")
+
+
+class CConfig(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int) for f in _CONFIG_FIELDS] + [("dtype", ctypes.c_int)]
+
+
+class CWeights(ctypes.Structure):
+    _fields_ = [("W_in", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
+                ("D", ctypes.c_void_p), ("W_out", ctypes.c_void_p), ("W_qkv", ctypes.c_void_p),
+                ("W_o", ctypes.c_void_p)]
+
+
+class MateError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+
+
+_lib = None
+
+
+def load():
+    """Load libmate.so from the package directory; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmate.so is not built ({LIB_PATH}); run linear_complexity_video_mate_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    cfgp, wp = ctypes.POINTER(CConfig), ctypes.POINTER(CWeights)
+    sigs = {
+        "mate_status_str": (ctypes.c_char_p, [ci]),
+        "mate_check_config": (ci, [cfgp]),
+        "mate_workspace_bytes": (sz, [cfgp]),
+        "mate_ssd_workspace_bytes": (sz, [cfgp, ci]),
+        "rms_permute": (ci, [vp, vp, ci, cfgp, vp]),
+        "rms_unpermute": (ci, [vp, vp, ci, cfgp, vp]),
+        "review_pool": (ci, [vp, vp, ci, cfgp, vp]),
+        "ssd_scan_bidir": (ci, [vp, vp, vp, vp, vp, vp, vp, ci, vp, cfgp, vp, sz, vp]),
+        "tesa_forward": (ci, [vp, vp, ci, cfgp, vp]),
+        "mate_forward": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
+        "mate_forward_host": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
+        "mate_forward_host_workspace_bytes": (sz, [cfgp]),
+        "mate_device_status": (ci, [vp, ctypes.POINTER(ctypes.c_uint)]),
+        "mate_last_launch_count": (ci, []),
+        "mate_project_bf16": (ci, [vp, ci, ctypes.c_longlong, ci, vp, ci, ci, vp, ci, vp]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_str(status: int) -> str:
+    return load().mate_status_str(int(status)).decode()
+
+
+def check(status: int, where: str):
+    if status != MATE_OK:
+        raise MateError(status, where)
+
+
+def make_config(cfg) -> CConfig:
+    """C config from any object with the block's shape attributes (e.g. mate_inputs.MateConfig)."""
+    c = CConfig()
+    for f in _CONFIG_FIELDS:
+        setattr(c, f, int(getattr(cfg, f)))
+    c.dtype = MATE_BF16 if cfg.dtype == "bf16" else MATE_F32
+    return c

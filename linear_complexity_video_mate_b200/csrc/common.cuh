@@ -1,0 +1,265 @@
+// Device-side building blocks shared by the MATE kernels (sm_100a only).
+//
+//  * scan-order index arithmetic of the Rotary Major Scan (LinGen news article, method section, RMS
+//    paragraphs; "LinGen：基于Mamba机制的线性复杂度高清长视频生成框架", 关键算法创新 / RMS);
+//  * mbarrier waits with an iteration limit (a wait that runs out records MATE_DEV_TIMEOUT in the device
+//    status word and lets the kernel finish instead of hanging the GPU);
+//  * TMA tiled loads, tcgen05 MMA / TMEM helpers and the shared-memory matrix descriptors.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mate {
+
+// ---------------------------------------------------------------------------------------------------
+// Device status word: bit flags OR-ed in by kernels, read and cleared by the host (mate_device_status).
+// ---------------------------------------------------------------------------------------------------
+enum : unsigned { MATE_DEV_TIMEOUT = 1u, MATE_DEV_BAD_ARG = 2u };
+// Defined here: the whole library is one translation unit.
+__device__ unsigned int g_dev_status = 0;
+
+__device__ __forceinline__ void flag_status(unsigned f) { atomicOr(&g_dev_status, f); }
+
+// ---------------------------------------------------------------------------------------------------
+// Rotary Major Scan index maps.  Order o lists the grid axes fastest-varying first:
+//   0: (W, H, T)  1: (H, W, T)  2: (T, W, H)  3: (T, H, W).
+// scan_to_raster(q) gives the raster index (t*H + h)*W + w of the token at scan position q.
+// ---------------------------------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int scan_to_raster(int q, int T, int H, int W, int order) {
+  int t, h, w;
+  switch (order) {
+    case 0: return q;
+    case 1: h = q % H; q /= H; w = q % W; t = q / W; break;
+    case 2: t = q % T; q /= T; w = q % W; h = q / W; break;
+    default: t = q % T; q /= T; h = q % H; w = q / H; break;
+  }
+  return (t * H + h) * W + w;
+}
+
+__host__ __device__ __forceinline__ int raster_to_scan(int r, int T, int H, int W, int order) {
+  int w = r % W, h = (r / W) % H, t = r / (W * H);
+  switch (order) {
+    case 0: return r;
+    case 1: return (t * W + w) * H + h;
+    case 2: return (h * W + w) * T + t;
+    default: return (w * H + h) * T + t;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------------
+// Small conversions
+// ---------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(v);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------------------------------
+// mbarrier
+// ---------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Upper bound on polls of one wait: each failed try_wait suspends the thread for a hardware-defined
+// time slice, so this bounds a stuck wait to well under a few seconds.
+constexpr unsigned kMaxPolls = 1u << 22;
+
+// Wait for the phase with the given parity to complete.  Returns false (and flags the device status)
+// if the limit is reached; callers then skip the dependent work and run to the end of the kernel.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  for (unsigned i = 0; i < kMaxPolls; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (i > 64) __nanosleep(64);
+  }
+  flag_status(MATE_DEV_TIMEOUT);
+  return false;
+}
+
+// ---------------------------------------------------------------------------------------------------
+// TMA (tiled tensor copies global -> shared, completion through an mbarrier transaction count)
+// ---------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------------------------------------------
+// Async copies (16 bytes) used to gather rows that TMA boxes cannot describe (scan-order and window
+// gathers).  Writes land in shared memory through the generic proxy: fence_proxy_async() must follow
+// before a tcgen05.mma reads them.
+// ---------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------------------
+// tcgen05: tensor memory allocation, MMA issue, commit, loads and fences
+// ---------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, unsigned ncols) {  // whole warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {  // whole warp
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, unsigned ncols) {  // whole warp
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulation.  One thread issues.
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+
+// Arrive on `bar` once all tcgen05 operations issued so far by this thread have completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// Warp-collective load of 32 lanes x 32 consecutive 32-bit columns (lane = TMEM lane of this warp's
+// quadrant); result in r[0..31] after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------------------
+// Shared-memory matrix descriptors (tcgen05 "version 1" descriptors), 128-byte swizzle.
+//
+// K-major operand (rows = M or N, 64 bf16 of K per 128-byte row): rows are 128 bytes apart, groups of
+// 8 rows (one 1024-byte swizzle atom) are `sbo` bytes apart; the 16-byte chunk index of each row is
+// XOR-ed with (row mod 8).  Stepping K by 16 elements inside the 128-byte row adds 32 bytes to the
+// start address.
+//
+// MN-major operand (64 bf16 of M/N per 128-byte row, one row per K index): K rows 128 bytes apart,
+// groups of 8 K rows `sbo` bytes apart, consecutive 64-element M/N blocks `lbo` bytes apart, same
+// chunk swizzle with (K row mod 8).
+// ---------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;  // descriptor version for sm_100
+  d |= 2ull << 61;  // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, dense, M x N tile, operand majors (0 = K, 1 = MN).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4)                                   // accumulator fp32
+         | (1u << 7)                                 // A bf16
+         | (1u << 10)                                // B bf16
+         | (static_cast<uint32_t>(a_mn_major) << 15)  // A major
+         | (static_cast<uint32_t>(b_mn_major) << 16)  // B major
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+// Byte offset of element (row, col) inside a K-major 128B-swizzled tile whose 64-column K blocks are
+// `kblock_bytes` apart (rows of one block are dense: 8-row groups 1024 bytes apart).  2-byte elements.
+__host__ __device__ __forceinline__ uint32_t sw128_kmajor_offset(int row, int col, uint32_t kblock_bytes) {
+  int kb = col >> 6;
+  int c = col & 63;
+  int chunk = (c >> 3) ^ (row & 7);
+  return kb * kblock_bytes + (row >> 3) * 1024 + (row & 7) * 128 + chunk * 16 + (c & 7) * 2;
+}
+
+// Byte offset of element (k, mn) inside an MN-major 128B-swizzled tile: MN blocks of 64 elements are
+// `mnblock_bytes` apart; inside a block the K rows are dense (8-row groups 1024 bytes apart).
+__host__ __device__ __forceinline__ uint32_t sw128_mnmajor_offset(int k, int mn, uint32_t mnblock_bytes) {
+  int mb = mn >> 6;
+  int c = mn & 63;
+  int chunk = (c >> 3) ^ (k & 7);
+  return mb * mnblock_bytes + (k >> 3) * 1024 + (k & 7) * 128 + chunk * 16 + (c & 7) * 2;
+}
+
+}  // namespace mate

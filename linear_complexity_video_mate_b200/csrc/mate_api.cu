@@ -1,0 +1,608 @@
+// libmate: host side of the C ABI declared in include/mate.h.  Validates arguments, plans the caller's
+// workspace, builds TMA descriptors and launches the kernels of the MATE block on the caller's stream.
+// One translation unit holds every kernel, so the device status word is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/mate.h"
+#include "common.cuh"
+#include "gemm_bf16.cuh"
+#include "simt.cuh"
+#include "ssd_bf16.cuh"
+#include "tesa_bf16.cuh"
+
+using namespace mate;
+
+namespace {
+
+thread_local int t_launches = 0;
+
+#define MATE_LAUNCH_CHECK()                         \
+  do {                                              \
+    ++t_launches;                                   \
+    if (cudaPeekAtLastError() != cudaSuccess) {     \
+      (void)cudaGetLastError();                     \
+      return MATE_ERR_CUDA;                         \
+    }                                               \
+  } while (0)
+
+#define MATE_TRY(expr)                 \
+  do {                                 \
+    mate_status _s = (expr);           \
+    if (_s != MATE_OK) return _s;      \
+  } while (0)
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kSmemLimit = 232448;  // opt-in dynamic shared memory per block on sm_100
+
+int device_sms() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
+         cudaSuccess;
+}
+
+// ------------------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 matrix [rows, cols] with row stride ld (elements); box = box_rows x 64 columns, 128B swizzle.
+bool make_tmap(CUtensorMap* m, const void* ptr, long long rows, long long cols, long long ld, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------------------ validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(const mate_config* c) { return c->dtype == MATE_BF16 ? 2 : 4; }
+
+mate_status check_config(const mate_config* c) {
+  if (c == nullptr) return MATE_ERR_ARG;
+  if (c->dtype != MATE_BF16 && c->dtype != MATE_F32) return MATE_ERR_ARG;
+  if (c->B <= 0 || c->T <= 0 || c->H <= 0 || c->W <= 0 || c->d <= 0 || c->nh <= 0 || c->P <= 0 || c->N <= 0 ||
+      c->Q <= 0 || c->R < 0 || c->th <= 0 || c->tp <= 0 || c->wt <= 0 || c->wh <= 0 || c->ww <= 0)
+    return MATE_ERR_SHAPE;
+  if (c->T % c->wt || c->H % c->wh || c->W % c->ww) return MATE_ERR_SHAPE;
+  if (c->st < 0 || c->sh < 0 || c->sw < 0 || c->st >= c->wt || c->sh >= c->wh || c->sw >= c->ww) return MATE_ERR_SHAPE;
+  if (c->R % 16) return MATE_ERR_SHAPE;
+  if (c->R > 0) {
+    const int Tr = c->R / 16;
+    if (c->T % Tr || c->H % 4 || c->W % 4) return MATE_ERR_SHAPE;
+  }
+  const long long n = (long long)c->T * c->H * c->W;
+  if ((long long)c->B * (n + c->R) >= (1LL << 31)) return MATE_ERR_SHAPE;
+  const size_t es = elem_size(c);
+  if ((c->d * es) % 16 || (c->nh * c->P * es) % 16 || (c->th * c->tp * es) % 16 || (c->N * es) % 16)
+    return MATE_ERR_SHAPE;
+  if (c->dtype == MATE_BF16) {
+    if (c->d % 64 || c->P != kSsdP || c->N != kSsdN || c->Q != kSsdQ || c->tp != 128 ||
+        c->wt * c->wh * c->ww != 256 || c->nh % 8)
+      return MATE_ERR_UNSUPPORTED;
+  } else {
+    if (c->P * c->N > 1024 || c->tp > 128) return MATE_ERR_UNSUPPORTED;
+  }
+  return MATE_OK;
+}
+
+// ------------------------------------------------------------------------------ workspace plans
+struct Carver {
+  char* base;
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+struct SsdScratch {
+  __nv_bfloat16 *Gm, *Sf, *Sb, *Hf, *Hb;
+  float *gl, *Gd;
+};
+
+int ceil_div(long long a, int b) { return static_cast<int>((a + b - 1) / b); }
+
+SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh) {
+  SsdScratch s;
+  const int nRc = ceil_div(R, kSsdQ), nVc = ceil_div(n, kSsdQ);
+  const size_t PN = (size_t)kSsdP * kSsdN;
+  s.Gm = cv.take<__nv_bfloat16>((size_t)B * nVc * kSsdQ * kSsdQ);
+  s.Sf = cv.take<__nv_bfloat16>((size_t)B * (nRc + nVc) * nh * PN);
+  s.Sb = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
+  s.Hf = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
+  s.Hb = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
+  s.gl = cv.take<float>((size_t)B * (nRc + nVc) * nh);
+  s.Gd = cv.take<float>((size_t)B * nVc * kSsdQ);
+  return s;
+}
+
+struct ForwardPlan {
+  int NIn, NI, KO;
+  void *Wi, *Wo, *Rv, *Zv, *Zr, *YO;
+  float *Dv, *Dr;
+  SsdScratch ssd;
+  size_t bytes;
+};
+
+ForwardPlan plan_forward(const mate_config* c, void* ws) {
+  ForwardPlan p;
+  Carver cv{static_cast<char*>(ws)};
+  const size_t es = elem_size(c);
+  const long long n = (long long)c->T * c->H * c->W;
+  p.NIn = c->nh * c->P + 2 * c->N + c->nh;
+  p.NI = p.NIn + 3 * c->th * c->tp;
+  p.KO = c->nh * c->P + c->th * c->tp;
+  p.Wi = cv.take<char>((size_t)p.NI * c->d * es);
+  p.Wo = cv.take<char>((size_t)c->d * p.KO * es);
+  p.Rv = cv.take<char>((size_t)c->B * c->R * c->d * es);
+  p.Zv = cv.take<char>((size_t)c->B * n * p.NI * es);
+  p.Zr = cv.take<char>((size_t)c->B * c->R * p.NI * es);
+  p.Dv = cv.take<float>((size_t)c->B * n * c->nh);
+  p.Dr = cv.take<float>((size_t)c->B * c->R * c->nh);
+  p.YO = cv.take<char>((size_t)c->B * n * p.KO * es);
+  if (c->dtype == MATE_BF16) p.ssd = carve_ssd(cv, c->B, n, c->R, c->nh);
+  else p.ssd = SsdScratch{};
+  p.bytes = cv.off + 256;
+  return p;
+}
+
+size_t ssd_ws_bytes(const mate_config* c, int prefix_len, float** delta, SsdScratch* s, void* ws) {
+  Carver cv{static_cast<char*>(ws)};
+  const long long n = (long long)c->T * c->H * c->W;
+  float* d = cv.take<float>((size_t)c->B * (n + prefix_len) * c->nh);
+  if (delta) *delta = d;
+  SsdScratch sc = c->dtype == MATE_BF16 ? carve_ssd(cv, c->B, n, prefix_len, c->nh) : SsdScratch{};
+  if (s) *s = sc;
+  return cv.off + 256;
+}
+
+// ------------------------------------------------------------------------------ launchers
+int choose_bn(int N) {
+  int best = 256;
+  long long best_cost = -1;
+  for (int bn = 256; bn >= 128; bn -= 16) {
+    const long long cost = (long long)ceil_div(N, bn) * (bn + 64);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+mate_status gemm_bf16(const void* A, int lda, long long M, int K, const void* Bw, int ldb, int N, void* C, int ldc,
+                      float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias, cudaStream_t st) {
+  if (M <= 0) return MATE_OK;
+  if (K % kGemmBK) return MATE_ERR_UNSUPPORTED;
+  GemmParams p;
+  p.M = static_cast<int>(M);
+  p.N = N;
+  p.K = K;
+  p.bn = choose_bn(N);
+  p.num_n_tiles = ceil_div(N, p.bn);
+  p.num_tiles = ceil_div(M, kGemmBM) * p.num_n_tiles;
+  const uint32_t sb = gemm_stage_bytes(p.bn);
+  p.stages = std::min<int>(8, static_cast<int>((kSmemLimit - 1024 - 256) / sb));
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.ldc = ldc;
+  p.delta = delta;
+  p.ld_delta = ld_delta;
+  p.dt_col0 = dt_col0;
+  p.dt_cols = dt_cols;
+  p.dt_bias = dt_bias;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, A, M, K, lda, kGemmBM) || !make_tmap(&tb, Bw, N, K, ldb, p.bn)) return MATE_ERR_CUDA;
+  const size_t smem = 1024 + (size_t)p.stages * sb + 256;
+  if (!set_smem(gemm_bf16_tc_kernel, smem)) return MATE_ERR_CUDA;
+  const int grid = std::min(p.num_tiles, device_sms());
+  gemm_bf16_tc_kernel<<<grid, kGemmThreads, smem, st>>>(ta, tb, p);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
+mate_status gemm_f32(const float* A, int lda, long long M, int K, const float* Bw, int ldb, int N, float* C, int ldc,
+                     float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias, cudaStream_t st) {
+  if (M <= 0) return MATE_OK;
+  dim3 grid(ceil_div(N, 64), ceil_div(M, 64));
+  gemm_f32_kernel<<<grid, 256, 0, st>>>(A, lda, Bw, ldb, C, ldc, static_cast<int>(M), N, K, delta, ld_delta, dt_col0,
+                                        dt_cols, dt_bias);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
+mate_status gather_rows(const void* src, void* dst, const mate_config* c, int order, int inverse, cudaStream_t st) {
+  const long long n = (long long)c->T * c->H * c->W;
+  const int vec = static_cast<int>(c->d * elem_size(c) / 16);
+  const long long rows = (long long)c->B * n;
+  const int blocks = static_cast<int>(std::min<long long>((rows + 7) / 8, (long long)device_sms() * 16));
+  rms_gather_rows_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows,
+                                                 static_cast<int>(n), vec, c->T, c->H, c->W, order, inverse);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
+mate_status pool(const void* X, void* Rv, const mate_config* c, int order, cudaStream_t st) {
+  if (c->R == 0) return MATE_OK;
+  const int per = 16 / static_cast<int>(elem_size(c));
+  const int threads = std::min(256, std::max(32, ((c->d / per) + 31) / 32 * 32));
+  dim3 grid(c->R, c->B);
+  if (c->dtype == MATE_BF16)
+    review_pool_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(X),
+                                                                static_cast<__nv_bfloat16*>(Rv), c->R, c->T, c->H,
+                                                                c->W, c->d, order);
+  else
+    review_pool_kernel<float><<<grid, threads, 0, st>>>(static_cast<const float*>(X), static_cast<float*>(Rv), c->R,
+                                                        c->T, c->H, c->W, c->d, order);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
+mate_status copy_block(const void* src, void* dst, int rows, int cols, int ld_dst, int row0, int col0, size_t es,
+                       cudaStream_t st) {
+  const int vcols = static_cast<int>(cols * es / 16);
+  const long long total = (long long)rows * vcols;
+  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4096));
+  copy_block_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows, vcols,
+                                            static_cast<int>(ld_dst * es / 16), row0, static_cast<int>(col0 * es / 16));
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
+// Scan over sequences described by `rows`; y row = b*y_bstride + map(q), ldy.  bf16 or fp32 path.
+mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_log, const float* Dp, void* y, int ldy,
+                    long long y_bstride, const SsdScratch& sc, cudaStream_t st) {
+  const long long n = (long long)c->T * c->H * c->W;
+  if (c->dtype == MATE_F32) {
+    const int threads = ((c->P * c->N) + 31) / 32 * 32;
+    ssd_f32_kernel<<<dim3(c->nh, c->B), threads, c->P * c->N * sizeof(float), st>>>(
+        rows, A_log, Dp, c->P, c->N, static_cast<float*>(y), ldy, y_bstride);
+    MATE_LAUNCH_CHECK();
+    return MATE_OK;
+  }
+  SsdBf16Params p;
+  p.s = rows;
+  p.B = c->B;
+  p.nh = c->nh;
+  p.nRc = ceil_div(rows.R, kSsdQ);
+  p.nVc = ceil_div(n, kSsdQ);
+  p.A_log = A_log;
+  p.Dp = Dp;
+  p.Gm = sc.Gm;
+  p.Sf = sc.Sf;
+  p.Sb = sc.Sb;
+  p.gl = sc.gl;
+  p.Gd = sc.Gd;
+  p.Hf = sc.Hf;
+  p.Hb = sc.Hb;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.ldy = ldy;
+  p.y_bstride = y_bstride;
+  const size_t smem_gram = 1024 + 98304 + 64;
+  const size_t smem_state = 1024 + 131072 + 2048 + 64 + 64;
+  const size_t smem_out = 1024 + 196608 + 3072 + 64 + 64;
+  if (!set_smem(ssd_gram_kernel, smem_gram) || !set_smem(ssd_state_kernel, smem_state) ||
+      !set_smem(ssd_output_kernel, smem_out))
+    return MATE_ERR_CUDA;
+  ssd_gram_kernel<<<dim3(p.nVc, c->B, 2), 128, smem_gram, st>>>(p);
+  MATE_LAUNCH_CHECK();
+  int hpc = 1;
+  while (hpc < 4 && c->nh % (hpc * 2) == 0) hpc *= 2;
+  ssd_state_kernel<<<dim3(p.nRc + p.nVc, c->B, c->nh / hpc), 256, smem_state, st>>>(p, hpc);
+  MATE_LAUNCH_CHECK();
+  ssd_carry_kernel<<<dim3(kSsdP * kSsdN / 8 / 128, c->nh, 2 * c->B), 128, 0, st>>>(p);
+  MATE_LAUNCH_CHECK();
+  ssd_output_kernel<<<dim3(p.nVc, c->B, c->nh), 256, smem_out, st>>>(p);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
+mate_status run_tesa(const mate_config* c, const void* qkv, int ldq, int qcol, int kcol, int vcol, void* O, int ldo,
+                     int ocol, int shifted, cudaStream_t st) {
+  const int sft = shifted ? 1 : 0;
+  if (c->dtype == MATE_F32) {
+    const long long n = (long long)c->T * c->H * c->W;
+    const long long warps = n * c->th;
+    dim3 grid(static_cast<unsigned>((warps + 7) / 8), c->B);
+    tesa_f32_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(qkv), ldq, qcol, kcol, vcol,
+                                          static_cast<float*>(O), ldo, ocol, c->T, c->H, c->W, c->th, c->tp, c->wt,
+                                          c->wh, c->ww, c->st, c->sh, c->sw, sft);
+    MATE_LAUNCH_CHECK();
+    return MATE_OK;
+  }
+  TesaBf16Params p;
+  p.qkv = static_cast<const __nv_bfloat16*>(qkv);
+  p.ldq = ldq;
+  p.qcol = qcol;
+  p.kcol = kcol;
+  p.vcol = vcol;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.ldo = ldo;
+  p.ocol = ocol;
+  p.T = c->T;
+  p.H = c->H;
+  p.W = c->W;
+  p.th = c->th;
+  p.wt = c->wt;
+  p.wh = c->wh;
+  p.ww = c->ww;
+  p.st = sft ? c->st : 0;
+  p.sh = sft ? c->sh : 0;
+  p.sw = sft ? c->sw : 0;
+  p.shifted = sft;
+  p.scale_log2 = 1.4426950408889634f / std::sqrt(static_cast<float>(c->tp));
+  const size_t smem = 1024 + 196608 + 2048 + 1024 + 64;
+  if (!set_smem(tesa_bf16_kernel, smem)) return MATE_ERR_CUDA;
+  const int nwin = (c->T / c->wt) * (c->H / c->wh) * (c->W / c->ww);
+  tesa_bf16_kernel<<<dim3(nwin, c->B, c->th), 256, smem, st>>>(p);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
+mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, void* Out, const mate_config* c,
+                         void* ws, size_t ws_bytes, cudaStream_t st) {
+  MATE_TRY(check_config(c));
+  if (X == nullptr || w == nullptr || Out == nullptr || ws == nullptr || layer_idx < 0) return MATE_ERR_ARG;
+  if (w->W_in == nullptr || w->dt_bias == nullptr || w->A_log == nullptr || w->D == nullptr || w->W_out == nullptr ||
+      w->W_qkv == nullptr || w->W_o == nullptr)
+    return MATE_ERR_ARG;
+  if (!aligned16(X) || !aligned16(Out) || !aligned16(ws) || !aligned16(w->W_in) || !aligned16(w->W_out) ||
+      !aligned16(w->W_qkv) || !aligned16(w->W_o))
+    return MATE_ERR_ARG;
+  ForwardPlan pl = plan_forward(c, nullptr);
+  if (ws_bytes < pl.bytes) return MATE_ERR_WORKSPACE;
+  pl = plan_forward(c, ws);
+  const int order = layer_idx % 4;
+  const int shifted = layer_idx % 2;
+  const size_t es = elem_size(c);
+  const long long n = (long long)c->T * c->H * c->W;
+  const long long Mv = (long long)c->B * n, Mr = (long long)c->B * c->R;
+  const int dI = c->nh * c->P;
+  const int NIn = pl.NIn, NI = pl.NI, KO = pl.KO;
+  const int dt0 = dI + 2 * c->N;
+
+  // packed weights: Wi = [W_in; W_qkv] (NI x d), Wo = [W_out | W_o] (d x KO)
+  MATE_TRY(copy_block(w->W_in, pl.Wi, NIn, c->d, c->d, 0, 0, es, st));
+  MATE_TRY(copy_block(w->W_qkv, pl.Wi, 3 * c->th * c->tp, c->d, c->d, NIn, 0, es, st));
+  MATE_TRY(copy_block(w->W_out, pl.Wo, c->d, dI, KO, 0, 0, es, st));
+  MATE_TRY(copy_block(w->W_o, pl.Wo, c->d, c->th * c->tp, KO, 0, dI, es, st));
+  // review tokens, then the projections of the video rows (grid order) and of the review rows
+  MATE_TRY(pool(X, pl.Rv, c, order, st));
+  if (c->dtype == MATE_BF16) {
+    MATE_TRY(gemm_bf16(X, c->d, Mv, c->d, pl.Wi, c->d, NI, pl.Zv, NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
+    MATE_TRY(gemm_bf16(pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
+  } else {
+    MATE_TRY(gemm_f32(static_cast<const float*>(X), c->d, Mv, c->d, static_cast<const float*>(pl.Wi), c->d, NI,
+                      static_cast<float*>(pl.Zv), NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
+    MATE_TRY(gemm_f32(static_cast<const float*>(pl.Rv), c->d, Mr, c->d, static_cast<const float*>(pl.Wi), c->d, NIn,
+                      static_cast<float*>(pl.Zr), NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
+  }
+  // MA: scan over [review rows; video rows in scan order], y written at grid-order rows of YO[:, :dI]
+  SeqRows rows;
+  const char* zv = static_cast<const char*>(pl.Zv);
+  const char* zr = static_cast<const char*>(pl.Zr);
+  rows.xv = zv;
+  rows.bv = zv + (size_t)dI * es;
+  rows.cv = zv + (size_t)(dI + c->N) * es;
+  rows.dv = pl.Dv;
+  rows.xr = zr;
+  rows.br = zr + (size_t)dI * es;
+  rows.cr = zr + (size_t)(dI + c->N) * es;
+  rows.dr = pl.Dr;
+  rows.ldxv = rows.ldbv = rows.ldcv = NI;
+  rows.ldxr = rows.ldbr = rows.ldcr = NI;
+  rows.lddv = rows.lddr = c->nh;
+  rows.v_bstride = n;
+  rows.v_off = 0;
+  rows.r_bstride = c->R;
+  rows.r_off = 0;
+  rows.n = static_cast<int>(n);
+  rows.R = c->R;
+  rows.T = c->T;
+  rows.H = c->H;
+  rows.W = c->W;
+  rows.order = order;
+  MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.YO, KO, n, pl.ssd, st));
+  // TE: window attention on the q | k | v columns of Zv, output into YO[:, dI:]
+  const int qc = NIn, ac = c->th * c->tp;
+  MATE_TRY(run_tesa(c, pl.Zv, NI, qc, qc + ac, qc + 2 * ac, pl.YO, KO, dI, shifted, st));
+  // Out = [y | O] [W_out | W_o]^T = MA + TE
+  if (c->dtype == MATE_BF16)
+    MATE_TRY(gemm_bf16(pl.YO, KO, Mv, KO, pl.Wo, KO, c->d, Out, c->d, nullptr, 0, 0, 0, nullptr, st));
+  else
+    MATE_TRY(gemm_f32(static_cast<const float*>(pl.YO), KO, Mv, KO, static_cast<const float*>(pl.Wo), KO, c->d,
+                      static_cast<float*>(Out), c->d, nullptr, 0, 0, 0, nullptr, st));
+  return MATE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mate_status_str(mate_status s) {
+  switch (s) {
+    case MATE_OK: return "ok";
+    case MATE_ERR_ARG: return "invalid argument";
+    case MATE_ERR_SHAPE: return "inconsistent shape";
+    case MATE_ERR_WORKSPACE: return "workspace too small";
+    case MATE_ERR_CUDA: return "CUDA error";
+    case MATE_ERR_TIMEOUT: return "device wait timed out";
+    case MATE_ERR_UNSUPPORTED: return "shape not supported by the tensor-core kernels";
+  }
+  return "unknown status";
+}
+
+mate_status mate_check_config(const mate_config* cfg) { return check_config(cfg); }
+
+size_t mate_workspace_bytes(const mate_config* cfg) {
+  if (check_config(cfg) != MATE_OK) return 0;
+  return plan_forward(cfg, nullptr).bytes;
+}
+
+size_t mate_ssd_workspace_bytes(const mate_config* cfg, int prefix_len) {
+  if (check_config(cfg) != MATE_OK || prefix_len < 0) return 0;
+  return ssd_ws_bytes(cfg, prefix_len, nullptr, nullptr, nullptr);
+}
+
+size_t mate_forward_host_workspace_bytes(const mate_config* cfg) {
+  if (check_config(cfg) != MATE_OK) return 0;
+  const size_t xb = (size_t)cfg->B * cfg->T * cfg->H * cfg->W * cfg->d * elem_size(cfg);
+  return mate_workspace_bytes(cfg) + 2 * ((xb + 255) & ~size_t(255));
+}
+
+mate_status rms_permute(const void* X, void* Xp, int order, const mate_config* cfg, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (X == nullptr || Xp == nullptr || order < 0 || order > 3 || !aligned16(X) || !aligned16(Xp)) return MATE_ERR_ARG;
+  t_launches = 0;
+  return gather_rows(X, Xp, cfg, order, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mate_status rms_unpermute(const void* Xp, void* X, int order, const mate_config* cfg, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (X == nullptr || Xp == nullptr || order < 0 || order > 3 || !aligned16(X) || !aligned16(Xp)) return MATE_ERR_ARG;
+  t_launches = 0;
+  return gather_rows(Xp, X, cfg, order, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mate_status review_pool(const void* X, void* Rv, int order, const mate_config* cfg, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (X == nullptr || (Rv == nullptr && cfg->R > 0) || order < 0 || order > 3 || !aligned16(X) || !aligned16(Rv))
+    return MATE_ERR_ARG;
+  t_launches = 0;
+  return pool(X, Rv, cfg, order, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const float* dt, const float* dt_bias,
+                           const float* A_log, const float* D, int prefix_len, void* y, const mate_config* cfg,
+                           void* ws, size_t ws_bytes, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (x == nullptr || Bm == nullptr || Cm == nullptr || dt == nullptr || dt_bias == nullptr || A_log == nullptr ||
+      D == nullptr || y == nullptr || ws == nullptr || prefix_len < 0)
+    return MATE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(y) || !aligned16(ws)) return MATE_ERR_ARG;
+  if (ws_bytes < ssd_ws_bytes(cfg, prefix_len, nullptr, nullptr, nullptr)) return MATE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  float* delta = nullptr;
+  SsdScratch sc;
+  ssd_ws_bytes(cfg, prefix_len, &delta, &sc, ws);
+  const long long n = (long long)cfg->T * cfg->H * cfg->W;
+  const long long L = n + prefix_len;
+  const long long total = (long long)cfg->B * L * cfg->nh;
+  softplus_kernel<<<static_cast<int>(std::min<long long>((total + 255) / 256, 4096)), 256, 0, st>>>(dt, dt_bias, delta,
+                                                                                                   total, cfg->nh);
+  MATE_LAUNCH_CHECK();
+  SeqRows rows;
+  rows.xv = rows.xr = x;
+  rows.bv = rows.br = Bm;
+  rows.cv = rows.cr = Cm;
+  rows.dv = rows.dr = delta;
+  rows.ldxv = rows.ldxr = cfg->nh * cfg->P;
+  rows.ldbv = rows.ldbr = rows.ldcv = rows.ldcr = cfg->N;
+  rows.lddv = rows.lddr = cfg->nh;
+  rows.v_bstride = L;
+  rows.v_off = prefix_len;
+  rows.r_bstride = L;
+  rows.r_off = 0;
+  rows.n = static_cast<int>(n);
+  rows.R = prefix_len;
+  rows.T = cfg->T;
+  rows.H = cfg->H;
+  rows.W = cfg->W;
+  rows.order = -1;
+  return run_ssd(cfg, rows, A_log, D, y, cfg->nh * cfg->P, n, sc, st);
+}
+
+mate_status tesa_forward(const void* qkv, void* O, int shifted, const mate_config* cfg, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (qkv == nullptr || O == nullptr || !aligned16(qkv) || !aligned16(O)) return MATE_ERR_ARG;
+  t_launches = 0;
+  const int a = cfg->th * cfg->tp;
+  return run_tesa(cfg, qkv, 3 * a, 0, a, 2 * a, O, a, 0, shifted, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mate_status mate_project_bf16(const void* A, int lda, long long M, int K, const void* Wt, int ldw, int N, void* C,
+                              int ldc, mate_stream_t stream) {
+  if (A == nullptr || Wt == nullptr || C == nullptr || M < 0 || K <= 0 || N <= 0) return MATE_ERR_ARG;
+  if (!aligned16(A) || !aligned16(Wt) || !aligned16(C) || lda % 8 || ldw % 8 || ldc % 8 || lda < K || ldw < K ||
+      ldc < N || M >= (1LL << 31))
+    return MATE_ERR_ARG;
+  if (K % kGemmBK) return MATE_ERR_UNSUPPORTED;
+  t_launches = 0;
+  return gemm_bf16(A, lda, M, K, Wt, ldw, N, C, ldc, nullptr, 0, 0, 0, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mate_status mate_forward(const void* X, const mate_weights* w, int layer_idx, void* Out, const mate_config* cfg,
+                         void* ws, size_t ws_bytes, mate_stream_t stream) {
+  t_launches = 0;
+  return forward_impl(X, w, layer_idx, Out, cfg, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mate_status mate_forward_host(const void* X_host, const mate_weights* w, int layer_idx, void* Out_host,
+                              const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (X_host == nullptr || Out_host == nullptr || ws == nullptr) return MATE_ERR_ARG;
+  if (ws_bytes < mate_forward_host_workspace_bytes(cfg)) return MATE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t fw = mate_workspace_bytes(cfg);
+  const size_t xb = (size_t)cfg->B * cfg->T * cfg->H * cfg->W * cfg->d * elem_size(cfg);
+  char* xdev = static_cast<char*>(ws) + ((fw + 255) & ~size_t(255));
+  char* odev = xdev + ((xb + 255) & ~size_t(255));
+  t_launches = 0;
+  if (cudaMemcpyAsync(xdev, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MATE_ERR_CUDA;
+  MATE_TRY(forward_impl(xdev, w, layer_idx, odev, cfg, ws, fw, st));
+  if (cudaMemcpyAsync(Out_host, odev, xb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MATE_ERR_CUDA;
+  return MATE_OK;
+}
+
+mate_status mate_device_status(mate_stream_t stream, unsigned int* flags) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MATE_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(v)) != cudaSuccess) return MATE_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(zero)) != cudaSuccess) return MATE_ERR_CUDA;
+  if (flags) *flags = v;
+  return v ? MATE_ERR_TIMEOUT : MATE_OK;
+}
+
+int mate_last_launch_count(void) { return t_launches; }
+
+}  // extern "C"

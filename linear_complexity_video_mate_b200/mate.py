@@ -1,0 +1,179 @@
+"""Python binding of libmate: argument marshalling only.
+
+Every step of the MATE block runs in the CUDA library (include/mate.h); PyTorch provides device memory
+and the current stream.  There is no Python or CPU implementation behind these calls: if libmate.so is
+missing, the first call raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Dict, Optional
+
+import torch
+
+from . import _lib
+
+__all__ = ["MateBlock", "rms_permute", "rms_unpermute", "review_pool", "ssd_scan_bidir", "tesa_forward",
+           "project_bf16", "device_status", "torch_dtype", "weights_to_device"]
+
+
+def torch_dtype(cfg) -> torch.dtype:
+    return torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, numel: int, name: str):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous() or t.numel() != numel:
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor with {numel} elements, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def weights_to_device(w: Dict, cfg, device="cuda") -> Dict[str, torch.Tensor]:
+    """Host weight arrays (numpy / tensors) -> device tensors in the library's dtypes."""
+    dt = torch_dtype(cfg)
+    out = {}
+    for k in ("W_in", "W_out", "W_qkv", "W_o"):
+        out[k] = torch.as_tensor(w[k]).to(device=device, dtype=dt).contiguous()
+    for k in ("dt_bias", "A_log", "D"):
+        out[k] = torch.as_tensor(w[k]).to(device=device, dtype=torch.float32).contiguous()
+    return out
+
+
+class MateBlock:
+    """One MATE block (MA + TE branches) with its weights resident on the GPU and a reusable workspace."""
+
+    def __init__(self, cfg, weights: Dict[str, torch.Tensor], device="cuda"):
+        lib = _lib.load()
+        self.cfg = cfg
+        self.ccfg = _lib.make_config(cfg)
+        _lib.check(lib.mate_check_config(ctypes.byref(self.ccfg)), "mate_check_config")
+        self.device = torch.device(device)
+        self.dtype = torch_dtype(cfg)
+        self.w = weights
+        n_in = cfg.nh * cfg.P + 2 * cfg.N + cfg.nh
+        _need(weights["W_in"], self.dtype, n_in * cfg.d, "W_in")
+        _need(weights["W_out"], self.dtype, cfg.d * cfg.nh * cfg.P, "W_out")
+        _need(weights["W_qkv"], self.dtype, 3 * cfg.th * cfg.tp * cfg.d, "W_qkv")
+        _need(weights["W_o"], self.dtype, cfg.d * cfg.th * cfg.tp, "W_o")
+        for k in ("dt_bias", "A_log", "D"):
+            _need(weights[k], torch.float32, cfg.nh, k)
+        self.cw = _lib.CWeights(*(weights[k].data_ptr() for k in
+                                  ("W_in", "dt_bias", "A_log", "D", "W_out", "W_qkv", "W_o")))
+        self.ws_bytes = lib.mate_workspace_bytes(ctypes.byref(self.ccfg))
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        self.ws_host = None
+        self.numel = cfg.B * cfg.T * cfg.H * cfg.W * cfg.d
+
+    def forward(self, X: torch.Tensor, layer_idx: int, out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """Out = MA(X) + TE(X) for X [B, T, H, W, d] on the GPU (stream-ordered, no synchronisation)."""
+        _need(X, self.dtype, self.numel, "X")
+        if out is None:
+            out = torch.empty_like(X)
+        _need(out, self.dtype, self.numel, "out")
+        st = _lib.load().mate_forward(_p(X), ctypes.byref(self.cw), int(layer_idx), _p(out), ctypes.byref(self.ccfg),
+                                      _p(self.ws), self.ws_bytes, _s(stream))
+        _lib.check(st, "mate_forward")
+        return out
+
+    def forward_host(self, X_host: torch.Tensor, layer_idx: int, out_host: torch.Tensor,
+                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """mate_forward_host: host (page-locked) input and output, copies inside the call."""
+        lib = _lib.load()
+        if self.ws_host is None:
+            nb = lib.mate_forward_host_workspace_bytes(ctypes.byref(self.ccfg))
+            self.ws_host = torch.empty(nb, dtype=torch.uint8, device=self.device)
+        for t, nm in ((X_host, "X_host"), (out_host, "out_host")):
+            if t.is_cuda or t.dtype != self.dtype or t.numel() != self.numel or not t.is_contiguous():
+                raise ValueError(f"{nm}: expected a contiguous host {self.dtype} tensor with {self.numel} elements")
+        st = lib.mate_forward_host(_p(X_host), ctypes.byref(self.cw), int(layer_idx), _p(out_host),
+                                   ctypes.byref(self.ccfg), _p(self.ws_host), self.ws_host.numel(), _s(stream))
+        _lib.check(st, "mate_forward_host")
+        return out_host
+
+    @staticmethod
+    def last_launch_count() -> int:
+        return _lib.load().mate_last_launch_count()
+
+
+def _cfg(cfg):
+    c = _lib.make_config(cfg)
+    return c
+
+
+def rms_permute(X: torch.Tensor, order: int, cfg, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    n = cfg.T * cfg.H * cfg.W
+    if out is None:
+        out = torch.empty((cfg.B, n, cfg.d), dtype=X.dtype, device=X.device)
+    c = _cfg(cfg)
+    _lib.check(_lib.load().rms_permute(_p(X), _p(out), int(order), ctypes.byref(c), _s(stream)), "rms_permute")
+    return out
+
+
+def rms_unpermute(Xp: torch.Tensor, order: int, cfg, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.W, cfg.d), dtype=Xp.dtype, device=Xp.device)
+    c = _cfg(cfg)
+    _lib.check(_lib.load().rms_unpermute(_p(Xp), _p(out), int(order), ctypes.byref(c), _s(stream)), "rms_unpermute")
+    return out
+
+
+def review_pool(X: torch.Tensor, order: int, cfg, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((cfg.B, cfg.R, cfg.d), dtype=X.dtype, device=X.device)
+    c = _cfg(cfg)
+    _lib.check(_lib.load().review_pool(_p(X), _p(out), int(order), ctypes.byref(c), _s(stream)), "review_pool")
+    return out
+
+
+def ssd_scan_bidir(x, Bm, Cm, dt, dt_bias, A_log, D, prefix_len: int, cfg, out=None, ws=None, stream=None):
+    """Bidirectional selective scan over [prefix; video] rows: x [B, L, nh*P], Bm/Cm [B, L, N], dt [B, L, nh]
+    (fp32, before softplus).  Returns y [B, T*H*W, nh*P] for the video rows."""
+    lib = _lib.load()
+    c = _cfg(cfg)
+    n = cfg.T * cfg.H * cfg.W
+    if out is None:
+        out = torch.empty((cfg.B, n, cfg.nh * cfg.P), dtype=x.dtype, device=x.device)
+    nb = lib.mate_ssd_workspace_bytes(ctypes.byref(c), int(prefix_len))
+    if ws is None or ws.numel() < nb:
+        ws = torch.empty(nb, dtype=torch.uint8, device=x.device)
+    st = lib.ssd_scan_bidir(_p(x), _p(Bm), _p(Cm), _p(dt), _p(dt_bias), _p(A_log), _p(D), int(prefix_len), _p(out),
+                            ctypes.byref(c), _p(ws), ws.numel(), _s(stream))
+    _lib.check(st, "ssd_scan_bidir")
+    return out
+
+
+def tesa_forward(qkv: torch.Tensor, shifted: bool, cfg, out: Optional[torch.Tensor] = None, stream=None):
+    if out is None:
+        out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.W, cfg.th * cfg.tp), dtype=qkv.dtype, device=qkv.device)
+    c = _cfg(cfg)
+    _lib.check(_lib.load().tesa_forward(_p(qkv), _p(out), int(bool(shifted)), ctypes.byref(c), _s(stream)),
+               "tesa_forward")
+    return out
+
+
+def project_bf16(A: torch.Tensor, Wt: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """C = A W^T on tensor cores: A [M, K] bf16, Wt [N, K] bf16 -> C [M, N] bf16."""
+    M, K = A.shape
+    N = Wt.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    st = _lib.load().mate_project_bf16(_p(A), A.stride(0), M, K, _p(Wt), Wt.stride(0), N, _p(out), out.stride(0),
+                                       _s(stream))
+    _lib.check(st, "mate_project_bf16")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise and read/clear the device status word (1 = a bounded wait ran out)."""
+    flags = ctypes.c_uint(0)
+    _lib.load().mate_device_status(_s(stream), ctypes.byref(flags))
+    return int(flags.value)

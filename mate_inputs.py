@@ -101,8 +101,8 @@ TEST_CONFIGS: Dict[str, MateConfig] = {
                                "bf16", 11),
     "bf16_ragged_12x16x24": _cfg("bf16_ragged_12x16x24", 1, 12, 16, 24, 1024, 16, 64, 128, 256, 48, 8, 128,
                                  (4, 8, 8), "bf16", 12),
-    "bf16_b2_8x16x16_d512": _cfg("bf16_b2_8x16x16_d512", 2, 8, 16, 16, 512, 8, 64, 128, 256, 272, 4, 128,
-                                 (4, 8, 8), "bf16", 13),
+    "bf16_b2_20x16x16_d512": _cfg("bf16_b2_20x16x16_d512", 2, 20, 16, 16, 512, 8, 64, 128, 256, 320, 4, 128,
+                                  (4, 8, 8), "bf16", 13),
     "f32_b2_4x8x12": _cfg("f32_b2_4x8x12", 2, 4, 8, 12, 64, 2, 32, 16, 64, 32, 2, 32, (2, 4, 4), "f32", 14,
                           shift=(1, 2, 2)),
 }

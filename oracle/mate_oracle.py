@@ -226,7 +226,8 @@ def tesa_attention(qkv: np.ndarray, th: int, tp: int, window, shift, shifted: bo
                 iw = np.array([m[2] for m in members])
                 Qw, Kw, Vw = q[it, ih, iw], k[it, ih, iw], v[it, ih, iw]      # [m, th, tp]
                 m = len(members)
-                allowed = np.array([[regions[i] == regions[j] for j in range(m)] for i in range(m)])
+                reg = np.array(regions)                                       # [m, 3]
+                allowed = (reg[:, None, :] == reg[None, :, :]).all(axis=2)    # same region on every axis
                 scores = np.einsum("ihc,jhc->hij", Qw, Kw) * scale
                 scores = np.where(allowed[None], scores, -np.inf)
                 scores = scores - scores.max(axis=2, keepdims=True)

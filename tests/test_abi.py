@@ -1,0 +1,103 @@
+"""The C ABI library: it builds, loads without a GPU, exports every symbol include/mate.h declares, and
+validates arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from helpers import ROOT
+from linear_complexity_video_mate_b200 import _lib, build
+import mate_inputs as mi
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _header_symbols():
+    with open(os.path.join(ROOT, "include", "mate.h")) as f:
+        text = f.read()
+    return set(re.findall(r"MATE_API\s+[\w\s\*]+?\b(\w+)\s*\(", text))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _header_symbols()
+    assert declared == set(_lib.EXPORTS), declared ^ set(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert _lib.status_str(s)
+
+
+def test_all_workloads_are_valid(lib):
+    for name, cfg in mi.all_configs().items():
+        c = _lib.make_config(cfg)
+        assert lib.mate_check_config(ctypes.byref(c)) == _lib.MATE_OK, name
+        assert lib.mate_workspace_bytes(ctypes.byref(c)) > 0, name
+
+
+def _cfg(**kw):
+    base = mi.CONFIGS["bf16_16x32x32"]
+    import dataclasses
+    return _lib.make_config(dataclasses.replace(base, **kw))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=15), _lib.MATE_ERR_SHAPE),            # window does not divide T
+    (dict(R=24), _lib.MATE_ERR_SHAPE),            # R not a multiple of 16
+    (dict(R=16 * 5), _lib.MATE_ERR_SHAPE),        # pooled grid 5 x 4 x 4 does not divide T = 16
+    (dict(st=4), _lib.MATE_ERR_SHAPE),            # shift not smaller than the window
+    (dict(P=32), _lib.MATE_ERR_UNSUPPORTED),      # bf16 tensor-core scan needs P = 64
+    (dict(tp=64), _lib.MATE_ERR_UNSUPPORTED),
+    (dict(d=1004), _lib.MATE_ERR_SHAPE),          # rows not a multiple of 16 bytes
+    (dict(d=1000), _lib.MATE_ERR_UNSUPPORTED),    # bf16 projections need d % 64 == 0
+    (dict(B=0), _lib.MATE_ERR_SHAPE),
+])
+def test_config_rejections(lib, kw, status):
+    c = _cfg(**kw)
+    assert lib.mate_check_config(ctypes.byref(c)) == status
+    assert lib.mate_workspace_bytes(ctypes.byref(c)) == 0
+
+
+def test_null_and_misaligned_arguments_are_rejected_before_launch(lib):
+    c = _cfg()
+    fake = ctypes.c_void_p(1 << 20)      # aligned, never dereferenced: validation fails first
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    w = _lib.CWeights(*([1 << 20] * 7))
+    cp = ctypes.byref(c)
+    assert lib.rms_permute(None, fake, 0, cp, None) == _lib.MATE_ERR_ARG
+    assert lib.rms_permute(fake, fake, 4, cp, None) == _lib.MATE_ERR_ARG
+    assert lib.rms_unpermute(mis, fake, 1, cp, None) == _lib.MATE_ERR_ARG
+    assert lib.review_pool(fake, None, 0, cp, None) == _lib.MATE_ERR_ARG
+    assert lib.tesa_forward(fake, None, 1, cp, None) == _lib.MATE_ERR_ARG
+    assert lib.mate_forward(fake, ctypes.byref(w), -1, fake, cp, fake, 1 << 40, None) == _lib.MATE_ERR_ARG
+    assert lib.mate_forward(fake, None, 0, fake, cp, fake, 1 << 40, None) == _lib.MATE_ERR_ARG
+    need = lib.mate_workspace_bytes(cp)
+    assert lib.mate_forward(fake, ctypes.byref(w), 0, fake, cp, fake, need - 1, None) == _lib.MATE_ERR_WORKSPACE
+    assert lib.ssd_scan_bidir(fake, fake, fake, fake, fake, fake, fake, -1, fake, cp, fake, 1 << 40, None) == \
+        _lib.MATE_ERR_ARG
+    nss = lib.mate_ssd_workspace_bytes(cp, 256)
+    assert lib.ssd_scan_bidir(fake, fake, fake, fake, fake, fake, fake, 256, fake, cp, fake, nss - 1, None) == \
+        _lib.MATE_ERR_WORKSPACE
+    assert lib.mate_project_bf16(fake, 512, 128, 1024, fake, 1024, 256, fake, 256, None) == _lib.MATE_ERR_ARG
+    assert lib.mate_project_bf16(fake, 1000, 128, 1000, fake, 1000, 256, fake, 256, None) == \
+        _lib.MATE_ERR_UNSUPPORTED
+    bad = _cfg(T=15)
+    assert lib.mate_forward(fake, ctypes.byref(w), 0, fake, ctypes.byref(bad), fake, 1 << 40, None) == \
+        _lib.MATE_ERR_SHAPE
+
+
+def test_workspace_grows_linearly_with_tokens(lib):
+    sizes = []
+    for T in (16, 64, 256):
+        c = _cfg(T=T, R=256)
+        sizes.append(lib.mate_workspace_bytes(ctypes.byref(c)))
+    per = [(sizes[i + 1] - sizes[i]) for i in range(2)]
+    # doubling-by-4 of T adds 4x the per-token bytes each time
+    assert abs(per[1] / per[0] - 4.0) < 0.01

@@ -1,0 +1,218 @@
+"""Parity of the CUDA library (through the C ABI) with the fp64 oracle, element by element, on seeded
+synthetic inputs.  Permutations are compared bit for bit; floating point within the block's tolerances
+(helpers.assert_close)."""
+import numpy as np
+import pytest
+
+from helpers import assert_close, assert_close_elementwise, oracle_cached, requires_gpu
+from bf16_floor import bf16_storage_forward, rms_normalised_max_err
+import mate_inputs as mi
+from oracle import mate_oracle as O
+
+pytestmark = [pytest.mark.gpu, requires_gpu]
+
+torch = pytest.importorskip("torch")
+from linear_complexity_video_mate_b200 import mate as M  # noqa: E402
+
+
+def dev(a, dtype):
+    return torch.as_tensor(np.ascontiguousarray(a)).to(device="cuda", dtype=dtype)
+
+
+def host(t):
+    return t.float().cpu().numpy()
+
+
+def tdt(cfg):
+    return torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+
+
+def cast(cfg, a):
+    return mi.round_to_bf16(a) if cfg.dtype == "bf16" else np.asarray(a, np.float32)
+
+
+SMALL = ["tiny_f32_4x8x8", "f32_b2_4x8x12", "bf16_small_8x16x16", "bf16_ragged_12x16x24", "bf16_b2_20x16x16_d512"]
+
+
+# ------------------------------------------------------------------ Rotary Major Scan + review tokens
+
+@pytest.mark.parametrize("name", SMALL + ["bf16_16x32x32", "bf16_256x32x32", "bf16_2x64x48x48_d2048"])
+def test_rms_permute_unpermute_bitexact(name):
+    cfg = mi.all_configs()[name]
+    X = mi.make_x_only(cfg, 100)
+    Xd = dev(X, tdt(cfg))
+    for order in range(4):
+        Xp = M.rms_permute(Xd, order, cfg)
+        torch.cuda.synchronize()
+        got = host(Xp)
+        for b in range(cfg.B):
+            pos = O.scan_positions(cfg.T, cfg.H, cfg.W, order).ravel()
+            expect = np.empty((cfg.n, cfg.d), np.float32)
+            expect[pos] = X[b].reshape(cfg.n, cfg.d)        # row s(t,h,w) = X[t,h,w]
+            assert np.array_equal(got[b], expect), (name, order, b)
+        back = M.rms_unpermute(Xp, order, cfg)
+        assert torch.equal(back, Xd), (name, order)
+
+
+@pytest.mark.parametrize("name", SMALL + ["bf16_256x32x32"])
+def test_review_pool(name):
+    cfg = mi.all_configs()[name]
+    X = mi.make_x_only(cfg, 101)
+    Xd = dev(X, tdt(cfg))
+    for order in range(4):
+        got = host(M.review_pool(Xd, order, cfg))
+        ref = np.stack([O.review_tokens(X[b], cfg.R, order) for b in range(cfg.B)])
+        if cfg.dtype == "bf16":
+            # fp32 accumulation then one bf16 rounding: within one bf16 unit of the exact mean
+            assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6), (name, order)
+        else:
+            np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6)
+
+
+# ------------------------------------------------------------------ tensor-core projection
+
+@pytest.mark.parametrize("M_,K,N", [(128, 64, 128), (300, 1024, 4368), (1024, 2048, 1024), (77, 512, 2336),
+                                    (4096, 1024, 8480)])
+def test_project_bf16(M_, K, N):
+    rng = np.random.default_rng(M_ + K + N)
+    A = mi.round_to_bf16(rng.standard_normal((M_, K)))
+    W = mi.round_to_bf16(rng.standard_normal((N, K)) / np.sqrt(K))
+    got = host(M.project_bf16(dev(A, torch.bfloat16), dev(W, torch.bfloat16)))
+    ref = A.astype(np.float64) @ W.astype(np.float64).T
+    assert_close(got, ref, "bf16", f"project {M_}x{K}x{N}")
+
+
+# ------------------------------------------------------------------ selective scan
+
+def _ssd_inputs(cfg, long_memory, seed):
+    rng = np.random.default_rng(seed)
+    L = cfg.R + cfg.n
+    x = cast(cfg, rng.standard_normal((cfg.B, L, cfg.nh * cfg.P)))
+    Bm = cast(cfg, rng.standard_normal((cfg.B, L, cfg.N)))
+    Cm = cast(cfg, rng.standard_normal((cfg.B, L, cfg.N)))
+    dt = rng.standard_normal((cfg.B, L, cfg.nh)).astype(np.float32)
+    dt_bias = np.full(cfg.nh, -4.0 if long_memory else 0.0, np.float32)
+    A_log = rng.uniform(-3.0, -1.0, cfg.nh).astype(np.float32) if long_memory else \
+        rng.uniform(0.0, 1.0, cfg.nh).astype(np.float32)
+    D = rng.standard_normal(cfg.nh).astype(np.float32)
+    return x, Bm, Cm, dt, dt_bias, A_log, D
+
+
+def _ssd_oracle(cfg, x, Bm, Cm, dt, dt_bias, A_log, D, heads=None):
+    heads = list(range(cfg.nh)) if heads is None else heads
+    out = []
+    for b in range(cfg.B):
+        xs = x[b].reshape(-1, cfg.nh, cfg.P)[:, heads]
+        delta = O.softplus(dt[b].astype(np.float64) + dt_bias.astype(np.float64))[:, heads]
+        A = -np.exp(A_log.astype(np.float64))[heads]
+        out.append(O.ssd_bidirectional(xs, Bm[b], Cm[b], delta, A, D.astype(np.float64)[heads], cfg.R))
+    return np.stack(out)   # [B, n, len(heads), P]
+
+
+@pytest.mark.parametrize("long_memory", [False, True])
+@pytest.mark.parametrize("name", SMALL)
+def test_ssd_scan_bidir(name, long_memory):
+    cfg = mi.all_configs()[name]
+    args = _ssd_inputs(cfg, long_memory, 7)
+    x, Bm, Cm, dt, dt_bias, A_log, D = args
+    td = tdt(cfg)
+    y = M.ssd_scan_bidir(dev(x, td), dev(Bm, td), dev(Cm, td), dev(dt, torch.float32), dev(dt_bias, torch.float32),
+                         dev(A_log, torch.float32), dev(D, torch.float32), cfg.R, cfg)
+    got = host(y).reshape(cfg.B, cfg.n, cfg.nh, cfg.P)
+    ref = oracle_cached(f"ssd-{name}-{long_memory}", lambda: _ssd_oracle(cfg, *args))
+    assert_close_elementwise(got, ref, cfg.dtype, f"ssd {name} long={long_memory}")
+
+
+# ------------------------------------------------------------------ TESA
+
+def _tesa_inputs(cfg, seed):
+    rng = np.random.default_rng(seed)
+    return cast(cfg, rng.standard_normal((cfg.B, cfg.T, cfg.H, cfg.W, 3 * cfg.th * cfg.tp)))
+
+
+@pytest.mark.parametrize("shifted", [False, True])
+@pytest.mark.parametrize("name", SMALL + ["bf16_16x32x32"])
+def test_tesa_forward(name, shifted):
+    cfg = mi.all_configs()[name]
+    qkv = _tesa_inputs(cfg, 8)
+    got = host(M.tesa_forward(dev(qkv, tdt(cfg)), shifted, cfg))
+    ref = oracle_cached(f"tesa-{name}-{shifted}", lambda: np.stack([
+        O.tesa_attention(qkv[b], cfg.th, cfg.tp, (cfg.wt, cfg.wh, cfg.ww), (cfg.st, cfg.sh, cfg.sw), shifted)
+        for b in range(cfg.B)]))
+    assert_close_elementwise(got, ref, cfg.dtype, f"tesa {name} shifted={shifted}")
+
+
+# ------------------------------------------------------------------ whole block
+
+def _floor(cfg, w, layer, variant, ref):
+    """RMS-normalised error of bf16 storage alone for this case (0 for fp32 blocks)."""
+    if cfg.dtype != "bf16":
+        return 0.0
+    f = oracle_cached(f"floor-{cfg.name}-{layer}-{variant}",
+                      lambda: np.array([rms_normalised_max_err(bf16_storage_forward(w["X"], w, cfg, layer), ref)]))
+    return float(f[0])
+
+
+def _block(cfg, variant):
+    kw = dict(dt_bias=-4.0, a_log_range=(-3.0, -1.0)) if variant == "long" else {}
+    return mi.make_inputs(cfg, **kw)
+
+
+@pytest.mark.parametrize("variant", ["default", "long"])
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+@pytest.mark.parametrize("name", SMALL + ["bf16_16x32x32"])
+def test_mate_forward(name, layer, variant):
+    cfg = mi.all_configs()[name]
+    w = _block(cfg, variant)
+    blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
+    out = host(blk.forward(dev(w["X"], tdt(cfg)), layer))
+    ref = oracle_cached(f"mate-{name}-{layer}-{variant}", lambda: O.mate_forward(w["X"], w, cfg, layer))
+    assert_close(out, ref, cfg.dtype, f"mate {name} layer {layer} {variant}", _floor(cfg, w, layer, variant, ref))
+
+
+def test_mate_forward_host_matches_device_path():
+    cfg = mi.TEST_CONFIGS["bf16_small_8x16x16"]
+    w = _block(cfg, "default")
+    blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
+    Xd = dev(w["X"], torch.bfloat16)
+    ref = blk.forward(Xd, 3)
+    xh = Xd.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    blk.forward_host(xh, 3, oh)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, ref.cpu())
+
+
+def test_repeated_calls_are_deterministic():
+    cfg = mi.TEST_CONFIGS["bf16_ragged_12x16x24"]
+    w = _block(cfg, "long")
+    blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
+    Xd = dev(w["X"], torch.bfloat16)
+    a = blk.forward(Xd, 1).clone()
+    for _ in range(3):
+        assert torch.equal(blk.forward(Xd, 1), a)
+    assert M.device_status() == 0
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+@pytest.mark.parametrize("name,layer", [("bf16_256x32x32", 1), ("bf16_64x32x32", 2)])
+def test_mate_forward_full_size(name, layer):
+    cfg = mi.CONFIGS[name]
+    w = mi.make_inputs(cfg)
+    blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
+    out = host(blk.forward(dev(w["X"], torch.bfloat16), layer))
+    ref = oracle_cached(f"mate-{name}-{layer}-default", lambda: O.mate_forward(w["X"], w, cfg, layer))
+    assert_close(out, ref, "bf16", f"mate {name} layer {layer}", _floor(cfg, w, layer, "default", ref))
+
+
+def test_ssd_full_size_sampled_head():
+    cfg = mi.CONFIGS["bf16_256x32x32"]
+    args = _ssd_inputs(cfg, True, 9)
+    x, Bm, Cm, dt, dt_bias, A_log, D = args
+    y = M.ssd_scan_bidir(dev(x, torch.bfloat16), dev(Bm, torch.bfloat16), dev(Cm, torch.bfloat16),
+                         dev(dt, torch.float32), dev(dt_bias, torch.float32), dev(A_log, torch.float32),
+                         dev(D, torch.float32), cfg.R, cfg)
+    got = host(y).reshape(cfg.B, cfg.n, cfg.nh, cfg.P)[:, :, [5]]
+    ref = oracle_cached("ssd-full-bf16_256x32x32-h5", lambda: _ssd_oracle(cfg, *args, heads=[5]))
+    assert_close_elementwise(got, ref, "bf16", "ssd full size head 5")
