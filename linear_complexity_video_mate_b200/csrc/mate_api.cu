@@ -316,9 +316,9 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   p.y = static_cast<__nv_bfloat16*>(y);
   p.ldy = ldy;
   p.y_bstride = y_bstride;
-  const size_t smem_gram = 1024 + 98304 + 64;
-  const size_t smem_state = 1024 + 131072 + 2048 + 64 + 64;
-  const size_t smem_out = 1024 + 196608 + 3072 + 64 + 64;
+  const size_t smem_gram = 1024 + 98304 + 2048 + 64;
+  const size_t smem_state = 1024 + 131072 + 2048 + 64 + 2048 + 64;
+  const size_t smem_out = 1024 + 196608 + (5 * 256 + 2048 + 16) * 4 + 2048 + 64;
   if (!set_smem(ssd_gram_kernel, smem_gram) || !set_smem(ssd_state_kernel, smem_state) ||
       !set_smem(ssd_output_kernel, smem_out))
     return MATE_ERR_CUDA;
@@ -330,7 +330,7 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   MATE_LAUNCH_CHECK();
   ssd_carry_kernel<<<dim3(kSsdP * kSsdN / 8 / 128, c->nh, 2 * c->B), 128, 0, st>>>(p);
   MATE_LAUNCH_CHECK();
-  ssd_output_kernel<<<dim3(p.nVc, c->B, c->nh), 256, smem_out, st>>>(p);
+  ssd_output_kernel<<<dim3(p.nVc, c->B, c->nh), kSsdOutThreads, smem_out, st>>>(p);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }
@@ -369,10 +369,10 @@ mate_status run_tesa(const mate_config* c, const void* qkv, int ldq, int qcol, i
   p.sw = sft ? c->sw : 0;
   p.shifted = sft;
   p.scale_log2 = 1.4426950408889634f / std::sqrt(static_cast<float>(c->tp));
-  const size_t smem = 1024 + 196608 + 2048 + 1024 + 64;
+  const size_t smem = 1024 + 196608 + 2048 + 1024 + 2048 + 64;
   if (!set_smem(tesa_bf16_kernel, smem)) return MATE_ERR_CUDA;
   const int nwin = (c->T / c->wt) * (c->H / c->wh) * (c->W / c->ww);
-  tesa_bf16_kernel<<<dim3(nwin, c->B, c->th), 256, smem, st>>>(p);
+  tesa_bf16_kernel<<<dim3(nwin, c->B, c->th), kTesaThreads, smem, st>>>(p);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }

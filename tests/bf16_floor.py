@@ -45,3 +45,65 @@ def bf16_storage_forward(X, w, cfg, layer):
 def rms_normalised_max_err(a, ref):
     ref = np.asarray(ref, np.float64)
     return float(np.abs(np.asarray(a, np.float64) - ref).max() / np.sqrt(np.mean(ref * ref)))
+
+
+def ssd_bf16_storage_emulation(x, Bm, Cm, delta, A, D, R, Q=256):
+    """Chunked bidirectional scan in exact (fp64) arithmetic that rounds to bf16 only what a bf16
+    tensor-core scan must hold in bf16: the MMA operands (G = C B^T, the intra-chunk coefficients,
+    the decay-weighted inputs of the chunk states, the carried states) and the stored chunk states and
+    output.  The scan test bounds the GPU's element-wise error by this emulation's error (the GPU adds
+    only accumulation-order differences on top).  x [L, nh, P], Bm / Cm [L, N], delta [L, nh]."""
+    x, Bm, Cm, delta = (np.asarray(a, np.float64) for a in (x, Bm, Cm, delta))
+    A, D = np.asarray(A, np.float64), np.asarray(D, np.float64)
+    L, nh, P = x.shape
+    N = Bm.shape[1]
+    n = L - R
+    nRc, nVc = -(-R // Q), -(-n // Q)
+    chunks = [(c * Q, min(c * Q + Q, R)) for c in range(nRc)] + [(R + v * Q, R + min(v * Q + Q, n)) for v in range(nVc)]
+    out = np.zeros((n, nh, P))
+    for h in range(nh):
+        Sf, Sb, gl = [], [], []
+        for a0, a1 in chunks:
+            a = delta[a0:a1, h] * A[h]
+            s = np.cumsum(a)
+            wf = np.exp(s[-1] - s) * delta[a0:a1, h]
+            wb = np.exp(s - a) * delta[a0:a1, h]
+            Sf.append(_r(_r(wf[:, None] * x[a0:a1, h]).T @ Bm[a0:a1]))
+            Sb.append(_r(_r(wb[:, None] * x[a0:a1, h]).T @ Bm[a0:a1]))
+            gl.append(s[-1])
+        H = np.zeros((P, N))
+        for c in range(nRc):
+            H = np.exp(gl[c]) * H + Sf[c]
+        Hr = H.copy()
+        Hf, Hb = [None] * nVc, [None] * nVc
+        for v in range(nVc):
+            Hf[v] = _r(H)
+            H = np.exp(gl[nRc + v]) * H + Sf[nRc + v]
+        H = Hr
+        for v in range(nVc - 1, -1, -1):
+            Hb[v] = _r(H)
+            H = np.exp(gl[nRc + v]) * H + Sb[nRc + v]
+        for v in range(nVc):
+            a0, a1 = chunks[nRc + v]
+            m = a1 - a0
+            a = delta[a0:a1, h] * A[h]
+            s = np.cumsum(a)
+            sx = s - a
+            G = Cm[a0:a1] @ Bm[a0:a1].T
+            i = np.arange(m)[:, None]
+            j = np.arange(m)[None, :]
+            dec = np.where(j < i, np.exp(np.minimum(s[:, None] - s[None, :], 0)),
+                           np.where(j > i, np.exp(np.minimum(sx[None, :] - sx[:, None], 0)), 0.0))
+            M = _r(_r(G) * delta[a0:a1, h][None, :] * dec)
+            y = M @ x[a0:a1, h] + np.exp(s)[:, None] * (Cm[a0:a1] @ Hf[v].T) + \
+                np.exp(s[-1] - sx)[:, None] * (Cm[a0:a1] @ Hb[v].T)
+            y += 2 * (np.diag(G) * delta[a0:a1, h] + D[h])[:, None] * x[a0:a1, h]
+            out[v * Q:v * Q + m, h] = _r(y)
+    return out
+
+
+def elementwise_err(a, ref):
+    """max_i |a_i - ref_i| / max(|ref_i|, rms(ref))."""
+    a, ref = np.asarray(a, np.float64), np.asarray(ref, np.float64)
+    rms = np.sqrt(np.mean(ref * ref))
+    return float((np.abs(a - ref) / np.maximum(np.abs(ref), rms)).max())

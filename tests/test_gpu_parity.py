@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 from helpers import assert_close, assert_close_elementwise, oracle_cached, requires_gpu
-from bf16_floor import bf16_storage_forward, rms_normalised_max_err
+from bf16_floor import bf16_storage_forward, elementwise_err, rms_normalised_max_err, ssd_bf16_storage_emulation
 import mate_inputs as mi
 from oracle import mate_oracle as O
 
@@ -120,7 +120,27 @@ def test_ssd_scan_bidir(name, long_memory):
                          dev(A_log, torch.float32), dev(D, torch.float32), cfg.R, cfg)
     got = host(y).reshape(cfg.B, cfg.n, cfg.nh, cfg.P)
     ref = oracle_cached(f"ssd-{name}-{long_memory}", lambda: _ssd_oracle(cfg, *args))
-    assert_close_elementwise(got, ref, cfg.dtype, f"ssd {name} long={long_memory}")
+    assert_close_elementwise(got, ref, cfg.dtype, f"ssd {name} long={long_memory}",
+                             _ssd_floor(cfg, args, ref, f"ssd-{name}-{long_memory}"))
+
+
+def _ssd_floor(cfg, args, ref, key, heads=None):
+    """Element-wise error of the bf16-storage emulation of the chunked scan (0 for fp32 blocks)."""
+    if cfg.dtype != "bf16":
+        return 0.0
+    x, Bm, Cm, dt, dt_bias, A_log, D = args
+    heads = list(range(cfg.nh)) if heads is None else heads
+
+    def emu():
+        outs = []
+        for b in range(cfg.B):
+            delta = O.softplus(dt[b].astype(np.float64) + dt_bias.astype(np.float64))[:, heads]
+            A = -np.exp(A_log.astype(np.float64))[heads]
+            xs = x[b].reshape(-1, cfg.nh, cfg.P)[:, heads]
+            outs.append(ssd_bf16_storage_emulation(xs, Bm[b], Cm[b], delta, A, D.astype(np.float64)[heads], cfg.R,
+                                                   cfg.Q))
+        return np.array([elementwise_err(np.stack(outs), ref)])
+    return float(oracle_cached(f"floor-{key}", emu)[0])
 
 
 # ------------------------------------------------------------------ TESA
@@ -215,4 +235,5 @@ def test_ssd_full_size_sampled_head():
                          dev(D, torch.float32), cfg.R, cfg)
     got = host(y).reshape(cfg.B, cfg.n, cfg.nh, cfg.P)[:, :, [5]]
     ref = oracle_cached("ssd-full-bf16_256x32x32-h5", lambda: _ssd_oracle(cfg, *args, heads=[5]))
-    assert_close_elementwise(got, ref, "bf16", "ssd full size head 5")
+    assert_close_elementwise(got, ref, "bf16", "ssd full size head 5",
+                             _ssd_floor(cfg, args, ref, "ssd-full-bf16_256x32x32-h5", heads=[5]))
