@@ -179,4 +179,165 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------------------------
+// Two-SM variant: a cluster of 2 CTAs computes a 256 x BN tile with tcgen05.mma.cta_group::2.  Each CTA
+// loads its own 128 rows of A and BN/2 rows of B (TMA, no multicast), so the pair moves 25% fewer
+// operand bytes per FLOP from L2 than two independent 128 x BN tiles and each stage is smaller (deeper
+// ring).  The leader CTA (rank 0) issues the MMAs; the stage barriers that gate operand reuse live in
+// both CTAs, the "operands landed" barriers only in the leader.  Each CTA's TMEM holds its 128 rows of
+// the accumulator (two buffers of up to 256 columns) and each CTA runs its own epilogue.
+// ---------------------------------------------------------------------------------------------------
+__host__ __device__ inline uint32_t gemm_pair_stage_bytes(int bn) { return 128 * 128 + (bn / 2) * 128; }
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t stage_bytes = gemm_pair_stage_bytes(p.bn);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.stages * stage_bytes);
+  uint64_t* full = bars;                  // leader only: operands of both CTAs landed
+  uint64_t* empty = bars + p.stages;      // both CTAs: the pair MMAs are done with this stage
+  uint64_t* tfull = bars + 2 * p.stages;  // both CTAs: accumulator ready
+  uint64_t* tempty = tfull + 2;           // leader only: both CTAs' epilogues drained the accumulator
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int nk = p.K / kGemmBK;
+  const int half_bn = p.bn / 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each of the 2 CTAs
+    }
+    mbar_fence_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any cross-CTA arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+        const int mb = tile / p.num_n_tiles, nb = tile % p.num_n_tiles;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+          uint8_t* sa = smem + stage * stage_bytes;
+          const uint32_t full_leader = map_to_cta(&full[stage], 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
+          tma_load_2d_pair(&tmA, full_leader, sa, kb * kGemmBK, mb * 256 + rank * 128);
+          tma_load_2d_pair(&tmB, full_leader, sa + 128 * 128, kb * kGemmBK, nb * p.bn + rank * half_bn);
+          if (++stage == (uint32_t)p.stages) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_par = (it >> 1) & 1;
+        // the last column tile of a ragged N only multiplies the columns it has (rounded up to 16)
+        const int nb = tile % p.num_n_tiles;
+        const int n_mma = min(p.bn, (p.N - nb * p.bn + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32(256, n_mma, 0, 0);
+        if (!mbar_wait(&tempty[acc], acc_par ^ 1)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * 256;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * stage_bytes);
+          const uint32_t sb = sa + 128 * 128;
+#pragma unroll
+          for (int k = 0; k < kGemmBK / 16; ++k)
+            mma_bf16_pair(d_tmem, desc_sw128(sa + k * 32, 16, 1024), desc_sw128(sb + k * 32, 16, 1024), idesc,
+                          (kb | k) != 0);
+          mma_commit_pair(map_to_cta(&empty[stage], 0));
+          mma_commit_pair(map_to_cta(&empty[stage], 1));
+          if (++stage == (uint32_t)p.stages) { stage = 0; phase ^= 1; }
+        }
+        mma_commit_pair(map_to_cta(&tfull[acc], 0));
+        mma_commit_pair(map_to_cta(&tfull[acc], 1));
+      }
+    }
+  } else {
+    // epilogue warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1 of this CTA's 128 rows
+    const int quad = warp & 3;
+    int it = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
+      const int mb = tile / p.num_n_tiles, nb = tile % p.num_n_tiles;
+      const int acc = it & 1;
+      const uint32_t acc_par = (it >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_par)) break;
+      tc_fence_after();
+      const int row = mb * 256 + rank * 128 + quad * 32 + lane;
+      const bool row_ok = row < p.M;
+      __nv_bfloat16* crow = p.C + static_cast<size_t>(row) * p.ldc;
+      const int col_end = min(p.N, nb * p.bn + p.bn);
+      for (int c0 = 0; c0 < col_end - nb * p.bn; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256 + c0, r);
+        tmem_wait_ld();
+        const int col0 = nb * p.bn + c0;
+        if (!row_ok || col0 >= col_end) continue;
+        if (col0 + 32 <= col_end) {
+          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 pk;
+            pk.x = pack_bf16x2(__uint_as_float(r[v * 8 + 0]), __uint_as_float(r[v * 8 + 1]));
+            pk.y = pack_bf16x2(__uint_as_float(r[v * 8 + 2]), __uint_as_float(r[v * 8 + 3]));
+            pk.z = pack_bf16x2(__uint_as_float(r[v * 8 + 4]), __uint_as_float(r[v * 8 + 5]));
+            pk.w = pack_bf16x2(__uint_as_float(r[v * 8 + 6]), __uint_as_float(r[v * 8 + 7]));
+            dst[v] = pk;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < col_end) crow[col0 + j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        }
+        if (p.delta != nullptr && col0 < p.dt_col0 + p.dt_cols && col0 + 32 > p.dt_col0) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int c = col0 + j - p.dt_col0;
+            if (c >= 0 && c < p.dt_cols && col0 + j < col_end)
+              p.delta[static_cast<size_t>(row) * p.ld_delta + c] = softplus_f(__uint_as_float(r[j]) + p.dt_bias[c]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_cta(&tempty[acc], 0));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the leader's MMAs read this CTA's shared memory: nobody leaves before both are done
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
 }  // namespace mate

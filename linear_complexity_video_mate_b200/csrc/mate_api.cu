@@ -196,18 +196,9 @@ size_t ssd_ws_bytes(const mate_config* c, int prefix_len, float** delta, SsdScra
 }
 
 // ------------------------------------------------------------------------------ launchers
-int choose_bn(int N) {
-  int best = 256;
-  long long best_cost = -1;
-  for (int bn = 256; bn >= 128; bn -= 16) {
-    const long long cost = (long long)ceil_div(N, bn) * (bn + 64);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = bn;
-    }
-  }
-  return best;
-}
+// Column tile of the projection GEMM.  256 wide tiles run the tensor cores best (measured against
+// narrower, padding-free tiles); a ragged last tile issues narrower MMAs instead of padding.
+int choose_bn(int N) { return N >= 256 ? 256 : ((N + 15) / 16) * 16; }
 
 mate_status gemm_bf16(const void* A, int lda, long long M, int K, const void* Bw, int ldb, int N, void* C, int ldc,
                       float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias, cudaStream_t st) {
@@ -229,12 +220,16 @@ mate_status gemm_bf16(const void* A, int lda, long long M, int K, const void* Bw
   p.dt_col0 = dt_col0;
   p.dt_cols = dt_cols;
   p.dt_bias = dt_bias;
+  // 256-row tiles computed by 2-CTA clusters (tcgen05 cta_group::2)
+  p.num_tiles = ceil_div(M, 256) * p.num_n_tiles;
+  const uint32_t psb = gemm_pair_stage_bytes(p.bn);
+  p.stages = std::min<int>(8, static_cast<int>((kSmemLimit - 1024 - 256) / psb));
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, A, M, K, lda, kGemmBM) || !make_tmap(&tb, Bw, N, K, ldb, p.bn)) return MATE_ERR_CUDA;
-  const size_t smem = 1024 + (size_t)p.stages * sb + 256;
-  if (!set_smem(gemm_bf16_tc_kernel, smem)) return MATE_ERR_CUDA;
-  const int grid = std::min(p.num_tiles, device_sms());
-  gemm_bf16_tc_kernel<<<grid, kGemmThreads, smem, st>>>(ta, tb, p);
+  if (!make_tmap(&ta, A, M, K, lda, 128) || !make_tmap(&tb, Bw, N, K, ldb, p.bn / 2)) return MATE_ERR_CUDA;
+  const size_t smem = 1024 + (size_t)p.stages * psb + 256;
+  if (!set_smem(gemm_bf16_pair_kernel, smem)) return MATE_ERR_CUDA;
+  const int pairs = std::min(p.num_tiles, device_sms() / 2);
+  gemm_bf16_pair_kernel<<<2 * pairs, kGemmThreads, smem, st>>>(ta, tb, p);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }
