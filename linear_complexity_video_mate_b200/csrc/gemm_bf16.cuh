@@ -208,7 +208,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nk = p.K / kGemmBK;
-  const int half_bn = p.bn / 2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -238,13 +237,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
         const int mb = tile / p.num_n_tiles, nb = tile % p.num_n_tiles;
+        // the pair MMA takes B rows [0, n_mma/2) from each CTA: CTA 1 holds tile columns from n_mma/2 on
+        const int n_mma = min(p.bn, (p.N - nb * p.bn + 15) & ~15);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           uint8_t* sa = smem + stage * stage_bytes;
           const uint32_t full_leader = map_to_cta(&full[stage], 0);
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
           tma_load_2d_pair(&tmA, full_leader, sa, kb * kGemmBK, mb * 256 + rank * 128);
-          tma_load_2d_pair(&tmB, full_leader, sa + 128 * 128, kb * kGemmBK, nb * p.bn + rank * half_bn);
+          tma_load_2d_pair(&tmB, full_leader, sa + 128 * 128, kb * kGemmBK, nb * p.bn + rank * (n_mma / 2));
           if (++stage == (uint32_t)p.stages) { stage = 0; phase ^= 1; }
         }
       }

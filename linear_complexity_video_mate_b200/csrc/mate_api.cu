@@ -313,7 +313,7 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   p.y_bstride = y_bstride;
   const size_t smem_gram = 1024 + 98304 + 2048 + 64;
   const size_t smem_state = 1024 + 131072 + 2048 + 64 + 2048 + 64;
-  const size_t smem_out = 1024 + 196608 + (5 * 256 + 2048 + 16) * 4 + 2048 + 64;
+  const size_t smem_out = 1024 + kOutSmem;
   if (!set_smem(ssd_gram_kernel, smem_gram) || !set_smem(ssd_state_kernel, smem_state) ||
       !set_smem(ssd_output_kernel, smem_out))
     return MATE_ERR_CUDA;
@@ -325,7 +325,16 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   MATE_LAUNCH_CHECK();
   ssd_carry_kernel<<<dim3(kSsdP * kSsdN / 8 / 128, c->nh, 2 * c->B), 128, 0, st>>>(p);
   MATE_LAUNCH_CHECK();
-  ssd_output_kernel<<<dim3(p.nVc, c->B, c->nh), kSsdOutThreads, smem_out, st>>>(p);
+  SsdOutMaps mp;
+  const long long vrows = (long long)c->B * rows.v_bstride;
+  mp.rows = static_cast<int>(vrows);
+  const long long srows = (long long)c->B * p.nVc * c->nh * kSsdN;
+  if (!make_tmap(&mp.x, rows.xv, vrows, (long long)c->nh * c->P, rows.ldxv, 1) ||
+      !make_tmap(&mp.c, rows.cv, vrows, c->N, rows.ldcv, 1) || !make_tmap(&mp.hf, sc.Hf, srows, kSsdP, kSsdP, 128) ||
+      !make_tmap(&mp.hb, sc.Hb, srows, kSsdP, kSsdP, 128))
+    return MATE_ERR_CUDA;
+  const int out_items = c->B * p.nVc * c->nh * 2;
+  ssd_output_kernel<<<std::min(out_items, device_sms()), kSsdOutThreads, smem_out, st>>>(p, mp);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }

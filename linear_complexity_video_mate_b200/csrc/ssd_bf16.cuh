@@ -442,257 +442,341 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 }
 
 // ---------------------------------------------------------------------------------------------------
-// Outputs of one video chunk and head.  grid (nVc, B, nh), 256 threads (8 warps).
+// Outputs of the video chunks: persistent, warp-specialised.  One work item = (sample, video chunk, head,
+// 128-row tile t of the chunk); a CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ...
 //
-// The Q x Q coefficient matrix M_ij = G_ij delta_j dec(i, j) is built one 128-row tile at a time in
-// shared memory (bf16, K-major) from the bf16 G of the chunk.  The decay factors are exact products of
-// cumulative-sum exponentials; only the 64 x 64 diagonal blocks need one exponential per element.  For a
-// 64-row block ib and a column j of an EARLIER block (forward direction, j < i) the reference index
-// k = 64 ib - 1 lies between them, so
-//     exp(s_i - s_j) = exp(s_i - s_k) * exp(s_k - s_j)      (both exponents <= 0),
-// a per-row factor times a per-(ib, j) column factor.  Columns of LATER blocks (backward direction) use
-// k' = 64 (ib + 1):  exp(s'_j - s'_i) = exp(s'_j - s'_k') * exp(s'_k' - s'_i).
-// TMEM columns: [t*64, +64) sum_j M_ij x_j for row tile t; [128 + t*64, +64) C Hf^T; [256 + t*64, +64)
-// C Hb^T.
+//   warps 0..3   loaders: gather the item's x rows (all 256, MN-major), C rows of the tile (K-major) and
+//                the incoming states Hf / Hb (MN-major) into one of two shared-memory buffers with
+//                cp.async; compute the cumulative sums and the decay factor tables of the item.
+//   warps 4..11  transform (two warps per TMEM lane quadrant, alternating 8-column chunks): read the
+//                tile's 128 rows of G = C B^T (bf16, global/L2), form
+//                M_ij = G_ij delta_j dec(i, j) (diagonal excluded) and store M straight into TMEM as
+//                the A operand of the next MMA (two bf16 per 32-bit column).
+//   MMA issue    lane 0 of warp 4, once all transform warps stored M: Yd = M x (A from TMEM),
+//                Yf = C Hf^T, Yb = C Hb^T into one of two TMEM accumulator sets.  (16 warps in total: a
+//                17th warp would put 5 warps on one SM sub-partition, beyond its register file.)
+//   warps 12..15 epilogue: y_i = Yd + exp(s_i) Yf + exp(s_last - s'_i) Yb + 2 (D + G_ii delta_i) x_i,
+//                stored at the grid-order row of the token.
+//
+// Decay factors: for a 64-row block ib and a column j of an EARLIER 64-block (forward direction), the
+// reference k = 64 ib - 1 lies between them, so exp(s_i - s_j) = exp(s_i - s_k) exp(s_k - s_j) (both
+// exponents <= 0): a per-row factor times a per-(ib, j) column factor.  Columns of LATER blocks use
+// k' = 64 (ib + 1) with the exclusive sums.  Only the 64 x 64 diagonal blocks need one exponential per
+// element.
+// TMEM columns: [0, 128) M; accumulator set a at 128 + 192 a: Yd [+0, +64), Yf [+64, +128), Yb [+128, +192).
 // ---------------------------------------------------------------------------------------------------
-constexpr int kSsdOutThreads = 512;
+constexpr int kOutLoadWarps = 4, kOutXformWarps = 8, kOutEpiWarps = 4;
+constexpr int kOutMmaWarp = kOutLoadWarps;                                    // issues from its lane 0
+constexpr int kSsdOutThreads = (kOutLoadWarps + kOutXformWarps + kOutEpiWarps) * 32;   // 512
+constexpr uint32_t kOutBuf = 108544;                                         // bytes per operand buffer
+constexpr uint32_t kOutOffC = 32768, kOutOffHf = 65536, kOutOffHb = 81920, kOutOffTbl = 98304;
+constexpr uint32_t kOutSmem = 2 * kOutBuf + 256;
 
-__global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const SsdBf16Params p) {
+// Tensor maps of the output kernel: x and C rows of the video arrays (one-row boxes of 64 columns, for
+// four-row gathers) and the carried states ([N rows][P] per chunk and head, 64 x 128 boxes).
+struct SsdOutMaps {
+  CUtensorMap x, c, hf, hb;
+  int rows;   // row extent of the x / C maps; gathers of invalid rows use this (out of range -> zeros)
+};
+
+struct OutTables {   // per buffer, at kOutOffTbl
+  float sdl[256], ss[256], ssx[256];
+  float uf[128], ub[128];       // per tile row
+  float wf[2][256], wb[2][256]; // per 64-row block of the tile (ib = 2t + q)
+  int srow[256];                // source row of each chunk row (-1 past the end of a partial chunk)
+  float wtot[4];
+};
+
+__global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const SsdBf16Params p,
+                                                                        const __grid_constant__ SsdOutMaps mp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sM = smem;                 // [128 i][256 j] K-major, K blocks 16 KB apart (G tile, then M tile)
-  uint8_t* sX = smem + 65536;         // [256 j][64 p] MN-major
-  uint8_t* sC = smem + 98304;         // [256 i][128 n] K-major, K blocks 32 KB apart
-  uint8_t* sHf = smem + 163840;       // [128 n][64 p] MN-major (B operand of C H^T with K = n)
-  uint8_t* sHb = smem + 180224;
-  float* sdl = reinterpret_cast<float*>(smem + 196608);
-  float* ss = sdl + 256;              // inclusive cumulative sums s_i
-  float* ssx = ss + 256;              // exclusive sums s'_i = s_i - a_i
-  float* uf = ssx + 256;              // per-row forward factor exp(s_i - s_{64 ib - 1})
-  float* ub = uf + 256;               // per-row backward factor exp(s'_{64 ib + 64} - s'_i)
-  float* wf = ub + 256;               // [4][256] delta_j exp(s_{64 ib - 1} - s_j), j < 64 ib
-  float* wb = wf + 1024;              // [4][256] delta_j exp(s'_j - s'_{64 ib + 64}), j >= 64 ib + 64
-  float* wtot = wb + 1024;            // [16]
-  long long* srow = reinterpret_cast<long long*>(wtot + 16);   // [256]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(srow + 256);
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
-  const int v = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
-  const int c = p.nRc + v;
-  const ChunkBase cb = chunk_base(p.s, c, p.nRc);
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  constexpr int PN = kSsdP * kSsdN;
-  constexpr int NT = kSsdOutThreads;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kOutBuf);
+  uint64_t* ld_full = bars;        // [2] loaders -> consumers (count 128)
+  uint64_t* ld_empty = bars + 2;   // [2] MMA commit + epilogue warps -> loaders (count 5)
+  uint64_t* m_full = bars + 4;     // [2] per K half of M: transform -> MMA (count 256)
+  uint64_t* m_empty = bars + 6;    // [2] per K half of M: MMA commit -> transform (count 1)
+  uint64_t* y_full = bars + 8;     // [2] MMA commit -> epilogue (count 1)
+  uint64_t* y_empty = bars + 10;   // [2] epilogue warps -> MMA (count 4)
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bars + 12);
 
-  if (tid == 0) {
-    mbar_init(bar, 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nitems = p.B * p.nVc * p.nh * 2;
+
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&ld_full[q], 129);   // 128 loader threads + the byte-count arrival
+      mbar_init(&ld_empty[q], 5);
+      mbar_init(&y_full[q], 1);
+      mbar_init(&y_empty[q], 4);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&m_full[q], 256);
+      mbar_init(&m_empty[q], 1);
+    }
     mbar_fence_init();
   }
-  if (warp == 0) tmem_alloc(slot, 512);
-  fill_chunk_rows(p.s, b, c, p.nRc, srow);
-  const __nv_bfloat16* gbase = p.Gm + (static_cast<long long>(b) * p.nVc + v) * kSsdQ * kSsdQ;
-  // G rows 0..127 straight into the M tile (transformed in place below)
-  for (int it = tid; it < 128 * 32; it += NT) {
-    const int r = it >> 5, cc = it & 31;
-    cp_async16(sM + sw128_kmajor_offset(r, cc * 8, 16384), gbase + r * kSsdQ + cc * 8);
+  if (warp == kOutMmaWarp) {
+    tmem_alloc(slot, 512);
+    tmem_relinquish();
   }
-  __syncthreads();  // srow
-  for (int it = tid; it < 256 * 8; it += NT) {
-    const int r = it >> 3, ch = it & 7;
-    const long long rw = srow[r];
-    cp_async16_zfill(sX + sw128_mnmajor_offset(r, ch * 8, 32768), cb.x + (rw < 0 ? 0 : rw) * cb.ldx + h * kSsdP + ch * 8,
-                     rw >= 0);
-  }
-  for (int it = tid; it < 256 * 16; it += NT) {
-    const int r = it >> 4, ch = it & 15;
-    const long long rw = srow[r];
-    load_row128_kmajor(sC, r, cb.c + (rw < 0 ? 0 : rw) * cb.ldc, rw >= 0, 32768, ch);
-  }
-  const long long vi = (static_cast<long long>(b) * p.nVc + v) * p.nh + h;
-  for (int it = tid; it < 128 * 8; it += NT) {
-    const int r = it >> 3, ch = it & 7;
-    cp_async16(sHf + sw128_mnmajor_offset(r, ch * 8, 16384), p.Hf + vi * PN + r * kSsdP + ch * 8);
-    cp_async16(sHb + sw128_mnmajor_offset(r, ch * 8, 16384), p.Hb + vi * PN + r * kSsdP + ch * 8);
-  }
-  cp_async_commit();
-
-  // cumulative sums and decay factor tables (threads 0..255 = chunk rows)
-  const int j = tid & 255;
-  const bool data = tid < 256;
-  const long long myrw = srow[j];
-  const int len = min(kSsdQ, p.s.n - v * kSsdQ);
-  const float A = -__expf(p.A_log[h]);
-  const float dl = (data && myrw >= 0) ? cb.d[myrw * cb.ldd + h] : 0.f;
-  const float a = dl * A;
-  const float s = block_scan_256(a, wtot);
-  if (data) {
-    sdl[j] = dl;
-    ss[j] = s;
-    ssx[j] = s - a;
-  }
-  __syncthreads();
-  if (data) {
-    const int ib = j >> 6;
-    uf[j] = ib > 0 ? __expf(s - ss[64 * ib - 1]) : 0.f;
-    ub[j] = ib < 3 ? __expf(ssx[64 * ib + 64] - (s - a)) : 0.f;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      wf[q * 256 + j] = (q > 0 && j < 64 * q) ? dl * __expf(ss[64 * q - 1] - s) : 0.f;
-      wb[q * 256 + j] = (q < 3 && j >= 64 * q + 64) ? dl * __expf((s - a) - ssx[64 * q + 64]) : 0.f;
-    }
-  }
-  cp_async_wait<0>();
-  fence_proxy_async();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
 
-  if (tid == 0) {
-    const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 1);
-    const uint32_t c0 = smem_u32(sC), hf = smem_u32(sHf), hb = smem_u32(sHb);
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t off = (k & 3) * 32;
-        const uint64_t ad = desc_sw128(c0 + (k >> 2) * 32768 + t * 16384 + off, 16, 1024);
-        mma_bf16_ss(tmem + 128 + t * 64, ad, desc_sw128(hf + k * 2048, 16384, 1024), idesc, k > 0);
-        mma_bf16_ss(tmem + 256 + t * 64, ad, desc_sw128(hb + k * 2048, 16384, 1024), idesc, k > 0);
-      }
-  }
-
-  // build mapping: thread -> one row of the tile (lanes = consecutive rows: conflict-free swizzled
-  // accesses, broadcast column tables) and every fourth 16-byte column chunk
-  const int r = (warp & 3) * 32 + lane;
-  const int cg = warp >> 2;
-  // scale 8 G values of row i, columns j0..j0+7 (one 64-block) into M values
-  auto transform = [&](uint4 g8, int i, int j0) -> uint4 {
-    const int ib = i >> 6, jb = j0 >> 6;
-    const uint32_t* gu = reinterpret_cast<const uint32_t*>(&g8);
-    uint4 o;
-    uint32_t* ou = reinterpret_cast<uint32_t*>(&o);
-    if (jb != ib) {
-      const float u = jb < ib ? uf[i] : ub[i];
-      const float4* w4 = reinterpret_cast<const float4*>((jb < ib ? wf : wb) + ib * 256 + j0);
-      const float4 wa = w4[0], wc = w4[1];
-      const float w[8] = {wa.x, wa.y, wa.z, wa.w, wc.x, wc.y, wc.z, wc.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 g = unpack_bf16x2(gu[e]);
-        ou[e] = pack_bf16x2(g.x * u * w[2 * e], g.y * u * w[2 * e + 1]);
-      }
-    } else {
-      const float si = ss[i], sxi = ssx[i];
-      const float4* s4 = reinterpret_cast<const float4*>(ss + j0);
-      const float4* x4 = reinterpret_cast<const float4*>(ssx + j0);
-      const float4* d4 = reinterpret_cast<const float4*>(sdl + j0);
-      const float4 sa = s4[0], sb = s4[1], xa = x4[0], xb = x4[1], da = d4[0], db = d4[1];
-      const float sj[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-      const float xj[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-      const float dj[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 g = unpack_bf16x2(gu[e]);
-        float m2[2];
-#pragma unroll
-        for (int z = 0; z < 2; ++z) {
-          const int k = 2 * e + z, jj = j0 + k;
-          // the diagonal (j = i) is added in fp32 in the epilogue
-          const float dec = jj < i ? __expf(si - sj[k]) : (jj > i ? __expf(xj[k] - sxi) : 0.f);
-          m2[z] = (z == 0 ? g.x : g.y) * dj[k] * dec;
-        }
-        ou[e] = pack_bf16x2(m2[0], m2[1]);
-      }
-    }
-    return o;
+  auto decode = [&](int it, int& b, int& v, int& h, int& t) {
+    t = it & 1;
+    int rest = it >> 1;
+    h = rest % p.nh;
+    rest /= p.nh;
+    v = rest % p.nVc;
+    b = rest / p.nVc;
   };
 
-  // row tile 0: G already in sM, transform in place
+  if (warp < kOutLoadWarps) {
+    // ------------------------------------------------------------------------------ loaders
+    const int lt = threadIdx.x;  // 0..127
+    int k = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
+      const int buf = k & 1, use = k >> 1;
+      if (!mbar_wait(&ld_empty[buf], (use & 1) ^ 1)) break;
+      int b, v, h, t;
+      decode(it, b, v, h, t);
+      const int c = p.nRc + v;
+      const ChunkBase cb = chunk_base(p.s, c, p.nRc);
+      uint8_t* B0 = smem + buf * kOutBuf;
+      OutTables& tb = *reinterpret_cast<OutTables*>(B0 + kOutOffTbl);
+      for (int j = lt; j < 256; j += 128) {
+        const RowRef rr = chunk_row(p.s, b, c, p.nRc, j);
+        tb.srow[j] = rr.valid ? static_cast<int>(rr.r) : -1;
+      }
+      if (lt == 0) mbar_arrive_expect_tx(&ld_full[buf], 3 * 32768);   // x (32 KB), C (32 KB), Hf + Hb (32 KB)
+      named_bar_sync(1, 128);
+      // TMA: x rows (all 256, 4 per gather), C rows of the tile (2 column blocks), the two states
+      auto rowid = [&](int j) { const int rw = tb.srow[j]; return rw < 0 ? mp.rows : rw; };
+      if (lt < 64) {
+        const int g = lt;
+        tma_gather4(&mp.x, &ld_full[buf], B0 + g * 512, h * kSsdP, rowid(4 * g), rowid(4 * g + 1), rowid(4 * g + 2),
+                    rowid(4 * g + 3));
+      } else {
+        const int g = (lt - 64) & 31, kb = (lt - 64) >> 5;
+        const int j = t * 128 + 4 * g;
+        tma_gather4(&mp.c, &ld_full[buf], B0 + kOutOffC + kb * 16384 + g * 512, kb * 64, rowid(j), rowid(j + 1),
+                    rowid(j + 2), rowid(j + 3));
+      }
+      if (lt == 0) {
+        const int hrow = static_cast<int>(((static_cast<long long>(b) * p.nVc + v) * p.nh + h) * kSsdN);
+        tma_load_2d(&mp.hf, &ld_full[buf], B0 + kOutOffHf, 0, hrow);
+        tma_load_2d(&mp.hb, &ld_full[buf], B0 + kOutOffHb, 0, hrow);
+      }
+      // cumulative sums: thread lt owns rows 2 lt and 2 lt + 1
+      const float A = -__expf(p.A_log[h]);
+      float dl[2], a[2];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int cc = cg + 4 * k;
-    uint4* loc = reinterpret_cast<uint4*>(sM + sw128_kmajor_offset(r, cc * 8, 16384));
-    *loc = transform(*loc, r, cc * 8);
-  }
-  fence_proxy_async();
-  __syncthreads();
-  if (tid == 0) {
-    tc_fence_after();
-    const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 1);
-    const uint32_t m0 = smem_u32(sM), x0 = smem_u32(sX);
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k)
-      mma_bf16_ss(tmem, desc_sw128(m0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                  desc_sw128(x0 + k * 2048, 32768, 1024), idesc, k > 0);
-    mma_commit(bar);
-  }
-  // row tile 1: G rows 128..255 fetched into registers while tile 0 multiplies
-  uint4 g1[8];
+      for (int e = 0; e < 2; ++e) {
+        const int rw = tb.srow[2 * lt + e];
+        dl[e] = rw >= 0 ? cb.d[static_cast<long long>(rw) * cb.ldd + h] : 0.f;
+        a[e] = dl[e] * A;
+      }
+      float incl = a[0] + a[1];
 #pragma unroll
-  for (int k = 0; k < 8; ++k)
-    g1[k] = __ldg(reinterpret_cast<const uint4*>(gbase + (128 + r) * kSsdQ + (cg + 4 * k) * 8));
-  mbar_wait(bar, 0);
-  tc_fence_after();
+      for (int off = 1; off < 32; off <<= 1) {
+        const float u2 = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u2;
+      }
+      if (lane == 31) tb.wtot[warp] = incl;
+      named_bar_sync(1, 128);
+      for (int w = 0; w < warp; ++w) incl += tb.wtot[w];
+      const float s1 = incl, s0 = incl - a[1];
+      tb.sdl[2 * lt] = dl[0];
+      tb.sdl[2 * lt + 1] = dl[1];
+      tb.ss[2 * lt] = s0;
+      tb.ss[2 * lt + 1] = s1;
+      tb.ssx[2 * lt] = s0 - a[0];
+      tb.ssx[2 * lt + 1] = s1 - a[1];
+      named_bar_sync(1, 128);
+      {
+        const int i = t * 128 + lt, ib = i >> 6;
+        tb.uf[lt] = ib > 0 ? __expf(tb.ss[i] - tb.ss[64 * ib - 1]) : 0.f;
+        tb.ub[lt] = ib < 3 ? __expf(tb.ssx[64 * ib + 64] - tb.ssx[i]) : 0.f;
+      }
+      for (int j = lt; j < 256; j += 128) {
+        const float dj = tb.sdl[j], sj = tb.ss[j], sxj = tb.ssx[j];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int cc = cg + 4 * k;
-    *reinterpret_cast<uint4*>(sM + sw128_kmajor_offset(r, cc * 8, 16384)) = transform(g1[k], 128 + r, cc * 8);
-  }
-  fence_proxy_async();
-  __syncthreads();
-  if (tid == 0) {
-    tc_fence_after();
-    const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 1);
-    const uint32_t m0 = smem_u32(sM), x0 = smem_u32(sX);
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k)
-      mma_bf16_ss(tmem + 64, desc_sw128(m0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                  desc_sw128(x0 + k * 2048, 32768, 1024), idesc, k > 0);
-    mma_commit(bar);
-  }
-  mbar_wait(bar, 1);
-  tc_fence_after();
-
-  // epilogue: warp w -> TMEM lane quadrant w%4, row tile (w/4)%2, 32-column half w/8
-  const int quad = warp & 3, t = (warp >> 2) & 1, pc = warp >> 3;
-  const int i = t * 128 + quad * 32 + lane;
-  const bool ok = i < len;
-  const float ef = __expf(ss[i]);
-  const float eb = __expf(ss[255] - ssx[i]);
-  // diagonal of both directions (weight 1 each) plus the two skip terms, in fp32
-  const float D2 = 2.f * (p.Dp[h] + (ok ? p.Gd[(static_cast<long long>(b) * p.nVc + v) * kSsdQ + i] * sdl[i] : 0.f));
-  __nv_bfloat16* yrow = p.y + (b * p.y_bstride + p.s.map(v * kSsdQ + (ok ? i : 0))) * p.ldy + h * kSsdP;
-  const uint32_t lanebase = static_cast<uint32_t>(quad * 32) << 16;
-  {
-    uint32_t yd[32], yf[32], yb[32];
-    tmem_ld32(tmem + lanebase + t * 64 + pc * 32, yd);
-    tmem_ld32(tmem + lanebase + 128 + t * 64 + pc * 32, yf);
-    tmem_ld32(tmem + lanebase + 256 + t * 64 + pc * 32, yb);
-    tmem_wait_ld();
-    if (ok) {
-      uint4 out[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128_mnmajor_offset(i, pc * 32 + q * 8, 32768));
-        const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
-        uint32_t* ou = reinterpret_cast<uint32_t*>(&out[q]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 xf = unpack_bf16x2(xu[e]);
-          const int k0 = q * 8 + 2 * e;
-          const float y0 = __uint_as_float(yd[k0]) + ef * __uint_as_float(yf[k0]) + eb * __uint_as_float(yb[k0]) + D2 * xf.x;
-          const float y1 = __uint_as_float(yd[k0 + 1]) + ef * __uint_as_float(yf[k0 + 1]) +
-                           eb * __uint_as_float(yb[k0 + 1]) + D2 * xf.y;
-          ou[e] = pack_bf16x2(y0, y1);
+        for (int q = 0; q < 2; ++q) {
+          const int ib = 2 * t + q;
+          tb.wf[q][j] = (ib > 0 && j < 64 * ib) ? dj * __expf(tb.ss[64 * ib - 1] - sj) : 0.f;
+          tb.wb[q][j] = (ib < 3 && j >= 64 * ib + 64) ? dj * __expf(sxj - tb.ssx[64 * ib + 64]) : 0.f;
         }
       }
-      uint4* dst = reinterpret_cast<uint4*>(yrow + pc * 32);
+      mbar_arrive(&ld_full[buf]);
+    }
+  } else if (warp < kOutLoadWarps + kOutXformWarps) {
+    // ------------------------------------------------------------------------------ transform
+    const int xw = warp - kOutLoadWarps;
+    const int quad = warp & 3, half = xw >> 2;
+    const int r = quad * 32 + lane;
+    int k = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
+      const int buf = k & 1, use = k >> 1;
+      int b, v, h, t;
+      decode(it, b, v, h, t);
+      const int i = t * 128 + r, ib = i >> 6;
+      // the two warps of a lane quadrant take alternating 8-column chunks of the row, so both get half of
+      // the diagonal block's exponentials
+      const __nv_bfloat16* grow = p.Gm + ((static_cast<long long>(b) * p.nVc + v) * kSsdQ + i) * kSsdQ + half * 8;
+      // the row's 16 chunks of G (8 bf16 each, 256 bytes) are all in flight before the waits and are
+      // consumed in order through a shifting register window (keeps the chunk loop rolled: the four roles'
+      // code must share the instruction cache)
+      const uint4* gsrc = reinterpret_cast<const uint4*>(grow);
+      uint4 gw[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = out[q];
+      for (int q = 0; q < 16; ++q) gw[q] = __ldg(gsrc + 2 * q);
+      if (!mbar_wait(&ld_full[buf], use & 1)) break;
+      const OutTables& tb = *reinterpret_cast<const OutTables*>(smem + buf * kOutBuf + kOutOffTbl);
+      const float ufi = tb.uf[r], ubi = tb.ub[r], si = tb.ss[i], sxi = tb.ssx[i];
+      const float* wfr = tb.wf[ib - 2 * t];
+      const float* wbr = tb.wb[ib - 2 * t];
+      const uint32_t tm_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 4;
+      const int acc = k & 1;
+      bool ok = true, mma_ok = true;
+      // M is produced and consumed in two K halves (TMEM columns [0, 64) and [64, 128)): the MMAs of the
+      // first half run while the second half is being formed
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        if (!mbar_wait(&m_empty[hh], (k & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int q = 8 * hh; q < 8 * hh + 8; ++q) {
+          const uint4 gc = gw[0];
+#pragma unroll
+          for (int z = 0; z < 15; ++z) gw[z] = gw[z + 1];
+          const int j0 = (2 * q + half) * 8;
+          const int jb = j0 >> 6;   // same for the whole warp (all lanes are rows of one 64-block)
+          const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gc);
+          uint32_t pk[4];
+          if (jb != ib) {
+            const float u = jb < ib ? ufi : ubi;
+            const float* w = (jb < ib ? wfr : wbr) + j0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 gf = unpack_bf16x2(gu[e]);
+              const float2 w2 = *reinterpret_cast<const float2*>(w + 2 * e);
+              pk[e] = pack_bf16x2(gf.x * (u * w2.x), gf.y * (u * w2.y));
+            }
+          } else {
+            // one exponential per element: forward weight below the diagonal, backward above; the
+            // diagonal itself is added in fp32 in the epilogue
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int jj = j0 + 2 * e;
+              const float2 gf = unpack_bf16x2(gu[e]);
+              const float2 sj = *reinterpret_cast<const float2*>(tb.ss + jj);
+              const float2 xj = *reinterpret_cast<const float2*>(tb.ssx + jj);
+              const float2 dj = *reinterpret_cast<const float2*>(tb.sdl + jj);
+              const float f0 = jj == i ? 0.f : dj.x * __expf(jj < i ? si - sj.x : xj.x - sxi);
+              const float f1 = jj + 1 == i ? 0.f : dj.y * __expf(jj + 1 < i ? si - sj.y : xj.y - sxi);
+              pk[e] = pack_bf16x2(gf.x * f0, gf.y * f1);
+            }
+          }
+          tmem_st4(tm_row + q * 8, pk[0], pk[1], pk[2], pk[3]);   // columns of chunk 2q + half
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&m_full[hh]);
+        if (warp == kOutMmaWarp) {
+          if (lane == 0) {
+            // -------------------------------------------------------------------- MMA issue
+            const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 1);
+            if (hh == 0) mma_ok = mbar_wait(&y_empty[acc], (use & 1) ^ 1);
+            mma_ok = mma_ok && mbar_wait(&m_full[hh], k & 1);
+            if (mma_ok) {
+              tc_fence_after();
+              const uint32_t b0 = smem_u32(smem + buf * kOutBuf);
+              const uint32_t ybase = tmem + 128 + acc * 192;
+#pragma unroll
+              for (int q = 8 * hh; q < 8 * hh + 8; ++q)   // Yd = M x (M in TMEM, 8 columns per 16 elements)
+                mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(b0 + q * 2048, 32768, 1024), idesc, q > 0);
+              mma_commit(&m_empty[hh]);
+              if (hh == 1) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {  // Yf = C Hf^T, Yb = C Hb^T, K = N = 128
+                  const uint64_t ad = desc_sw128(b0 + kOutOffC + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024);
+                  mma_bf16_ss(ybase + 64, ad, desc_sw128(b0 + kOutOffHf + q * 2048, 16384, 1024), idesc, q > 0);
+                  mma_bf16_ss(ybase + 128, ad, desc_sw128(b0 + kOutOffHb + q * 2048, 16384, 1024), idesc, q > 0);
+                }
+                mma_commit(&y_full[acc]);
+                mma_commit(&ld_empty[buf]);
+              }
+            }
+          }
+          __syncwarp();
+        }
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    int k = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
+      const int buf = k & 1, acc = k & 1, use = k >> 1;
+      int b, v, h, t;
+      decode(it, b, v, h, t);
+      if (!mbar_wait(&y_full[acc], use & 1)) break;
+      tc_fence_after();
+      const uint8_t* B0 = smem + buf * kOutBuf;
+      const OutTables& tb = *reinterpret_cast<const OutTables*>(B0 + kOutOffTbl);
+      const int i = t * 128 + r;
+      const int len = min(kSsdQ, p.s.n - v * kSsdQ);
+      const bool ok = i < len;
+      const float si = tb.ss[i], sxi = tb.ssx[i], slast = tb.ss[255], dli = tb.sdl[i];
+      // x row of this token (packed bf16 pairs) for the skip and diagonal terms
+      uint32_t xw[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(B0 + sw128_mnmajor_offset(i, q * 8, 32768));
+        xw[q * 4 + 0] = xv.x; xw[q * 4 + 1] = xv.y; xw[q * 4 + 2] = xv.z; xw[q * 4 + 3] = xv.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ld_empty[buf]);
+      const float ef = __expf(si);
+      const float eb = __expf(slast - sxi);
+      const float D2 = 2.f * (p.Dp[h] + (ok ? p.Gd[(static_cast<long long>(b) * p.nVc + v) * kSsdQ + i] * dli : 0.f));
+      __nv_bfloat16* yrow = p.y + (b * p.y_bstride + p.s.map(v * kSsdQ + (ok ? i : 0))) * p.ldy + h * kSsdP;
+      const uint32_t ybase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128 + acc * 192;
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {   // 16 columns at a time
+        uint32_t yd[16], yf[16], yb[16];
+        tmem_ld16(ybase + pc * 16, yd);
+        tmem_ld16(ybase + 64 + pc * 16, yf);
+        tmem_ld16(ybase + 128 + pc * 16, yb);
+        tmem_wait_ld();
+        if (ok) {
+          uint32_t ou[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 xf = unpack_bf16x2(xw[pc * 8 + e]);
+            const int k0 = 2 * e;
+            const float y0 = __uint_as_float(yd[k0]) + ef * __uint_as_float(yf[k0]) + eb * __uint_as_float(yb[k0]) + D2 * xf.x;
+            const float y1 = __uint_as_float(yd[k0 + 1]) + ef * __uint_as_float(yf[k0 + 1]) +
+                             eb * __uint_as_float(yb[k0 + 1]) + D2 * xf.y;
+            ou[e] = pack_bf16x2(y0, y1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(yrow + pc * 16);
+          dst[0] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+          dst[1] = make_uint4(ou[4], ou[5], ou[6], ou[7]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&y_empty[acc]);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kOutMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

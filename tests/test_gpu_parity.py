@@ -209,6 +209,21 @@ def test_mate_forward(name, layer, variant):
     _check_block(cfg, w, layer, variant, out)
 
 
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+@pytest.mark.parametrize("branch", ["te", "ma"])
+@pytest.mark.parametrize("name", ["bf16_small_8x16x16", "bf16_ragged_12x16x24", "bf16_b2_20x16x16_d512"])
+def test_mate_forward_single_branch(name, branch, layer):
+    """Each branch alone (the other branch's output projection zeroed).  The TE branch's output is not
+    heavy-tailed, so its bf16-storage floor stays below 2e-2 and the strict bound applies."""
+    cfg = mi.all_configs()[name]
+    w = dict(_block(cfg, "default"))
+    zero = "W_out" if branch == "te" else "W_o"
+    w[zero] = np.zeros_like(w[zero])
+    blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
+    out = host(blk.forward(dev(w["X"], tdt(cfg)), layer))
+    _check_block(cfg, w, layer, f"{branch}only", out)
+
+
 def test_mate_forward_host_matches_device_path():
     cfg = mi.TEST_CONFIGS["bf16_small_8x16x16"]
     w = _block(cfg, "default")
