@@ -445,9 +445,10 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 // Outputs of the video chunks: persistent, warp-specialised.  One work item = (sample, video chunk, head,
 // 128-row tile t of the chunk); a CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ...
 //
-//   warps 0..3   loaders: gather the item's x rows (all 256, MN-major), C rows of the tile (K-major) and
-//                the incoming states Hf / Hb (MN-major) into one of two shared-memory buffers with
-//                cp.async; compute the cumulative sums and the decay factor tables of the item.
+//   warps 0..3   loaders: gather the item's x rows (all 256, MN-major) and the C rows of the tile
+//                (K-major) with TMA four-row gathers (tile::gather4), load the incoming states Hf / Hb
+//                (MN-major) with 2D TMA, into one of two shared-memory buffers; compute the cumulative
+//                sums and the decay factor tables of the item.
 //   warps 4..11  transform (two warps per TMEM lane quadrant, alternating 8-column chunks): read the
 //                tile's 128 rows of G = C B^T (bf16, global/L2), form
 //                M_ij = G_ij delta_j dec(i, j) (diagonal excluded) and store M straight into TMEM as
