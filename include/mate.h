@@ -52,7 +52,8 @@ typedef enum {
   MATE_ERR_WORKSPACE = 3,   /* ws_bytes smaller than the queried workspace size */
   MATE_ERR_CUDA = 4,        /* a CUDA launch or copy failed (cudaGetLastError after the launch) */
   MATE_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (reported by mate_device_status) */
-  MATE_ERR_UNSUPPORTED = 6  /* valid shape that the bf16 tensor-core kernels do not cover */
+  MATE_ERR_UNSUPPORTED = 6, /* valid shape that the bf16 tensor-core kernels do not cover */
+  MATE_ERR_TOO_LARGE = 7    /* problem needs more scratch than the library's fixed device buffer holds */
 } mate_status;
 
 typedef enum { MATE_BF16 = 0, MATE_F32 = 1 } mate_dtype;
@@ -138,6 +139,41 @@ MATE_API mate_status review_pool(const void* X, void* Rv, int order, const mate_
 MATE_API mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const float* dt, const float* dt_bias,
                            const float* A_log, const float* D, int prefix_len, void* y, const mate_config* cfg,
                            void* ws, size_t ws_bytes, mate_stream_t stream);
+
+/* Size of the fixed device scratch buffer behind ssd_scan_bidir_noalloc: 32 MiB. */
+#define MATE_SSD_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * ssd_scan_bidir for callers that must not allocate device memory.  The paper has no counterpart to
+ * this entry point; it computes exactly what ssd_scan_bidir computes, with the same arguments minus
+ * the workspace.  It exists for callers that are handed their input and output buffers but may not
+ * create device allocations of their own: a plugin inside a host framework that owns every device
+ * allocation, or a latency-bound serving loop where cudaMalloc and cudaFree would synchronise the
+ * device and stall work on other streams.  Such callers can neither size nor own a workspace.
+ *
+ * Scratch: instead of a caller workspace the scan uses one fixed array of
+ * MATE_SSD_NOALLOC_SCRATCH_BYTES bytes in device global memory, part of this library's device code.
+ * Every GPU on which the library's device code is loaded holds that array until the process exits.
+ * A problem with mate_ssd_workspace_bytes(cfg, prefix_len) > MATE_SSD_NOALLOC_SCRATCH_BYTES is
+ * rejected with MATE_ERR_TOO_LARGE before any device work (with the bf16 kernels, nh = 16, B = 1 and
+ * 128 prefix rows, that admits up to about 7 000 video tokens).
+ *
+ * Set-up: the first call on a device (the device current at the call) looks up the array's device
+ * address once, which can load the library's device code onto that device; make that first call
+ * before any stream capture on the device.  Later calls on the device reuse the address.
+ *
+ * Sharing: all calls on one device use the same array, and it keeps what the last call left in it.
+ * Each call writes every scratch byte it reads before reading it, so nothing needs clearing between
+ * calls.  Calls whose executions overlap on the GPU (on streams with no ordering between them, from
+ * one host thread or several) race on the array and give wrong results; calls on one stream run one
+ * after the other and are safe.
+ *
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine is called.  Errors as
+ * ssd_scan_bidir, plus MATE_ERR_TOO_LARGE; MATE_ERR_CUDA if the address look-up fails.
+ */
+MATE_API mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const void* Cm, const float* dt,
+                                            const float* dt_bias, const float* A_log, const float* D, int prefix_len,
+                                            void* y, const mate_config* cfg, mate_stream_t stream);
 
 /*
  * TEmporal Swin Attention ([NEWS] TESA paragraph; [FEAT] TESA): window attention on qkv

@@ -5,7 +5,9 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmate.so")
 
-MATE_OK, MATE_ERR_ARG, MATE_ERR_SHAPE, MATE_ERR_WORKSPACE, MATE_ERR_CUDA, MATE_ERR_TIMEOUT, MATE_ERR_UNSUPPORTED = range(7)
+(MATE_OK, MATE_ERR_ARG, MATE_ERR_SHAPE, MATE_ERR_WORKSPACE, MATE_ERR_CUDA, MATE_ERR_TIMEOUT, MATE_ERR_UNSUPPORTED,
+ MATE_ERR_TOO_LARGE) = range(8)
+MATE_SSD_NOALLOC_SCRATCH_BYTES = 32 << 20
 MATE_BF16, MATE_F32 = 0, 1
 
 # every symbol include/mate.h declares
@@ -13,6 +15,7 @@ EXPORTS = (
     "mate_status_str", "mate_check_config", "mate_workspace_bytes", "mate_ssd_workspace_bytes", "rms_permute",
     "rms_unpermute", "review_pool", "ssd_scan_bidir", "tesa_forward", "mate_forward", "mate_forward_host",
     "mate_forward_host_workspace_bytes", "mate_device_status", "mate_last_launch_count", "mate_project_bf16",
+    "ssd_scan_bidir_noalloc",
 )
 
 _CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp", "wt", "wh", "ww", "st", "sh", "sw")
@@ -56,6 +59,7 @@ def load():
         "rms_unpermute": (ci, [vp, vp, ci, cfgp, vp]),
         "review_pool": (ci, [vp, vp, ci, cfgp, vp]),
         "ssd_scan_bidir": (ci, [vp, vp, vp, vp, vp, vp, vp, ci, vp, cfgp, vp, sz, vp]),
+        "ssd_scan_bidir_noalloc": (ci, [vp, vp, vp, vp, vp, vp, vp, ci, vp, cfgp, vp]),
         "tesa_forward": (ci, [vp, vp, ci, cfgp, vp]),
         "mate_forward": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
         "mate_forward_host": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/mate.h"
 #include "common.cuh"
@@ -470,6 +471,7 @@ const char* mate_status_str(mate_status s) {
     case MATE_ERR_CUDA: return "CUDA error";
     case MATE_ERR_TIMEOUT: return "device wait timed out";
     case MATE_ERR_UNSUPPORTED: return "shape not supported by the tensor-core kernels";
+    case MATE_ERR_TOO_LARGE: return "problem needs more scratch than the fixed device buffer holds";
   }
   return "unknown status";
 }
@@ -553,6 +555,45 @@ mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const 
   rows.W = cfg->W;
   rows.order = -1;
   return run_ssd(cfg, rows, A_log, D, y, cfg->nh * cfg->P, n, sc, st);
+}
+
+// Fixed scratch behind ssd_scan_bidir_noalloc.  In host code this name is only a stand-in for the
+// device symbol; its device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_ssd_noalloc_scratch[MATE_SSD_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoallocMaxDevices = 128;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNoallocMaxDevices];  // device address of the scratch, by device ordinal
+}  // namespace
+
+mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const void* Cm, const float* dt,
+                                   const float* dt_bias, const float* A_log, const float* D, int prefix_len, void* y,
+                                   const mate_config* cfg, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (prefix_len < 0) return MATE_ERR_ARG;
+  if (ssd_ws_bytes(cfg, prefix_len, nullptr, nullptr, nullptr) > MATE_SSD_NOALLOC_SCRATCH_BYTES)
+    return MATE_ERR_TOO_LARGE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) {
+    cudaGetLastError();
+    return MATE_ERR_CUDA;
+  }
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_ssd_noalloc_scratch) != cudaSuccess || addr == nullptr) {
+        cudaGetLastError();
+        return MATE_ERR_CUDA;
+      }
+      g_noalloc_addr[dev] = addr;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  return ssd_scan_bidir(x, Bm, Cm, dt, dt_bias, A_log, D, prefix_len, y, cfg, scratch, MATE_SSD_NOALLOC_SCRATCH_BYTES,
+                        stream);
 }
 
 mate_status tesa_forward(const void* qkv, void* O, int shifted, const mate_config* cfg, mate_stream_t stream) {

@@ -151,6 +151,16 @@ def ssd_scan_bidir(x, Bm, Cm, dt, dt_bias, A_log, D, prefix_len: int, cfg, out=N
     return out
 
 
+def ssd_scan_bidir_noalloc(x, Bm, Cm, dt, dt_bias, A_log, D, prefix_len: int, cfg, out, stream=None):
+    """ssd_scan_bidir on the library's fixed device scratch, for callers that may not allocate device memory.
+    Nothing is allocated here either: the caller passes the output `out` [B, T*H*W, nh*P]."""
+    c = _cfg(cfg)
+    st = _lib.load().ssd_scan_bidir_noalloc(_p(x), _p(Bm), _p(Cm), _p(dt), _p(dt_bias), _p(A_log), _p(D),
+                                            int(prefix_len), _p(out), ctypes.byref(c), _s(stream))
+    _lib.check(st, "ssd_scan_bidir_noalloc")
+    return out
+
+
 def tesa_forward(qkv: torch.Tensor, shifted: bool, cfg, out: Optional[torch.Tensor] = None, stream=None):
     if out is None:
         out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.W, cfg.th * cfg.tp), dtype=qkv.dtype, device=qkv.device)

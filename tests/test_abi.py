@@ -31,7 +31,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for s in range(7):
+    for s in range(8):
         assert _lib.status_str(s)
 
 
@@ -101,3 +101,12 @@ def test_workspace_grows_linearly_with_tokens(lib):
     per = [(sizes[i + 1] - sizes[i]) for i in range(2)]
     # doubling-by-4 of T adds 4x the per-token bytes each time
     assert abs(per[1] / per[0] - 4.0) < 0.01
+
+
+def test_noalloc_scan_rejects_problems_beyond_its_scratch(lib):
+    """The fixed-scratch scan refuses, before touching the device, a problem whose scratch exceeds the buffer."""
+    cfg = mi.CONFIGS["bf16_16x32x32"]
+    c = _lib.make_config(cfg)
+    assert lib.mate_ssd_workspace_bytes(ctypes.byref(c), cfg.R) > _lib.MATE_SSD_NOALLOC_SCRATCH_BYTES
+    st = lib.ssd_scan_bidir_noalloc(16, 16, 16, 16, 16, 16, 16, cfg.R, 16, ctypes.byref(c), None)
+    assert st == _lib.MATE_ERR_TOO_LARGE, _lib.status_str(st)
