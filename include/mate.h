@@ -225,6 +225,44 @@ MATE_API mate_status mate_device_status(mate_stream_t stream, unsigned int* flag
 /* Number of kernel launches the last successful mate_forward call issued on this thread. */
 MATE_API int mate_last_launch_count(void);
 
+/*
+ * Kernel timing trace (an instrumentation aid; the pages have no counterpart).  Between
+ * mate_trace_start(capacity) and mate_trace_stop(), each kernel launch of this library (up to `capacity`
+ * launches, from any thread) records a CUDA event on its stream just before and just after the launch.
+ * mate_trace_read then waits for those events and writes, per launch in launch order, the kernel's
+ * identity and its device duration in milliseconds; it returns the number of records (-1 while a trace
+ * is on or on a CUDA error).  Starting a trace discards the previous one.  Events are created on the
+ * device current at mate_trace_start, so launches must run on that device; they are kept for reuse.
+ * The events add a few microseconds of host work per launch and nothing to the kernels themselves.
+ */
+typedef enum {
+  MATE_K_PACK_WEIGHTS = 0,     /* packing [W_in; W_qkv] and [W_out | W_o] */
+  MATE_K_REVIEW_POOL = 1,
+  MATE_K_IN_PROJ = 2,          /* fused MA in-projection + TESA qkv projection of the video rows */
+  MATE_K_IN_PROJ_REVIEW = 3,   /* MA in-projection of the review rows */
+  MATE_K_SOFTPLUS = 4,         /* delta = softplus(dt + dt_bias), standalone scan only */
+  MATE_K_SSD_GRAM = 5,
+  MATE_K_SSD_STATE = 6,
+  MATE_K_SSD_CARRY = 7,
+  MATE_K_SSD_OUTPUT = 8,
+  MATE_K_SSD_F32 = 9,
+  MATE_K_TESA = 10,
+  MATE_K_TESA_F32 = 11,
+  MATE_K_OUT_PROJ = 12,        /* fused out-projection [y | O] [W_out | W_o]^T (the branch sum) */
+  MATE_K_RMS_GATHER = 13,
+  MATE_K_PROJECT = 14          /* mate_project_bf16 */
+} mate_kernel;
+
+typedef struct {
+  int kernel;   /* a mate_kernel value */
+  float ms;     /* device time between the events around the launch */
+} mate_trace_record;
+
+MATE_API mate_status mate_trace_start(int capacity);
+MATE_API mate_status mate_trace_stop(void);
+MATE_API int mate_trace_read(mate_trace_record* out, int max_records);
+MATE_API const char* mate_kernel_name(int kernel);
+
 #ifdef __cplusplus
 }
 #endif

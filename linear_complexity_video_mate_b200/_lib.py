@@ -15,7 +15,7 @@ EXPORTS = (
     "mate_status_str", "mate_check_config", "mate_workspace_bytes", "mate_ssd_workspace_bytes", "rms_permute",
     "rms_unpermute", "review_pool", "ssd_scan_bidir", "tesa_forward", "mate_forward", "mate_forward_host",
     "mate_forward_host_workspace_bytes", "mate_device_status", "mate_last_launch_count", "mate_project_bf16",
-    "ssd_scan_bidir_noalloc",
+    "ssd_scan_bidir_noalloc", "mate_trace_start", "mate_trace_stop", "mate_trace_read", "mate_kernel_name",
 )
 
 _CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp", "wt", "wh", "ww", "st", "sh", "sw")
@@ -29,6 +29,10 @@ class CWeights(ctypes.Structure):
     _fields_ = [("W_in", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
                 ("D", ctypes.c_void_p), ("W_out", ctypes.c_void_p), ("W_qkv", ctypes.c_void_p),
                 ("W_o", ctypes.c_void_p)]
+
+
+class CTraceRecord(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int), ("ms", ctypes.c_float)]
 
 
 class MateError(RuntimeError):
@@ -60,6 +64,10 @@ def load():
         "review_pool": (ci, [vp, vp, ci, cfgp, vp]),
         "ssd_scan_bidir": (ci, [vp, vp, vp, vp, vp, vp, vp, ci, vp, cfgp, vp, sz, vp]),
         "ssd_scan_bidir_noalloc": (ci, [vp, vp, vp, vp, vp, vp, vp, ci, vp, cfgp, vp]),
+        "mate_trace_start": (ci, [ci]),
+        "mate_trace_stop": (ci, []),
+        "mate_trace_read": (ci, [ctypes.POINTER(CTraceRecord), ci]),
+        "mate_kernel_name": (ctypes.c_char_p, [ci]),
         "tesa_forward": (ci, [vp, vp, ci, cfgp, vp]),
         "mate_forward": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
         "mate_forward_host": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),

@@ -8,7 +8,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "../../include/mate.h"
 #include "common.cuh"
@@ -23,9 +25,41 @@ namespace {
 
 thread_local int t_launches = 0;
 
+// ------------------------------------------------------------------------------ kernel timing trace
+// While a trace is on, every launch records a CUDA event before and after it on its stream.
+struct Trace {
+  std::mutex mu;
+  std::atomic<bool> on{false};
+  int cap = 0, n = 0;
+  std::vector<cudaEvent_t> ev;   // 2 per record
+  std::vector<int> kid;
+};
+Trace g_trace;
+thread_local int t_trace_slot = -1;          // record opened by the last trace_begin on this thread
+thread_local cudaStream_t t_trace_stream = nullptr;
+
+void trace_begin(int kid, cudaStream_t st) {
+  t_trace_slot = -1;
+  if (!g_trace.on) return;
+  std::lock_guard<std::mutex> lock(g_trace.mu);
+  if (!g_trace.on || g_trace.n >= g_trace.cap) return;
+  const int slot = g_trace.n++;
+  g_trace.kid[slot] = kid;
+  cudaEventRecord(g_trace.ev[2 * slot], st);
+  t_trace_slot = slot;
+  t_trace_stream = st;
+}
+
+void trace_end() {
+  if (t_trace_slot < 0) return;
+  cudaEventRecord(g_trace.ev[2 * t_trace_slot + 1], t_trace_stream);
+  t_trace_slot = -1;
+}
+
 #define MATE_LAUNCH_CHECK()                         \
   do {                                              \
     ++t_launches;                                   \
+    trace_end();                                    \
     if (cudaPeekAtLastError() != cudaSuccess) {     \
       (void)cudaGetLastError();                     \
       return MATE_ERR_CUDA;                         \
@@ -137,7 +171,8 @@ struct Carver {
 
 struct SsdScratch {
   __nv_bfloat16 *Gm, *Sf, *Sb, *Hf, *Hb;
-  float *gl, *Gd;
+  float *gl, *Gd, *cs, *cdl;
+  int* crow;
 };
 
 int ceil_div(long long a, int b) { return static_cast<int>((a + b - 1) / b); }
@@ -153,6 +188,9 @@ SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh) {
   s.Hb = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
   s.gl = cv.take<float>((size_t)B * (nRc + nVc) * nh);
   s.Gd = cv.take<float>((size_t)B * nVc * kSsdQ);
+  s.cs = cv.take<float>((size_t)B * nVc * nh * kSsdQ);
+  s.cdl = cv.take<float>((size_t)B * nVc * nh * kSsdQ);
+  s.crow = cv.take<int>((size_t)B * nVc * kSsdQ);
   return s;
 }
 
@@ -201,8 +239,9 @@ size_t ssd_ws_bytes(const mate_config* c, int prefix_len, float** delta, SsdScra
 // narrower, padding-free tiles); a ragged last tile issues narrower MMAs instead of padding.
 int choose_bn(int N) { return N >= 256 ? 256 : ((N + 15) / 16) * 16; }
 
-mate_status gemm_bf16(const void* A, int lda, long long M, int K, const void* Bw, int ldb, int N, void* C, int ldc,
-                      float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias, cudaStream_t st) {
+mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const void* Bw, int ldb, int N, void* C,
+                      int ldc, float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias,
+                      cudaStream_t st) {
   if (M <= 0) return MATE_OK;
   if (K % kGemmBK) return MATE_ERR_UNSUPPORTED;
   GemmParams p;
@@ -230,15 +269,18 @@ mate_status gemm_bf16(const void* A, int lda, long long M, int K, const void* Bw
   const size_t smem = 1024 + (size_t)p.stages * psb + 256;
   if (!set_smem(gemm_bf16_pair_kernel, smem)) return MATE_ERR_CUDA;
   const int pairs = std::min(p.num_tiles, device_sms() / 2);
+  trace_begin(kid, st);
   gemm_bf16_pair_kernel<<<2 * pairs, kGemmThreads, smem, st>>>(ta, tb, p);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }
 
-mate_status gemm_f32(const float* A, int lda, long long M, int K, const float* Bw, int ldb, int N, float* C, int ldc,
-                     float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias, cudaStream_t st) {
+mate_status gemm_f32(int kid, const float* A, int lda, long long M, int K, const float* Bw, int ldb, int N, float* C,
+                     int ldc, float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias,
+                     cudaStream_t st) {
   if (M <= 0) return MATE_OK;
   dim3 grid(ceil_div(N, 64), ceil_div(M, 64));
+  trace_begin(kid, st);
   gemm_f32_kernel<<<grid, 256, 0, st>>>(A, lda, Bw, ldb, C, ldc, static_cast<int>(M), N, K, delta, ld_delta, dt_col0,
                                         dt_cols, dt_bias);
   MATE_LAUNCH_CHECK();
@@ -250,6 +292,7 @@ mate_status gather_rows(const void* src, void* dst, const mate_config* c, int or
   const int vec = static_cast<int>(c->d * elem_size(c) / 16);
   const long long rows = (long long)c->B * n;
   const int blocks = static_cast<int>(std::min<long long>((rows + 7) / 8, (long long)device_sms() * 16));
+  trace_begin(MATE_K_RMS_GATHER, st);
   rms_gather_rows_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows,
                                                  static_cast<int>(n), vec, c->T, c->H, c->W, order, inverse);
   MATE_LAUNCH_CHECK();
@@ -261,6 +304,7 @@ mate_status pool(const void* X, void* Rv, const mate_config* c, int order, cudaS
   const int per = 16 / static_cast<int>(elem_size(c));
   const int threads = std::min(256, std::max(32, ((c->d / per) + 31) / 32 * 32));
   dim3 grid(c->R, c->B);
+  trace_begin(MATE_K_REVIEW_POOL, st);
   if (c->dtype == MATE_BF16)
     review_pool_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(X),
                                                                 static_cast<__nv_bfloat16*>(Rv), c->R, c->T, c->H,
@@ -277,6 +321,7 @@ mate_status copy_block(const void* src, void* dst, int rows, int cols, int ld_ds
   const int vcols = static_cast<int>(cols * es / 16);
   const long long total = (long long)rows * vcols;
   const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4096));
+  trace_begin(MATE_K_PACK_WEIGHTS, st);
   copy_block_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows, vcols,
                                             static_cast<int>(ld_dst * es / 16), row0, static_cast<int>(col0 * es / 16));
   MATE_LAUNCH_CHECK();
@@ -289,6 +334,7 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   const long long n = (long long)c->T * c->H * c->W;
   if (c->dtype == MATE_F32) {
     const int threads = ((c->P * c->N) + 31) / 32 * 32;
+    trace_begin(MATE_K_SSD_F32, st);
     ssd_f32_kernel<<<dim3(c->nh, c->B), threads, c->P * c->N * sizeof(float), st>>>(
         rows, A_log, Dp, c->P, c->N, static_cast<float*>(y), ldy, y_bstride);
     MATE_LAUNCH_CHECK();
@@ -309,6 +355,9 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   p.Gd = sc.Gd;
   p.Hf = sc.Hf;
   p.Hb = sc.Hb;
+  p.crow = sc.crow;
+  p.cs = sc.cs;
+  p.cdl = sc.cdl;
   p.y = static_cast<__nv_bfloat16*>(y);
   p.ldy = ldy;
   p.y_bstride = y_bstride;
@@ -318,12 +367,15 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   if (!set_smem(ssd_gram_kernel, smem_gram) || !set_smem(ssd_state_kernel, smem_state) ||
       !set_smem(ssd_output_kernel, smem_out))
     return MATE_ERR_CUDA;
+  trace_begin(MATE_K_SSD_GRAM, st);
   ssd_gram_kernel<<<dim3(p.nVc, c->B, 2), 128, smem_gram, st>>>(p);
   MATE_LAUNCH_CHECK();
   int hpc = 1;
   while (hpc < 4 && c->nh % (hpc * 2) == 0) hpc *= 2;
+  trace_begin(MATE_K_SSD_STATE, st);
   ssd_state_kernel<<<dim3(p.nRc + p.nVc, c->B, c->nh / hpc), 256, smem_state, st>>>(p, hpc);
   MATE_LAUNCH_CHECK();
+  trace_begin(MATE_K_SSD_CARRY, st);
   ssd_carry_kernel<<<dim3(kSsdP * kSsdN / 8 / 128, c->nh, 2 * c->B), 128, 0, st>>>(p);
   MATE_LAUNCH_CHECK();
   SsdOutMaps mp;
@@ -332,9 +384,11 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   const long long srows = (long long)c->B * p.nVc * c->nh * kSsdN;
   if (!make_tmap(&mp.x, rows.xv, vrows, (long long)c->nh * c->P, rows.ldxv, 1) ||
       !make_tmap(&mp.c, rows.cv, vrows, c->N, rows.ldcv, 1) || !make_tmap(&mp.hf, sc.Hf, srows, kSsdP, kSsdP, 128) ||
-      !make_tmap(&mp.hb, sc.Hb, srows, kSsdP, kSsdP, 128))
+      !make_tmap(&mp.hb, sc.Hb, srows, kSsdP, kSsdP, 128) ||
+      !make_tmap(&mp.g, sc.Gm, (long long)c->B * p.nVc * kSsdQ, kSsdQ, kSsdQ, 128))
     return MATE_ERR_CUDA;
   const int out_items = c->B * p.nVc * c->nh * 2;
+  trace_begin(MATE_K_SSD_OUTPUT, st);
   ssd_output_kernel<<<std::min(out_items, device_sms()), kSsdOutThreads, smem_out, st>>>(p, mp);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
@@ -347,6 +401,7 @@ mate_status run_tesa(const mate_config* c, const void* qkv, int ldq, int qcol, i
     const long long n = (long long)c->T * c->H * c->W;
     const long long warps = n * c->th;
     dim3 grid(static_cast<unsigned>((warps + 7) / 8), c->B);
+    trace_begin(MATE_K_TESA_F32, st);
     tesa_f32_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(qkv), ldq, qcol, kcol, vcol,
                                           static_cast<float*>(O), ldo, ocol, c->T, c->H, c->W, c->th, c->tp, c->wt,
                                           c->wh, c->ww, c->st, c->sh, c->sw, sft);
@@ -377,6 +432,7 @@ mate_status run_tesa(const mate_config* c, const void* qkv, int ldq, int qcol, i
   const size_t smem = 1024 + 196608 + 2048 + 1024 + 2048 + 64;
   if (!set_smem(tesa_bf16_kernel, smem)) return MATE_ERR_CUDA;
   const int nwin = (c->T / c->wt) * (c->H / c->wh) * (c->W / c->ww);
+  trace_begin(MATE_K_TESA, st);
   tesa_bf16_kernel<<<dim3(nwin, c->B, c->th), kTesaThreads, smem, st>>>(p);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
@@ -412,12 +468,12 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   // review tokens, then the projections of the video rows (grid order) and of the review rows
   MATE_TRY(pool(X, pl.Rv, c, order, st));
   if (c->dtype == MATE_BF16) {
-    MATE_TRY(gemm_bf16(X, c->d, Mv, c->d, pl.Wi, c->d, NI, pl.Zv, NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
-    MATE_TRY(gemm_bf16(pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, X, c->d, Mv, c->d, pl.Wi, c->d, NI, pl.Zv, NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
   } else {
-    MATE_TRY(gemm_f32(static_cast<const float*>(X), c->d, Mv, c->d, static_cast<const float*>(pl.Wi), c->d, NI,
+    MATE_TRY(gemm_f32(MATE_K_IN_PROJ, static_cast<const float*>(X), c->d, Mv, c->d, static_cast<const float*>(pl.Wi), c->d, NI,
                       static_cast<float*>(pl.Zv), NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
-    MATE_TRY(gemm_f32(static_cast<const float*>(pl.Rv), c->d, Mr, c->d, static_cast<const float*>(pl.Wi), c->d, NIn,
+    MATE_TRY(gemm_f32(MATE_K_IN_PROJ_REVIEW, static_cast<const float*>(pl.Rv), c->d, Mr, c->d, static_cast<const float*>(pl.Wi), c->d, NIn,
                       static_cast<float*>(pl.Zr), NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
   }
   // MA: scan over [review rows; video rows in scan order], y written at grid-order rows of YO[:, :dI]
@@ -451,9 +507,9 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   MATE_TRY(run_tesa(c, pl.Zv, NI, qc, qc + ac, qc + 2 * ac, pl.YO, KO, dI, shifted, st));
   // Out = [y | O] [W_out | W_o]^T = MA + TE
   if (c->dtype == MATE_BF16)
-    MATE_TRY(gemm_bf16(pl.YO, KO, Mv, KO, pl.Wo, KO, c->d, Out, c->d, nullptr, 0, 0, 0, nullptr, st));
+    MATE_TRY(gemm_bf16(MATE_K_OUT_PROJ, pl.YO, KO, Mv, KO, pl.Wo, KO, c->d, Out, c->d, nullptr, 0, 0, 0, nullptr, st));
   else
-    MATE_TRY(gemm_f32(static_cast<const float*>(pl.YO), KO, Mv, KO, static_cast<const float*>(pl.Wo), KO, c->d,
+    MATE_TRY(gemm_f32(MATE_K_OUT_PROJ, static_cast<const float*>(pl.YO), KO, Mv, KO, static_cast<const float*>(pl.Wo), KO, c->d,
                       static_cast<float*>(Out), c->d, nullptr, 0, 0, 0, nullptr, st));
   return MATE_OK;
 }
@@ -533,6 +589,7 @@ mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const 
   const long long n = (long long)cfg->T * cfg->H * cfg->W;
   const long long L = n + prefix_len;
   const long long total = (long long)cfg->B * L * cfg->nh;
+  trace_begin(MATE_K_SOFTPLUS, st);
   softplus_kernel<<<static_cast<int>(std::min<long long>((total + 255) / 256, 4096)), 256, 0, st>>>(dt, dt_bias, delta,
                                                                                                    total, cfg->nh);
   MATE_LAUNCH_CHECK();
@@ -612,7 +669,7 @@ mate_status mate_project_bf16(const void* A, int lda, long long M, int K, const 
     return MATE_ERR_ARG;
   if (K % kGemmBK) return MATE_ERR_UNSUPPORTED;
   t_launches = 0;
-  return gemm_bf16(A, lda, M, K, Wt, ldw, N, C, ldc, nullptr, 0, 0, 0, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return gemm_bf16(MATE_K_PROJECT, A, lda, M, K, Wt, ldw, N, C, ldc, nullptr, 0, 0, 0, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 mate_status mate_forward(const void* X, const mate_weights* w, int layer_idx, void* Out, const mate_config* cfg,
@@ -649,5 +706,70 @@ mate_status mate_device_status(mate_stream_t stream, unsigned int* flags) {
 }
 
 int mate_last_launch_count(void) { return t_launches; }
+
+mate_status mate_trace_start(int capacity) {
+  if (capacity < 0) return MATE_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_trace.mu);
+  g_trace.on = false;
+  if (static_cast<int>(g_trace.ev.size()) < 2 * capacity) {
+    for (size_t e = g_trace.ev.size(); e < static_cast<size_t>(2 * capacity); ++e) {
+      cudaEvent_t ev;
+      if (cudaEventCreate(&ev) != cudaSuccess) {
+        cudaGetLastError();
+        return MATE_ERR_CUDA;
+      }
+      g_trace.ev.push_back(ev);
+    }
+  }
+  g_trace.kid.assign(capacity, -1);
+  g_trace.cap = capacity;
+  g_trace.n = 0;
+  g_trace.on = capacity > 0;
+  return MATE_OK;
+}
+
+mate_status mate_trace_stop(void) {
+  std::lock_guard<std::mutex> lock(g_trace.mu);
+  g_trace.on = false;
+  return MATE_OK;
+}
+
+int mate_trace_read(mate_trace_record* out, int max_records) {
+  std::lock_guard<std::mutex> lock(g_trace.mu);
+  if (g_trace.on || out == nullptr || max_records < 0) return -1;
+  const int n = std::min(g_trace.n, max_records);
+  for (int r = 0; r < n; ++r) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(g_trace.ev[2 * r + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, g_trace.ev[2 * r], g_trace.ev[2 * r + 1]) != cudaSuccess) {
+      cudaGetLastError();
+      return -1;
+    }
+    out[r].kernel = g_trace.kid[r];
+    out[r].ms = ms;
+  }
+  return n;
+}
+
+const char* mate_kernel_name(int kernel) {
+  switch (kernel) {
+    case MATE_K_PACK_WEIGHTS: return "pack_weights";
+    case MATE_K_REVIEW_POOL: return "review_pool";
+    case MATE_K_IN_PROJ: return "in_projection";
+    case MATE_K_IN_PROJ_REVIEW: return "in_projection_review";
+    case MATE_K_SOFTPLUS: return "softplus";
+    case MATE_K_SSD_GRAM: return "ssd_gram";
+    case MATE_K_SSD_STATE: return "ssd_state";
+    case MATE_K_SSD_CARRY: return "ssd_carry";
+    case MATE_K_SSD_OUTPUT: return "ssd_output";
+    case MATE_K_SSD_F32: return "ssd_f32";
+    case MATE_K_TESA: return "tesa";
+    case MATE_K_TESA_F32: return "tesa_f32";
+    case MATE_K_OUT_PROJ: return "out_projection";
+    case MATE_K_RMS_GATHER: return "rms_gather";
+    case MATE_K_PROJECT: return "project";
+  }
+  return "unknown";
+}
 
 }  // extern "C"

@@ -49,6 +49,9 @@ struct SsdBf16Params {
   float* gl;          // [B][nRc + nVc][nh]  s_last of each chunk
   __nv_bfloat16* Hf;  // [B][nVc][nh][N][P]  state entering video chunk v, forward traversal
   __nv_bfloat16* Hb;  // [B][nVc][nh][N][P]  state entering video chunk v, backward traversal
+  int* crow;          // [B][nVc][Q]     source row of each video-chunk row (-1 past the end)
+  float* cs;          // [B][nVc][nh][Q] inclusive cumulative sum of delta * A over the chunk
+  float* cdl;         // [B][nVc][nh][Q] delta of each chunk row (0 past the end)
   __nv_bfloat16* y;   // row b*y_bstride + map(q), column h*P
   int ldy;
   long long y_bstride;
@@ -296,6 +299,12 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
     const float dl = dl_next;
     const float a = dl * A;
     const float s = block_scan_256(a, wtot);
+    if (video) {   // per-row tables of the output kernel
+      const long long cv = static_cast<long long>(b) * p.nVc + (c - p.nRc);
+      p.cs[(cv * p.nh + h) * kSsdQ + j] = s;
+      p.cdl[(cv * p.nh + h) * kSsdQ + j] = dl;
+      if (hh == 0 && blockIdx.z == 0) p.crow[cv * kSsdQ + j] = myrw >= 0 ? static_cast<int>(myrw) : -1;
+    }
     if (j == 255) wtot[8 - 1] = s;  // reuse slot 7 for s_last after the scan finished with wtot
     __syncthreads();
     const float s_last = wtot[7];
@@ -445,17 +454,20 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 // Outputs of the video chunks: persistent, warp-specialised.  One work item = (sample, video chunk, head,
 // 128-row tile t of the chunk); a CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ...
 //
-//   warps 0..3   loaders: gather the item's x rows (all 256, MN-major) and the C rows of the tile
-//                (K-major) with TMA four-row gathers (tile::gather4), load the incoming states Hf / Hb
-//                (MN-major) with 2D TMA, into one of two shared-memory buffers; compute the cumulative
-//                sums and the decay factor tables of the item.
-//   warps 4..11  transform (two warps per TMEM lane quadrant, alternating 8-column chunks): read the
-//                tile's 128 rows of G = C B^T (bf16, global/L2), form
-//                M_ij = G_ij delta_j dec(i, j) (diagonal excluded) and store M straight into TMEM as
-//                the A operand of the next MMA (two bf16 per 32-bit column).
-//   MMA issue    lane 0 of warp 4, once all transform warps stored M: Yd = M x (A from TMEM),
-//                Yf = C Hf^T, Yb = C Hb^T into one of two TMEM accumulator sets.  (16 warps in total: a
-//                17th warp would put 5 warps on one SM sub-partition, beyond its register file.)
+//   warps 0..2   loaders.  Per item: the chunk's row table and the head's cumulative sums and step sizes
+//                (written by the state kernel, fetched one item ahead) -> decay-factor tables; the item's
+//                x rows (all 256, MN-major) by TMA four-row gathers into one of two x buffers; the tile's
+//                C rows (K-major, four-row gathers) and the incoming states Hf / Hb (MN-major, 2D TMA)
+//                into the single C/H buffer once the previous item's C H^T products are done; the
+//                tile's rows of G = C B^T (2D TMA) into four 64-column slots, each refilled as soon as the
+//                transform has read it.
+//   warp 3       MMA issue (lane 0 only; an issuing thread stalls while the tensor pipe is busy, so it has
+//                no other work): Yd = M x per K half of M (A from TMEM) and, after the first half,
+//                [Yf | Yb] = C [Hf | Hb]^T as one N = 128 product (which frees the C/H buffer for the next
+//                item), into one of two TMEM accumulator sets.
+//   warps 4..11  transform (two warps per TMEM lane quadrant, alternating 8-column chunks): form
+//                M_ij = G_ij delta_j dec(i, j) (diagonal excluded) from the G slots and store M straight
+//                into TMEM as the A operand of the MMA (two bf16 per 32-bit column), in two K halves.
 //   warps 12..15 epilogue: y_i = Yd + exp(s_i) Yf + exp(s_last - s'_i) Yb + 2 (D + G_ii delta_i) x_i,
 //                stored at the grid-order row of the token.
 //
@@ -466,54 +478,77 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 // element.
 // TMEM columns: [0, 128) M; accumulator set a at 128 + 192 a: Yd [+0, +64), Yf [+64, +128), Yb [+128, +192).
 // ---------------------------------------------------------------------------------------------------
-constexpr int kOutLoadWarps = 4, kOutXformWarps = 8, kOutEpiWarps = 4;
+constexpr int kOutLoadWarps = 3, kOutXformWarps = 8, kOutEpiWarps = 4;
+constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kOutMmaWarp = kOutLoadWarps;                                    // issues from its lane 0
-constexpr int kSsdOutThreads = (kOutLoadWarps + kOutXformWarps + kOutEpiWarps) * 32;   // 512
-constexpr uint32_t kOutBuf = 108544;                                         // bytes per operand buffer
-constexpr uint32_t kOutOffC = 32768, kOutOffHf = 65536, kOutOffHb = 81920, kOutOffTbl = 98304;
-constexpr uint32_t kOutSmem = 2 * kOutBuf + 256;
+constexpr int kOutFirstXformWarp = kOutMmaWarp + 1, kOutFirstEpiWarp = kOutFirstXformWarp + kOutXformWarps;
+constexpr int kSsdOutThreads = (kOutFirstEpiWarp + kOutEpiWarps) * 32;        // 512
+static_assert(kOutFirstXformWarp % 4 == 0 && kOutFirstEpiWarp % 4 == 0, "TMEM lane quadrants follow warp % 4");
 
-// Tensor maps of the output kernel: x and C rows of the video arrays (one-row boxes of 64 columns, for
-// four-row gathers) and the carried states ([N rows][P] per chunk and head, 64 x 128 boxes).
-struct SsdOutMaps {
-  CUtensorMap x, c, hf, hb;
-  int rows;   // row extent of the x / C maps; gathers of invalid rows use this (out of range -> zeros)
-};
-
-struct OutTables {   // per buffer, at kOutOffTbl
+struct OutTables {   // per x buffer, after the x tile
   float sdl[256], ss[256], ssx[256];
+  float lf[256], lb[256];       // diagonal blocks: log2(delta_j) - s_j log2(e), log2(delta_j) + s'_j log2(e)
   float uf[128], ub[128];       // per tile row
+  float gd[128];                // G_ii of the tile rows (fp32)
   float wf[2][256], wb[2][256]; // per 64-row block of the tile (ib = 2t + q)
   int srow[256];                // source row of each chunk row (-1 past the end of a partial chunk)
-  float wtot[4];
+  float D;
+};
+
+// shared memory map (offsets from the 1024-aligned base)
+constexpr uint32_t kOutXBuf = 45056;                    // x tile (32 KB) + tables, two of them
+constexpr uint32_t kOutOffTbl = 32768;
+constexpr uint32_t kOutOffC = 2 * kOutXBuf;             // C rows of the tile: 2 K blocks of 16 KB
+constexpr uint32_t kOutOffHf = kOutOffC + 32768;        // [N = 128][P = 64] MN-major
+constexpr uint32_t kOutOffHb = kOutOffHf + 16384;
+constexpr uint32_t kOutOffG = kOutOffHb + 16384;        // 4 slots of [128 rows][64 cols] K-major
+constexpr uint32_t kOutOffBar = kOutOffG + 4 * 16384;
+constexpr uint32_t kOutSmem = kOutOffBar + 256;
+static_assert(sizeof(OutTables) <= kOutXBuf - kOutOffTbl, "tables overflow the x buffer");
+static_assert(kOutOffC % 1024 == 0 && kOutOffG % 1024 == 0, "operand tiles must be 1024-byte aligned");
+
+// Tensor maps of the output kernel: x and C rows of the video arrays (one-row boxes of 64 columns, for
+// four-row gathers), the carried states ([N rows][P] per chunk and head, 64 x 128 boxes) and G
+// ([chunk rows][Q] bf16, 64 x 128 boxes).
+struct SsdOutMaps {
+  CUtensorMap x, c, hf, hb, g;
+  int rows;   // row extent of the x / C maps; gathers of invalid rows use this (out of range -> zeros)
 };
 
 __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const SsdBf16Params p,
                                                                         const __grid_constant__ SsdOutMaps mp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kOutBuf);
-  uint64_t* ld_full = bars;        // [2] loaders -> consumers (count 128)
-  uint64_t* ld_empty = bars + 2;   // [2] MMA commit + epilogue warps -> loaders (count 5)
-  uint64_t* m_full = bars + 4;     // [2] per K half of M: transform -> MMA (count 256)
-  uint64_t* m_empty = bars + 6;    // [2] per K half of M: MMA commit -> transform (count 1)
-  uint64_t* y_full = bars + 8;     // [2] MMA commit -> epilogue (count 1)
-  uint64_t* y_empty = bars + 10;   // [2] epilogue warps -> MMA (count 4)
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOutOffBar);
+  uint64_t* x_full = bars;         // [2] x bytes + the loader threads (tables written)
+  uint64_t* x_empty = bars + 2;    // [2] last Yd MMA commit + 4 epilogue warps
+  uint64_t* ch_full = bars + 4;    // C + Hf + Hb bytes
+  uint64_t* ch_empty = bars + 5;   // Yf / Yb MMA commit
+  uint64_t* g_full = bars + 6;     // [4] one G slot's bytes
+  uint64_t* g_empty = bars + 10;   // [4] the 8 transform warps have read the slot
+  uint64_t* m_full = bars + 14;    // [2] per K half of M: transform -> MMA (count 256)
+  uint64_t* m_empty = bars + 16;   // [2] per K half of M: MMA commit -> transform
+  uint64_t* y_full = bars + 18;    // [2] MMA commit -> epilogue
+  uint64_t* y_empty = bars + 20;   // [2] epilogue warps -> MMA (count 4)
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bars + 22);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nitems = p.B * p.nVc * p.nh * 2;
 
   if (threadIdx.x == 0) {
     for (int q = 0; q < 2; ++q) {
-      mbar_init(&ld_full[q], 129);   // 128 loader threads + the byte-count arrival
-      mbar_init(&ld_empty[q], 5);
+      mbar_init(&x_full[q], kOutLoadWarps * 32 + 1);
+      mbar_init(&x_empty[q], 5);
+      mbar_init(&m_full[q], 256);
+      mbar_init(&m_empty[q], 1);
       mbar_init(&y_full[q], 1);
       mbar_init(&y_empty[q], 4);
     }
-    for (int q = 0; q < 2; ++q) {
-      mbar_init(&m_full[q], 256);
-      mbar_init(&m_empty[q], 1);
+    mbar_init(ch_full, 1);
+    mbar_init(ch_empty, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&g_full[q], 1);
+      mbar_init(&g_empty[q], kOutXformWarps);
     }
     mbar_fence_init();
   }
@@ -536,73 +571,88 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
 
   if (warp < kOutLoadWarps) {
     // ------------------------------------------------------------------------------ loaders
-    const int lt = threadIdx.x;  // 0..127
+    constexpr int NL = kOutLoadWarps * 32;   // 96 loader threads
+    const int lt = threadIdx.x;
+    // A wait that ran out is carried to the next item's first barrier, where all loader threads leave
+    // the loop together (a thread leaving alone would strand the others at a named barrier).
+    bool failed = false;
+    // per-row inputs of an item (chunk row table, cumulative sums, step sizes, G diagonal), fetched one
+    // item ahead so that their latency overlaps the previous item
+    struct RowIn {
+      int rw[3];
+      float s[3], d[3], gd[2], A, D;
+    };
+    auto fetch = [&](int it, RowIn& in) {
+      if (it >= nitems) return;
+      int b, v, h, t;
+      decode(it, b, v, h, t);
+      const long long cidx = static_cast<long long>(b) * p.nVc + v;
+      const long long hidx = (cidx * p.nh + h) * kSsdQ;
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const int j = lt + u * NL;
+        if (j < kSsdQ) {
+          in.rw[u] = p.crow[cidx * kSsdQ + j];
+          in.s[u] = p.cs[hidx + j];
+          in.d[u] = p.cdl[hidx + j];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (lt + u * NL < 128) in.gd[u] = p.Gd[cidx * kSsdQ + t * 128 + lt + u * NL];
+      in.A = -__expf(p.A_log[h]);
+      in.D = p.Dp[h];
+    };
+    RowIn cur, nxt;
+    fetch(blockIdx.x, cur);
     int k = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
       const int buf = k & 1, use = k >> 1;
-      if (!mbar_wait(&ld_empty[buf], (use & 1) ^ 1)) break;
       int b, v, h, t;
       decode(it, b, v, h, t);
-      const int c = p.nRc + v;
-      const ChunkBase cb = chunk_base(p.s, c, p.nRc);
-      uint8_t* B0 = smem + buf * kOutBuf;
-      OutTables& tb = *reinterpret_cast<OutTables*>(B0 + kOutOffTbl);
-      for (int j = lt; j < 256; j += 128) {
-        const RowRef rr = chunk_row(p.s, b, c, p.nRc, j);
-        tb.srow[j] = rr.valid ? static_cast<int>(rr.r) : -1;
+      const long long cidx = static_cast<long long>(b) * p.nVc + v;
+      fetch(it + gridDim.x, nxt);
+      const bool okx = mbar_wait(&x_empty[buf], (use & 1) ^ 1);
+      if (named_bar_any(1, NL, failed || !okx)) break;
+      uint8_t* XB = smem + buf * kOutXBuf;
+      OutTables& tb = *reinterpret_cast<OutTables*>(XB + kOutOffTbl);
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const int j = lt + u * NL;
+        if (j < kSsdQ) {
+          tb.srow[j] = cur.rw[u];
+          tb.sdl[j] = cur.d[u];
+          tb.ss[j] = cur.s[u];
+          tb.ssx[j] = cur.s[u] - cur.d[u] * cur.A;
+        }
       }
-      if (lt == 0) mbar_arrive_expect_tx(&ld_full[buf], 3 * 32768);   // x (32 KB), C (32 KB), Hf + Hb (32 KB)
-      named_bar_sync(1, 128);
-      // TMA: x rows (all 256, 4 per gather), C rows of the tile (2 column blocks), the two states
-      auto rowid = [&](int j) { const int rw = tb.srow[j]; return rw < 0 ? mp.rows : rw; };
-      if (lt < 64) {
-        const int g = lt;
-        tma_gather4(&mp.x, &ld_full[buf], B0 + g * 512, h * kSsdP, rowid(4 * g), rowid(4 * g + 1), rowid(4 * g + 2),
-                    rowid(4 * g + 3));
-      } else {
-        const int g = (lt - 64) & 31, kb = (lt - 64) >> 5;
-        const int j = t * 128 + 4 * g;
-        tma_gather4(&mp.c, &ld_full[buf], B0 + kOutOffC + kb * 16384 + g * 512, kb * 64, rowid(j), rowid(j + 1),
-                    rowid(j + 2), rowid(j + 3));
-      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (lt + u * NL < 128) tb.gd[lt + u * NL] = cur.gd[u];
       if (lt == 0) {
-        const int hrow = static_cast<int>(((static_cast<long long>(b) * p.nVc + v) * p.nh + h) * kSsdN);
-        tma_load_2d(&mp.hf, &ld_full[buf], B0 + kOutOffHf, 0, hrow);
-        tma_load_2d(&mp.hb, &ld_full[buf], B0 + kOutOffHb, 0, hrow);
+        tb.D = cur.D;
+        mbar_arrive_expect_tx(&x_full[buf], 32768);
       }
-      // cumulative sums: thread lt owns rows 2 lt and 2 lt + 1
-      const float A = -__expf(p.A_log[h]);
-      float dl[2], a[2];
+      named_bar_sync(1, NL);
+      auto rowid = [&](int j) { const int rw = tb.srow[j]; return rw < 0 ? mp.rows : rw; };
+      if (lt < 64) {   // x rows: all 256 of the chunk, 4 per gather
+        tma_gather4(&mp.x, &x_full[buf], XB + lt * 512, h * kSsdP, rowid(4 * lt), rowid(4 * lt + 1),
+                    rowid(4 * lt + 2), rowid(4 * lt + 3));
+      }
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int rw = tb.srow[2 * lt + e];
-        dl[e] = rw >= 0 ? cb.d[static_cast<long long>(rw) * cb.ldd + h] : 0.f;
-        a[e] = dl[e] * A;
+      for (int u = 0; u < 2; ++u) {
+        const int rr = lt + u * NL;
+        if (rr < 128) {
+          const int i = t * 128 + rr, ib = i >> 6;
+          tb.uf[rr] = ib > 0 ? __expf(tb.ss[i] - tb.ss[64 * ib - 1]) : 0.f;
+          tb.ub[rr] = ib < 3 ? __expf(tb.ssx[64 * ib + 64] - tb.ssx[i]) : 0.f;
+        }
       }
-      float incl = a[0] + a[1];
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float u2 = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += u2;
-      }
-      if (lane == 31) tb.wtot[warp] = incl;
-      named_bar_sync(1, 128);
-      for (int w = 0; w < warp; ++w) incl += tb.wtot[w];
-      const float s1 = incl, s0 = incl - a[1];
-      tb.sdl[2 * lt] = dl[0];
-      tb.sdl[2 * lt + 1] = dl[1];
-      tb.ss[2 * lt] = s0;
-      tb.ss[2 * lt + 1] = s1;
-      tb.ssx[2 * lt] = s0 - a[0];
-      tb.ssx[2 * lt + 1] = s1 - a[1];
-      named_bar_sync(1, 128);
-      {
-        const int i = t * 128 + lt, ib = i >> 6;
-        tb.uf[lt] = ib > 0 ? __expf(tb.ss[i] - tb.ss[64 * ib - 1]) : 0.f;
-        tb.ub[lt] = ib < 3 ? __expf(tb.ssx[64 * ib + 64] - tb.ssx[i]) : 0.f;
-      }
-      for (int j = lt; j < 256; j += 128) {
+      for (int j = lt; j < kSsdQ; j += NL) {
         const float dj = tb.sdl[j], sj = tb.ss[j], sxj = tb.ssx[j];
+        const float l2d = dj > 0.f ? __log2f(dj) : -INFINITY;
+        tb.lf[j] = l2d - sj * kLog2e;
+        tb.lb[j] = l2d + sxj * kLog2e;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int ib = 2 * t + q;
@@ -610,11 +660,75 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           tb.wb[q][j] = (ib < 3 && j >= 64 * ib + 64) ? dj * __expf(sxj - tb.ssx[64 * ib + 64]) : 0.f;
         }
       }
-      mbar_arrive(&ld_full[buf]);
+      mbar_arrive(&x_full[buf]);
+      if (lt >= NL - 64) {
+        // C rows of the tile and the two states, into the single C/H buffer
+        const int lc = lt - (NL - 64);   // 0..63
+        const bool okc = mbar_wait(ch_empty, (k & 1) ^ 1);
+        failed = !okc;
+        if (okc && lc == 0) {
+          mbar_arrive_expect_tx(ch_full, 65536);
+          const int hrow = static_cast<int>((cidx * p.nh + h) * kSsdN);
+          tma_load_2d(&mp.hf, ch_full, smem + kOutOffHf, 0, hrow);
+          tma_load_2d(&mp.hb, ch_full, smem + kOutOffHb, 0, hrow);
+        }
+        named_bar_sync(2, 64);
+        const int g = lc & 31, kb = lc >> 5;
+        const int j = t * 128 + 4 * g;
+        if (okc)
+          tma_gather4(&mp.c, ch_full, smem + kOutOffC + kb * 16384 + g * 512, kb * 64, rowid(j), rowid(j + 1),
+                      rowid(j + 2), rowid(j + 3));
+      } else if (lt == 0) {
+        // G rows of the tile, one 64-column slot at a time as the transform releases them
+        const int grow = static_cast<int>(cidx * kSsdQ + t * 128);
+        for (int cb = 0; cb < 4 && !failed; ++cb) {
+          failed = !mbar_wait(&g_empty[cb], (k & 1) ^ 1);
+          if (!failed) {
+            mbar_arrive_expect_tx(&g_full[cb], 16384);
+            tma_load_2d(&mp.g, &g_full[cb], smem + kOutOffG + cb * 16384, cb * 64, grow);
+          }
+        }
+      }
+      cur = nxt;
     }
-  } else if (warp < kOutLoadWarps + kOutXformWarps) {
+  } else if (warp == kOutMmaWarp) {
+    // ------------------------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc_d = idesc_bf16_f32(128, 64, 0, 1);    // Yd: N = P
+      const uint32_t idesc_h = idesc_bf16_f32(128, 128, 0, 1);   // [Yf | Yb]: N = 2 P, B = [Hf | Hb]
+      const uint32_t cbase = smem_u32(smem + kOutOffC), hbase = smem_u32(smem + kOutOffHf);
+      int k = 0;
+      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
+        const int buf = k & 1, use = k >> 1, acc = k & 1;
+        const uint32_t xb = smem_u32(smem + buf * kOutXBuf);
+        const uint32_t ybase = tmem + 128 + acc * 192;
+        if (!mbar_wait(&y_empty[acc], (use & 1) ^ 1) || !mbar_wait(&m_full[0], k & 1)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)   // Yd = M x, first K half (M in TMEM, 8 columns per 16 elements)
+          mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, q > 0);
+        mma_commit(&m_empty[0]);
+        if (!mbar_wait(ch_full, k & 1)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)   // [Yf | Yb] = C [Hf | Hb]^T, K = N_state = 128
+          mma_bf16_ss(ybase + 64, desc_sw128(cbase + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
+                      desc_sw128(hbase + q * 2048, 16384, 1024), idesc_h, q > 0);
+        mma_commit(ch_empty);
+        if (!mbar_wait(&m_full[1], k & 1)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int q = 8; q < 16; ++q)   // Yd, second K half
+          mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, true);
+        mma_commit(&m_empty[1]);
+        mma_commit(&y_full[acc]);
+        mma_commit(&x_empty[buf]);
+      }
+    }
+    __syncwarp();
+  } else if (warp < kOutFirstEpiWarp) {
     // ------------------------------------------------------------------------------ transform
-    const int xw = warp - kOutLoadWarps;
+    const int xw = warp - kOutFirstXformWarp;
     const int quad = warp & 3, half = xw >> 2;
     const int r = quad * 32 + lane;
     int k = 0;
@@ -623,95 +737,80 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
       int b, v, h, t;
       decode(it, b, v, h, t);
       const int i = t * 128 + r, ib = i >> 6;
-      // the two warps of a lane quadrant take alternating 8-column chunks of the row, so both get half of
-      // the diagonal block's exponentials
-      const __nv_bfloat16* grow = p.Gm + ((static_cast<long long>(b) * p.nVc + v) * kSsdQ + i) * kSsdQ + half * 8;
-      // the row's 16 chunks of G (8 bf16 each, 256 bytes) are all in flight before the waits and are
-      // consumed in order through a shifting register window (keeps the chunk loop rolled: the four roles'
-      // code must share the instruction cache)
-      const uint4* gsrc = reinterpret_cast<const uint4*>(grow);
-      uint4 gw[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) gw[q] = __ldg(gsrc + 2 * q);
-      if (!mbar_wait(&ld_full[buf], use & 1)) break;
-      const OutTables& tb = *reinterpret_cast<const OutTables*>(smem + buf * kOutBuf + kOutOffTbl);
-      const float ufi = tb.uf[r], ubi = tb.ub[r], si = tb.ss[i], sxi = tb.ssx[i];
+      bool ok = true;
+      // every exit decision below is warp-uniform (a lane leaving alone would strand __syncwarp)
+      if (__any_sync(0xffffffffu, !mbar_wait(&x_full[buf], use & 1))) break;
+      const OutTables& tb = *reinterpret_cast<const OutTables*>(smem + buf * kOutXBuf + kOutOffTbl);
+      const float ufi = tb.uf[r], ubi = tb.ub[r];
+      const float si2 = tb.ss[i] * kLog2e, sxi2 = tb.ssx[i] * kLog2e;
       const float* wfr = tb.wf[ib - 2 * t];
       const float* wbr = tb.wb[ib - 2 * t];
       const uint32_t tm_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 4;
-      const int acc = k & 1;
-      bool ok = true, mma_ok = true;
-      // M is produced and consumed in two K halves (TMEM columns [0, 64) and [64, 128)): the MMAs of the
-      // first half run while the second half is being formed
 #pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        if (!mbar_wait(&m_empty[hh], (k & 1) ^ 1)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int q = 8 * hh; q < 8 * hh + 8; ++q) {
-          const uint4 gc = gw[0];
-#pragma unroll
-          for (int z = 0; z < 15; ++z) gw[z] = gw[z + 1];
-          const int j0 = (2 * q + half) * 8;
-          const int jb = j0 >> 6;   // same for the whole warp (all lanes are rows of one 64-block)
-          const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gc);
-          uint32_t pk[4];
-          if (jb != ib) {
-            const float u = jb < ib ? ufi : ubi;
-            const float* w = (jb < ib ? wfr : wbr) + j0;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 gf = unpack_bf16x2(gu[e]);
-              const float2 w2 = *reinterpret_cast<const float2*>(w + 2 * e);
-              pk[e] = pack_bf16x2(gf.x * (u * w2.x), gf.y * (u * w2.y));
-            }
-          } else {
-            // one exponential per element: forward weight below the diagonal, backward above; the
-            // diagonal itself is added in fp32 in the epilogue
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int jj = j0 + 2 * e;
-              const float2 gf = unpack_bf16x2(gu[e]);
-              const float2 sj = *reinterpret_cast<const float2*>(tb.ss + jj);
-              const float2 xj = *reinterpret_cast<const float2*>(tb.ssx + jj);
-              const float2 dj = *reinterpret_cast<const float2*>(tb.sdl + jj);
-              const float f0 = jj == i ? 0.f : dj.x * __expf(jj < i ? si - sj.x : xj.x - sxi);
-              const float f1 = jj + 1 == i ? 0.f : dj.y * __expf(jj + 1 < i ? si - sj.y : xj.y - sxi);
-              pk[e] = pack_bf16x2(gf.x * f0, gf.y * f1);
-            }
-          }
-          tmem_st4(tm_row + q * 8, pk[0], pk[1], pk[2], pk[3]);   // columns of chunk 2q + half
+      for (int cb = 0; cb < 4; ++cb) {
+        const int hh = cb >> 1;
+        if ((cb & 1) == 0) {
+          if (__any_sync(0xffffffffu, !mbar_wait(&m_empty[hh], (k & 1) ^ 1))) { ok = false; break; }
+          tc_fence_after();
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&m_full[hh]);
-        if (warp == kOutMmaWarp) {
-          if (lane == 0) {
-            // -------------------------------------------------------------------- MMA issue
-            const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 1);
-            if (hh == 0) mma_ok = mbar_wait(&y_empty[acc], (use & 1) ^ 1);
-            mma_ok = mma_ok && mbar_wait(&m_full[hh], k & 1);
-            if (mma_ok) {
-              tc_fence_after();
-              const uint32_t b0 = smem_u32(smem + buf * kOutBuf);
-              const uint32_t ybase = tmem + 128 + acc * 192;
+        if (__any_sync(0xffffffffu, !mbar_wait(&g_full[cb], k & 1))) { ok = false; break; }
+        const uint8_t* grow = smem + kOutOffG + cb * 16384 + r * 128;
+        const uint32_t tcol = tm_row + cb * 32;
+        if (cb != ib) {
+          const float u = cb < ib ? ufi : ubi;
+          const float* w = (cb < ib ? wfr : wbr) + cb * 64 + half * 8;
 #pragma unroll
-              for (int q = 8 * hh; q < 8 * hh + 8; ++q)   // Yd = M x (M in TMEM, 8 columns per 16 elements)
-                mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(b0 + q * 2048, 32768, 1024), idesc, q > 0);
-              mma_commit(&m_empty[hh]);
-              if (hh == 1) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {  // Yf = C Hf^T, Yb = C Hb^T, K = N = 128
-                  const uint64_t ad = desc_sw128(b0 + kOutOffC + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024);
-                  mma_bf16_ss(ybase + 64, ad, desc_sw128(b0 + kOutOffHf + q * 2048, 16384, 1024), idesc, q > 0);
-                  mma_bf16_ss(ybase + 128, ad, desc_sw128(b0 + kOutOffHb + q * 2048, 16384, 1024), idesc, q > 0);
-                }
-                mma_commit(&y_full[acc]);
-                mma_commit(&ld_empty[buf]);
-              }
-            }
+          for (int qq = 0; qq < 4; ++qq) {
+            const int ch = 2 * qq + half;
+            const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
+            const float4 wa = *reinterpret_cast<const float4*>(w + qq * 16);
+            const float4 wc = *reinterpret_cast<const float4*>(w + qq * 16 + 4);
+            const float2 g0 = unpack_bf16x2(gc.x), g1 = unpack_bf16x2(gc.y);
+            const float2 g2 = unpack_bf16x2(gc.z), g3 = unpack_bf16x2(gc.w);
+            tmem_st4(tcol + qq * 8, pack_bf16x2(g0.x * (u * wa.x), g0.y * (u * wa.y)),
+                     pack_bf16x2(g1.x * (u * wa.z), g1.y * (u * wa.w)),
+                     pack_bf16x2(g2.x * (u * wc.x), g2.y * (u * wc.y)),
+                     pack_bf16x2(g3.x * (u * wc.z), g3.y * (u * wc.w)));
           }
-          __syncwarp();
+        } else {
+          // one exponential per element, in the log2 domain with delta_j folded into the column
+          // tables: delta_j exp(s_i - s_j) = 2^(s_i log2e + lf_j) below the diagonal,
+          // delta_j exp(s'_j - s'_i) = 2^(lb_j - s'_i log2e) above it; the diagonal itself is added in
+          // fp32 in the epilogue
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int ch = 2 * qq + half;
+            const int j0 = cb * 64 + ch * 8;
+            const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
+            const float4 f0 = *reinterpret_cast<const float4*>(tb.lf + j0);
+            const float4 f1 = *reinterpret_cast<const float4*>(tb.lf + j0 + 4);
+            const float4 b0 = *reinterpret_cast<const float4*>(tb.lb + j0);
+            const float4 b1 = *reinterpret_cast<const float4*>(tb.lb + j0 + 4);
+            const float lf8[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+            const float lb8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gc);
+            float m[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int jj = j0 + e;
+              const float w = ex2_approx(jj < i ? si2 + lf8[e] : lb8[e] - sxi2);
+              m[e] = jj == i ? 0.f : w;
+            }
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 gf = unpack_bf16x2(gu[e]);
+              pk[e] = pack_bf16x2(gf.x * m[2 * e], gf.y * m[2 * e + 1]);
+            }
+            tmem_st4(tcol + qq * 8, pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&g_empty[cb]);
+        if (cb & 1) {
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&m_full[hh]);
         }
       }
       if (!ok) break;
@@ -725,27 +824,27 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
       const int buf = k & 1, acc = k & 1, use = k >> 1;
       int b, v, h, t;
       decode(it, b, v, h, t);
-      if (!mbar_wait(&y_full[acc], use & 1)) break;
-      tc_fence_after();
-      const uint8_t* B0 = smem + buf * kOutBuf;
-      const OutTables& tb = *reinterpret_cast<const OutTables*>(B0 + kOutOffTbl);
       const int i = t * 128 + r;
       const int len = min(kSsdQ, p.s.n - v * kSsdQ);
       const bool ok = i < len;
+      __nv_bfloat16* yrow = p.y + (b * p.y_bstride + p.s.map(v * kSsdQ + (ok ? i : 0))) * p.ldy + h * kSsdP;
+      if (__any_sync(0xffffffffu, !mbar_wait(&y_full[acc], use & 1))) break;
+      tc_fence_after();
+      const uint8_t* XB = smem + buf * kOutXBuf;
+      const OutTables& tb = *reinterpret_cast<const OutTables*>(XB + kOutOffTbl);
       const float si = tb.ss[i], sxi = tb.ssx[i], slast = tb.ss[255], dli = tb.sdl[i];
+      const float D2 = 2.f * (tb.D + (ok ? tb.gd[r] * dli : 0.f));
       // x row of this token (packed bf16 pairs) for the skip and diagonal terms
       uint32_t xw[32];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(B0 + sw128_mnmajor_offset(i, q * 8, 32768));
+        const uint4 xv = *reinterpret_cast<const uint4*>(XB + sw128_mnmajor_offset(i, q * 8, 32768));
         xw[q * 4 + 0] = xv.x; xw[q * 4 + 1] = xv.y; xw[q * 4 + 2] = xv.z; xw[q * 4 + 3] = xv.w;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ld_empty[buf]);
+      if (lane == 0) mbar_arrive(&x_empty[buf]);
       const float ef = __expf(si);
       const float eb = __expf(slast - sxi);
-      const float D2 = 2.f * (p.Dp[h] + (ok ? p.Gd[(static_cast<long long>(b) * p.nVc + v) * kSsdQ + i] * dli : 0.f));
-      __nv_bfloat16* yrow = p.y + (b * p.y_bstride + p.s.map(v * kSsdQ + (ok ? i : 0))) * p.ldy + h * kSsdP;
       const uint32_t ybase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128 + acc * 192;
 #pragma unroll
       for (int pc = 0; pc < 4; ++pc) {   // 16 columns at a time

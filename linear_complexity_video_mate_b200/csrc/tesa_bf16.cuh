@@ -30,12 +30,6 @@ struct TesaBf16Params {
 
 __device__ __forceinline__ int tesa_region(int p, int D, int w, int s) { return p < D - w ? 0 : (p < D - s ? 1 : 2); }
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 constexpr int kTesaThreads = 512;
 
 // 16 warps: warp w reads TMEM lane quadrant w%4 of query tile t = (w/4)%2 and key half w/8 (softmax),

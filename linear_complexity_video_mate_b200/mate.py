@@ -187,3 +187,26 @@ def device_status(stream=None) -> int:
     flags = ctypes.c_uint(0)
     _lib.load().mate_device_status(_s(stream), ctypes.byref(flags))
     return int(flags.value)
+
+
+class KernelTrace:
+    """Per-launch device times of this library's kernels between start() and stop() (CUDA events around
+    each launch, recorded by the library).  read() -> list of (kernel name, ms) in launch order."""
+
+    def __init__(self, capacity: int):
+        self.capacity = int(capacity)
+
+    def start(self):
+        _lib.check(_lib.load().mate_trace_start(self.capacity), "mate_trace_start")
+        return self
+
+    def stop(self):
+        _lib.check(_lib.load().mate_trace_stop(), "mate_trace_stop")
+
+    def read(self):
+        lib = _lib.load()
+        recs = (_lib.CTraceRecord * max(self.capacity, 1))()
+        n = lib.mate_trace_read(recs, self.capacity)
+        if n < 0:
+            raise _lib.MateError(_lib.MATE_ERR_CUDA, "mate_trace_read")
+        return [(lib.mate_kernel_name(recs[r].kernel).decode(), float(recs[r].ms)) for r in range(n)]

@@ -110,3 +110,10 @@ def test_noalloc_scan_rejects_problems_beyond_its_scratch(lib):
     assert lib.mate_ssd_workspace_bytes(ctypes.byref(c), cfg.R) > _lib.MATE_SSD_NOALLOC_SCRATCH_BYTES
     st = lib.ssd_scan_bidir_noalloc(16, 16, 16, 16, 16, 16, 16, cfg.R, 16, ctypes.byref(c), None)
     assert st == _lib.MATE_ERR_TOO_LARGE, _lib.status_str(st)
+
+
+def test_kernel_names_are_distinct(lib):
+    names = [lib.mate_kernel_name(k).decode() for k in range(15)]
+    assert len(set(names)) == 15 and "unknown" not in names, names
+    assert lib.mate_kernel_name(99).decode() == "unknown"
+    assert lib.mate_trace_start(-1) == _lib.MATE_ERR_ARG
