@@ -117,6 +117,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
 // ---------------------------------------------------------------------------------------------------
 // TMA (tiled tensor copies global -> shared, completion through an mbarrier transaction count)
 // ---------------------------------------------------------------------------------------------------
+// Bulk copy (no tensor map) of `bytes` bytes, global -> shared, completion on an mbarrier transaction
+// count.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
@@ -236,9 +245,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  // no memory clobber: TMEM is not C++-visible memory, and the volatile asm statements that order TMEM
+  // traffic (tcgen05.wait::st, fences, mbarrier arrivals) keep their program order among themselves
   asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2),
-               "r"(r3)
-               : "memory");
+               "r"(r3));
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 

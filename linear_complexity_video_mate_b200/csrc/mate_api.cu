@@ -171,7 +171,7 @@ struct Carver {
 
 struct SsdScratch {
   __nv_bfloat16 *Gm, *Sf, *Sb, *Hf, *Hb;
-  float *gl, *Gd, *cs, *cdl;
+  float *gl, *Gd, *tbl;
   int* crow;
 };
 
@@ -188,8 +188,7 @@ SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh) {
   s.Hb = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
   s.gl = cv.take<float>((size_t)B * (nRc + nVc) * nh);
   s.Gd = cv.take<float>((size_t)B * nVc * kSsdQ);
-  s.cs = cv.take<float>((size_t)B * nVc * nh * kSsdQ);
-  s.cdl = cv.take<float>((size_t)B * nVc * nh * kSsdQ);
+  s.tbl = cv.take<float>((size_t)B * nVc * nh * 2 * kOutTbl);
   s.crow = cv.take<int>((size_t)B * nVc * kSsdQ);
   return s;
 }
@@ -356,8 +355,7 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   p.Hf = sc.Hf;
   p.Hb = sc.Hb;
   p.crow = sc.crow;
-  p.cs = sc.cs;
-  p.cdl = sc.cdl;
+  p.tbl = sc.tbl;
   p.y = static_cast<__nv_bfloat16*>(y);
   p.ldy = ldy;
   p.y_bstride = y_bstride;
@@ -387,9 +385,9 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
       !make_tmap(&mp.hb, sc.Hb, srows, kSsdP, kSsdP, 128) ||
       !make_tmap(&mp.g, sc.Gm, (long long)c->B * p.nVc * kSsdQ, kSsdQ, kSsdQ, 128))
     return MATE_ERR_CUDA;
-  const int out_items = c->B * p.nVc * c->nh * 2;
+  const int out_groups = c->B * p.nVc * 2;
   trace_begin(MATE_K_SSD_OUTPUT, st);
-  ssd_output_kernel<<<std::min(out_items, device_sms()), kSsdOutThreads, smem_out, st>>>(p, mp);
+  ssd_output_kernel<<<std::min(out_groups, device_sms()), kSsdOutThreads, smem_out, st>>>(p, mp);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }

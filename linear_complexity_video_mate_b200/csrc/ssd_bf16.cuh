@@ -37,6 +37,18 @@ constexpr int kSsdQ = 256;   // chunk length of the tensor-core scan
 constexpr int kSsdP = 64;    // head size
 constexpr int kSsdN = 128;   // state size
 
+// Decay tables of one (video chunk, head, 128-row tile t), written by the state kernel and read by the
+// output kernel, in floats.  Row fields are indexed by the tile row r (token i = 128 t + r), column
+// fields by the chunk column j:
+//   uf, ub   row factors exp(s_i - s_{64 ib - 1}), exp(s'_{64 ib + 64} - s'_i) of row block ib = i / 64
+//   si, sx   s_i log2(e), s'_i log2(e)               ef, eb  exp(s_i), exp(s_last - s'_i)
+//   dl       delta_i                                  wf, wb  [2][256] column factors of row blocks 2t, 2t + 1
+//   lf, lb   log2(delta_j) - s_j log2(e), log2(delta_j) + s'_j log2(e) for the tile's own columns
+// (s inclusive and s' = s - delta A exclusive cumulative sums of delta A over the chunk).
+constexpr int kTUf = 0, kTUb = 128, kTSi = 256, kTSx = 384, kTEf = 512, kTEb = 640, kTDl = 768, kTWf = 896,
+              kTWb = 1408, kTLf = 1920, kTLb = 2048, kOutTbl = 2176;
+constexpr float kLog2e = 1.4426950408889634f;
+
 struct SsdBf16Params {
   SeqRows s;
   int B, nh, nRc, nVc;
@@ -50,8 +62,7 @@ struct SsdBf16Params {
   __nv_bfloat16* Hf;  // [B][nVc][nh][N][P]  state entering video chunk v, forward traversal
   __nv_bfloat16* Hb;  // [B][nVc][nh][N][P]  state entering video chunk v, backward traversal
   int* crow;          // [B][nVc][Q]     source row of each video-chunk row (-1 past the end)
-  float* cs;          // [B][nVc][nh][Q] inclusive cumulative sum of delta * A over the chunk
-  float* cdl;         // [B][nVc][nh][Q] delta of each chunk row (0 past the end)
+  float* tbl;         // [B][nVc][nh][2][kOutTbl]  decay tables of each 128-row tile (layout below)
   __nv_bfloat16* y;   // row b*y_bstride + map(q), column h*P
   int ldy;
   long long y_bstride;
@@ -253,6 +264,7 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
   long long* srow = reinterpret_cast<long long*>(wtot + 8);   // [256]
   uint64_t* bar = reinterpret_cast<uint64_t*>(srow + 256);
   uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
+  float* bnd = reinterpret_cast<float*>(bar + 2);   // s at the ends of row blocks 0..2, s' at starts of 1..3
   const int c = blockIdx.x, b = blockIdx.y;
   const ChunkBase cb = chunk_base(p.s, c, p.nRc);
   const bool video = c >= p.nRc;
@@ -299,15 +311,36 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
     const float dl = dl_next;
     const float a = dl * A;
     const float s = block_scan_256(a, wtot);
-    if (video) {   // per-row tables of the output kernel
-      const long long cv = static_cast<long long>(b) * p.nVc + (c - p.nRc);
-      p.cs[(cv * p.nh + h) * kSsdQ + j] = s;
-      p.cdl[(cv * p.nh + h) * kSsdQ + j] = dl;
-      if (hh == 0 && blockIdx.z == 0) p.crow[cv * kSsdQ + j] = myrw >= 0 ? static_cast<int>(myrw) : -1;
-    }
+    const float sx = s - a;
     if (j == 255) wtot[8 - 1] = s;  // reuse slot 7 for s_last after the scan finished with wtot
+    if ((j & 63) == 63 && j < 255) bnd[j >> 6] = s;          // bnd[ib - 1] = s_{64 ib - 1}, ib = 1..3
+    if ((j & 63) == 0 && j > 0) bnd[4 + (j >> 6) - 1] = sx;  // bnd[4 + ib] = s'_{64 ib + 64}, ib = 0..2
     __syncthreads();
     const float s_last = wtot[7];
+    if (video) {
+      // decay tables of the output kernel (see kOutTbl); thread j is token j of the chunk
+      const long long cv = static_cast<long long>(b) * p.nVc + (c - p.nRc);
+      if (hh == 0 && blockIdx.z == 0) p.crow[cv * kSsdQ + j] = myrw >= 0 ? static_cast<int>(myrw) : -1;
+      float* T0 = p.tbl + (cv * p.nh + h) * 2 * kOutTbl;
+      float* T = T0 + (j >> 7) * kOutTbl;
+      const int r = j & 127, ib = j >> 6;
+      T[kTUf + r] = ib > 0 ? __expf(s - bnd[ib - 1]) : 0.f;
+      T[kTUb + r] = ib < 3 ? __expf(bnd[4 + ib] - sx) : 0.f;
+      T[kTSi + r] = s * kLog2e;
+      T[kTSx + r] = sx * kLog2e;
+      T[kTEf + r] = __expf(s);
+      T[kTEb + r] = __expf(s_last - sx);
+      T[kTDl + r] = dl;
+      const float l2d = dl > 0.f ? __log2f(dl) : -INFINITY;
+      T[kTLf + r] = l2d - s * kLog2e;
+      T[kTLb + r] = l2d + sx * kLog2e;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {   // column factors of row block q (stored with the tile holding it)
+        float* W = T0 + (q >> 1) * kOutTbl + (q & 1) * 256 + j;
+        W[kTWf] = (q > 0 && j < 64 * q) ? dl * __expf(bnd[q - 1] - s) : 0.f;
+        W[kTWb] = (q < 3 && j >= 64 * q + 64) ? dl * __expf(sx - bnd[4 + q]) : 0.f;
+      }
+    }
     sWf[j] = __expf(s_last - s) * dl;
     sWb[j] = __expf(s - a) * dl;
     __syncthreads();
@@ -451,20 +484,21 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 }
 
 // ---------------------------------------------------------------------------------------------------
-// Outputs of the video chunks: persistent, warp-specialised.  One work item = (sample, video chunk, head,
-// 128-row tile t of the chunk); a CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ...
+// Outputs of the video chunks: persistent, warp-specialised.  A group = (sample, video chunk, 128-row
+// tile t); a CTA walks groups blockIdx.x, blockIdx.x + gridDim.x, ... and within a group all heads in
+// turn (one work item per head).  The tile's rows of G = C B^T and of C are the same for every head, so
+// they are loaded once per group and stay in shared memory.
 //
-//   warps 0..2   loaders.  Per item: the chunk's row table and the head's cumulative sums and step sizes
-//                (written by the state kernel, fetched one item ahead) -> decay-factor tables; the item's
-//                x rows (all 256, MN-major) by TMA four-row gathers into one of two x buffers; the tile's
-//                C rows (K-major, four-row gathers) and the incoming states Hf / Hb (MN-major, 2D TMA)
-//                into the single C/H buffer once the previous item's C H^T products are done; the
-//                tile's rows of G = C B^T (2D TMA) into four 64-column slots, each refilled as soon as the
-//                transform has read it.
+//   warp 0       per item: the head's decay tables (one bulk copy) and x rows (all 256 of the chunk,
+//                MN-major, TMA four-row gathers) into one of two x buffers; the head's incoming states
+//                [Hf | Hb] (MN-major, 2D TMA) into the H buffer once the previous item's C H^T product
+//                is done.
+//   warp 1       per group: the tile's C rows (K-major, four-row gathers).
+//   warp 2       per group: the tile's rows of G (2D TMA) into four 64-column slots, each refilled once
+//                the last head of the previous group has read it.
 //   warp 3       MMA issue (lane 0 only; an issuing thread stalls while the tensor pipe is busy, so it has
 //                no other work): Yd = M x per K half of M (A from TMEM) and, after the first half,
-//                [Yf | Yb] = C [Hf | Hb]^T as one N = 128 product (which frees the C/H buffer for the next
-//                item), into one of two TMEM accumulator sets.
+//                [Yf | Yb] = C [Hf | Hb]^T as one N = 128 product, into one of two TMEM accumulator sets.
 //   warps 4..11  transform (two warps per TMEM lane quadrant, alternating 8-column chunks): form
 //                M_ij = G_ij delta_j dec(i, j) (diagonal excluded) from the G slots and store M straight
 //                into TMEM as the A operand of the MMA (two bf16 per 32-bit column), in two K halves.
@@ -475,37 +509,27 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 // reference k = 64 ib - 1 lies between them, so exp(s_i - s_j) = exp(s_i - s_k) exp(s_k - s_j) (both
 // exponents <= 0): a per-row factor times a per-(ib, j) column factor.  Columns of LATER blocks use
 // k' = 64 (ib + 1) with the exclusive sums.  Only the 64 x 64 diagonal blocks need one exponential per
-// element.
+// element, taken in the log2 domain: delta_j exp(s_i - s_j) = 2^(s_i log2e + lf_j) below the diagonal,
+// delta_j exp(s'_j - s'_i) = 2^(lb_j - s'_i log2e) above it.
 // TMEM columns: [0, 128) M; accumulator set a at 128 + 192 a: Yd [+0, +64), Yf [+64, +128), Yb [+128, +192).
 // ---------------------------------------------------------------------------------------------------
 constexpr int kOutLoadWarps = 3, kOutXformWarps = 8, kOutEpiWarps = 4;
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kOutMmaWarp = kOutLoadWarps;                                    // issues from its lane 0
 constexpr int kOutFirstXformWarp = kOutMmaWarp + 1, kOutFirstEpiWarp = kOutFirstXformWarp + kOutXformWarps;
 constexpr int kSsdOutThreads = (kOutFirstEpiWarp + kOutEpiWarps) * 32;        // 512
 static_assert(kOutFirstXformWarp % 4 == 0 && kOutFirstEpiWarp % 4 == 0, "TMEM lane quadrants follow warp % 4");
 
-struct OutTables {   // per x buffer, after the x tile
-  float sdl[256], ss[256], ssx[256];
-  float lf[256], lb[256];       // diagonal blocks: log2(delta_j) - s_j log2(e), log2(delta_j) + s'_j log2(e)
-  float uf[128], ub[128];       // per tile row
-  float gd[128];                // G_ii of the tile rows (fp32)
-  float wf[2][256], wb[2][256]; // per 64-row block of the tile (ib = 2t + q)
-  int srow[256];                // source row of each chunk row (-1 past the end of a partial chunk)
-  float D;
-};
-
 // shared memory map (offsets from the 1024-aligned base)
-constexpr uint32_t kOutXBuf = 45056;                    // x tile (32 KB) + tables, two of them
+constexpr uint32_t kOutTblBytes = kOutTbl * 4;         // 8704
+constexpr uint32_t kOutXBuf = 41984;                    // x tile (32 KB) + the head's tables, two of them
 constexpr uint32_t kOutOffTbl = 32768;
 constexpr uint32_t kOutOffC = 2 * kOutXBuf;             // C rows of the tile: 2 K blocks of 16 KB
-constexpr uint32_t kOutOffHf = kOutOffC + 32768;        // [N = 128][P = 64] MN-major
-constexpr uint32_t kOutOffHb = kOutOffHf + 16384;
-constexpr uint32_t kOutOffG = kOutOffHb + 16384;        // 4 slots of [128 rows][64 cols] K-major
+constexpr uint32_t kOutOffH = kOutOffC + 32768;         // [Hf | Hb]: 2 MN blocks of [N = 128][P = 64]
+constexpr uint32_t kOutOffG = kOutOffH + 32768;         // 4 slots of [128 rows][64 cols] K-major
 constexpr uint32_t kOutOffBar = kOutOffG + 4 * 16384;
 constexpr uint32_t kOutSmem = kOutOffBar + 256;
-static_assert(sizeof(OutTables) <= kOutXBuf - kOutOffTbl, "tables overflow the x buffer");
-static_assert(kOutOffC % 1024 == 0 && kOutOffG % 1024 == 0, "operand tiles must be 1024-byte aligned");
+static_assert(kOutOffTbl + kOutTblBytes <= kOutXBuf, "tables overflow the x buffer");
+static_assert(kOutXBuf % 1024 == 0 && kOutOffC % 1024 == 0 && kOutOffG % 1024 == 0, "1024-byte operand tiles");
 
 // Tensor maps of the output kernel: x and C rows of the video arrays (one-row boxes of 64 columns, for
 // four-row gathers), the carried states ([N rows][P] per chunk and head, 64 x 128 boxes) and G
@@ -520,32 +544,37 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOutOffBar);
-  uint64_t* x_full = bars;         // [2] x bytes + the loader threads (tables written)
+  uint64_t* x_full = bars;         // [2] x + table bytes
   uint64_t* x_empty = bars + 2;    // [2] last Yd MMA commit + 4 epilogue warps
-  uint64_t* ch_full = bars + 4;    // C + Hf + Hb bytes
-  uint64_t* ch_empty = bars + 5;   // Yf / Yb MMA commit
-  uint64_t* g_full = bars + 6;     // [4] one G slot's bytes
-  uint64_t* g_empty = bars + 10;   // [4] the 8 transform warps have read the slot
-  uint64_t* m_full = bars + 14;    // [2] per K half of M: transform -> MMA (count 256)
-  uint64_t* m_empty = bars + 16;   // [2] per K half of M: MMA commit -> transform
-  uint64_t* y_full = bars + 18;    // [2] MMA commit -> epilogue
-  uint64_t* y_empty = bars + 20;   // [2] epilogue warps -> MMA (count 4)
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint64_t* h_full = bars + 4;     // Hf + Hb bytes
+  uint64_t* h_empty = bars + 5;    // Yf / Yb MMA commit
+  uint64_t* c_full = bars + 6;     // C bytes (per group)
+  uint64_t* c_empty = bars + 7;    // last head's Yf / Yb MMA commit
+  uint64_t* g_full = bars + 8;     // [4] one G slot's bytes (per group)
+  uint64_t* g_empty = bars + 12;   // [4] the 8 transform warps have read the slot for the last head
+  uint64_t* m_full = bars + 16;    // [2] per K half of M: transform -> MMA (count 256)
+  uint64_t* m_empty = bars + 18;   // [2] per K half of M: MMA commit -> transform
+  uint64_t* y_full = bars + 20;    // [2] MMA commit -> epilogue
+  uint64_t* y_empty = bars + 22;   // [2] epilogue warps -> MMA (count 4)
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bars + 24);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nitems = p.B * p.nVc * p.nh * 2;
+  const int nh = p.nh;
+  const int ngroups = p.B * p.nVc * 2;
 
   if (threadIdx.x == 0) {
     for (int q = 0; q < 2; ++q) {
-      mbar_init(&x_full[q], kOutLoadWarps * 32 + 1);
+      mbar_init(&x_full[q], 1);
       mbar_init(&x_empty[q], 5);
-      mbar_init(&m_full[q], 256);
+      mbar_init(&m_full[q], kOutXformWarps * 32);
       mbar_init(&m_empty[q], 1);
       mbar_init(&y_full[q], 1);
-      mbar_init(&y_empty[q], 4);
+      mbar_init(&y_empty[q], kOutEpiWarps);
     }
-    mbar_init(ch_full, 1);
-    mbar_init(ch_empty, 1);
+    mbar_init(h_full, 1);
+    mbar_init(h_empty, 1);
+    mbar_init(c_full, 1);
+    mbar_init(c_empty, 1);
     for (int q = 0; q < 4; ++q) {
       mbar_init(&g_full[q], 1);
       mbar_init(&g_empty[q], kOutXformWarps);
@@ -560,169 +589,138 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
   tc_fence_after();
   const uint32_t tmem = *slot;
 
-  auto decode = [&](int it, int& b, int& v, int& h, int& t) {
-    t = it & 1;
-    int rest = it >> 1;
-    h = rest % p.nh;
-    rest /= p.nh;
+  auto decode = [&](int g, int& b, int& v, int& t) {
+    t = g & 1;
+    const int rest = g >> 1;
     v = rest % p.nVc;
     b = rest / p.nVc;
   };
+  // every exit decision inside a warp is warp-uniform (a lane leaving alone would strand __syncwarp)
+  auto wait_all = [&](uint64_t* bar, unsigned parity) { return !__any_sync(0xffffffffu, !mbar_wait(bar, parity)); };
 
-  if (warp < kOutLoadWarps) {
-    // ------------------------------------------------------------------------------ loaders
-    constexpr int NL = kOutLoadWarps * 32;   // 96 loader threads
-    const int lt = threadIdx.x;
-    // A wait that ran out is carried to the next item's first barrier, where all loader threads leave
-    // the loop together (a thread leaving alone would strand the others at a named barrier).
-    bool failed = false;
-    // per-row inputs of an item (chunk row table, cumulative sums, step sizes, G diagonal), fetched one
-    // item ahead so that their latency overlaps the previous item
-    struct RowIn {
-      int rw[3];
-      float s[3], d[3], gd[2], A, D;
+  if (warp == 0) {
+    // ------------------------------------------------------------------------------ x, tables, H
+    int rows[8], rows_next[8];   // chunk rows 8 lane .. 8 lane + 7 of the current / next group
+    auto fetch_rows = [&](int g, int (&rw)[8]) {
+      if (g >= ngroups) return;
+      int b, v, t;
+      decode(g, b, v, t);
+      const int4* src = reinterpret_cast<const int4*>(p.crow + (static_cast<long long>(b) * p.nVc + v) * kSsdQ);
+      const int4 a0 = src[2 * lane], a1 = src[2 * lane + 1];
+      rw[0] = a0.x; rw[1] = a0.y; rw[2] = a0.z; rw[3] = a0.w;
+      rw[4] = a1.x; rw[5] = a1.y; rw[6] = a1.z; rw[7] = a1.w;
     };
-    auto fetch = [&](int it, RowIn& in) {
-      if (it >= nitems) return;
-      int b, v, h, t;
-      decode(it, b, v, h, t);
-      const long long cidx = static_cast<long long>(b) * p.nVc + v;
-      const long long hidx = (cidx * p.nh + h) * kSsdQ;
-#pragma unroll
-      for (int u = 0; u < 3; ++u) {
-        const int j = lt + u * NL;
-        if (j < kSsdQ) {
-          in.rw[u] = p.crow[cidx * kSsdQ + j];
-          in.s[u] = p.cs[hidx + j];
-          in.d[u] = p.cdl[hidx + j];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-        if (lt + u * NL < 128) in.gd[u] = p.Gd[cidx * kSsdQ + t * 128 + lt + u * NL];
-      in.A = -__expf(p.A_log[h]);
-      in.D = p.Dp[h];
-    };
-    RowIn cur, nxt;
-    fetch(blockIdx.x, cur);
+    fetch_rows(blockIdx.x, rows);
     int k = 0;
-    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
-      const int buf = k & 1, use = k >> 1;
-      int b, v, h, t;
-      decode(it, b, v, h, t);
+    bool ok = true;
+    for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x) {
+      int b, v, t;
+      decode(g, b, v, t);
       const long long cidx = static_cast<long long>(b) * p.nVc + v;
-      fetch(it + gridDim.x, nxt);
-      const bool okx = mbar_wait(&x_empty[buf], (use & 1) ^ 1);
-      if (named_bar_any(1, NL, failed || !okx)) break;
-      uint8_t* XB = smem + buf * kOutXBuf;
-      OutTables& tb = *reinterpret_cast<OutTables*>(XB + kOutOffTbl);
-#pragma unroll
-      for (int u = 0; u < 3; ++u) {
-        const int j = lt + u * NL;
-        if (j < kSsdQ) {
-          tb.srow[j] = cur.rw[u];
-          tb.sdl[j] = cur.d[u];
-          tb.ss[j] = cur.s[u];
-          tb.ssx[j] = cur.s[u] - cur.d[u] * cur.A;
+      fetch_rows(g + gridDim.x, rows_next);
+      for (int h = 0; h < nh; ++h, ++k) {
+        const int buf = k & 1, use = k >> 1;
+        if (!wait_all(&x_empty[buf], (use & 1) ^ 1)) { ok = false; break; }
+        uint8_t* XB = smem + buf * kOutXBuf;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&x_full[buf], 32768 + kOutTblBytes);
+          bulk_load(XB + kOutOffTbl, p.tbl + ((cidx * nh + h) * 2 + t) * kOutTbl, kOutTblBytes, &x_full[buf]);
         }
-      }
+        __syncwarp();
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
-        if (lt + u * NL < 128) tb.gd[lt + u * NL] = cur.gd[u];
-      if (lt == 0) {
-        tb.D = cur.D;
-        mbar_arrive_expect_tx(&x_full[buf], 32768);
-      }
-      named_bar_sync(1, NL);
-      auto rowid = [&](int j) { const int rw = tb.srow[j]; return rw < 0 ? mp.rows : rw; };
-      if (lt < 64) {   // x rows: all 256 of the chunk, 4 per gather
-        tma_gather4(&mp.x, &x_full[buf], XB + lt * 512, h * kSsdP, rowid(4 * lt), rowid(4 * lt + 1),
-                    rowid(4 * lt + 2), rowid(4 * lt + 3));
+        for (int u = 0; u < 2; ++u) {   // 4 rows per gather, 8 rows per lane
+          int id[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) id[e] = rows[4 * u + e] < 0 ? mp.rows : rows[4 * u + e];
+          tma_gather4(&mp.x, &x_full[buf], XB + (2 * lane + u) * 512, h * kSsdP, id[0], id[1], id[2], id[3]);
+        }
+        if (!wait_all(h_empty, (k & 1) ^ 1)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(h_full, 32768);
+          const int hrow = static_cast<int>((cidx * nh + h) * kSsdN);
+          tma_load_2d(&mp.hf, h_full, smem + kOutOffH, 0, hrow);
+          tma_load_2d(&mp.hb, h_full, smem + kOutOffH + 16384, 0, hrow);
+        }
+        __syncwarp();
       }
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int rr = lt + u * NL;
-        if (rr < 128) {
-          const int i = t * 128 + rr, ib = i >> 6;
-          tb.uf[rr] = ib > 0 ? __expf(tb.ss[i] - tb.ss[64 * ib - 1]) : 0.f;
-          tb.ub[rr] = ib < 3 ? __expf(tb.ssx[64 * ib + 64] - tb.ssx[i]) : 0.f;
-        }
-      }
-      for (int j = lt; j < kSsdQ; j += NL) {
-        const float dj = tb.sdl[j], sj = tb.ss[j], sxj = tb.ssx[j];
-        const float l2d = dj > 0.f ? __log2f(dj) : -INFINITY;
-        tb.lf[j] = l2d - sj * kLog2e;
-        tb.lb[j] = l2d + sxj * kLog2e;
+      for (int e = 0; e < 8; ++e) rows[e] = rows_next[e];
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------------------ C rows, per group
+    int kg = 0;
+    for (int g = blockIdx.x; g < ngroups; g += gridDim.x, ++kg) {
+      int b, v, t;
+      decode(g, b, v, t);
+      const int4 r4 = reinterpret_cast<const int4*>(p.crow + (static_cast<long long>(b) * p.nVc + v) * kSsdQ +
+                                                    t * 128)[lane];
+      const int id[4] = {r4.x < 0 ? mp.rows : r4.x, r4.y < 0 ? mp.rows : r4.y, r4.z < 0 ? mp.rows : r4.z,
+                         r4.w < 0 ? mp.rows : r4.w};
+      if (!wait_all(c_empty, (kg & 1) ^ 1)) break;
+      if (lane == 0) mbar_arrive_expect_tx(c_full, 32768);
+      __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int ib = 2 * t + q;
-          tb.wf[q][j] = (ib > 0 && j < 64 * ib) ? dj * __expf(tb.ss[64 * ib - 1] - sj) : 0.f;
-          tb.wb[q][j] = (ib < 3 && j >= 64 * ib + 64) ? dj * __expf(sxj - tb.ssx[64 * ib + 64]) : 0.f;
-        }
-      }
-      mbar_arrive(&x_full[buf]);
-      if (lt >= NL - 64) {
-        // C rows of the tile and the two states, into the single C/H buffer
-        const int lc = lt - (NL - 64);   // 0..63
-        const bool okc = mbar_wait(ch_empty, (k & 1) ^ 1);
-        failed = !okc;
-        if (okc && lc == 0) {
-          mbar_arrive_expect_tx(ch_full, 65536);
-          const int hrow = static_cast<int>((cidx * p.nh + h) * kSsdN);
-          tma_load_2d(&mp.hf, ch_full, smem + kOutOffHf, 0, hrow);
-          tma_load_2d(&mp.hb, ch_full, smem + kOutOffHb, 0, hrow);
-        }
-        named_bar_sync(2, 64);
-        const int g = lc & 31, kb = lc >> 5;
-        const int j = t * 128 + 4 * g;
-        if (okc)
-          tma_gather4(&mp.c, ch_full, smem + kOutOffC + kb * 16384 + g * 512, kb * 64, rowid(j), rowid(j + 1),
-                      rowid(j + 2), rowid(j + 3));
-      } else if (lt == 0) {
-        // G rows of the tile, one 64-column slot at a time as the transform releases them
-        const int grow = static_cast<int>(cidx * kSsdQ + t * 128);
-        for (int cb = 0; cb < 4 && !failed; ++cb) {
-          failed = !mbar_wait(&g_empty[cb], (k & 1) ^ 1);
-          if (!failed) {
+      for (int kb = 0; kb < 2; ++kb)
+        tma_gather4(&mp.c, c_full, smem + kOutOffC + kb * 16384 + lane * 512, kb * 64, id[0], id[1], id[2], id[3]);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------------------ G rows, per group
+    if (lane == 0) {
+      int kg = 0;
+      bool ok = true;
+      for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x, ++kg) {
+        int b, v, t;
+        decode(g, b, v, t);
+        const int grow = static_cast<int>((static_cast<long long>(b) * p.nVc + v) * kSsdQ + t * 128);
+        for (int cb = 0; cb < 4 && ok; ++cb) {
+          ok = mbar_wait(&g_empty[cb], (kg & 1) ^ 1);
+          if (ok) {
             mbar_arrive_expect_tx(&g_full[cb], 16384);
             tma_load_2d(&mp.g, &g_full[cb], smem + kOutOffG + cb * 16384, cb * 64, grow);
           }
         }
       }
-      cur = nxt;
     }
+    __syncwarp();
   } else if (warp == kOutMmaWarp) {
     // ------------------------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t idesc_d = idesc_bf16_f32(128, 64, 0, 1);    // Yd: N = P
       const uint32_t idesc_h = idesc_bf16_f32(128, 128, 0, 1);   // [Yf | Yb]: N = 2 P, B = [Hf | Hb]
-      const uint32_t cbase = smem_u32(smem + kOutOffC), hbase = smem_u32(smem + kOutOffHf);
-      int k = 0;
-      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
-        const int buf = k & 1, use = k >> 1, acc = k & 1;
-        const uint32_t xb = smem_u32(smem + buf * kOutXBuf);
-        const uint32_t ybase = tmem + 128 + acc * 192;
-        if (!mbar_wait(&y_empty[acc], (use & 1) ^ 1) || !mbar_wait(&m_full[0], k & 1)) break;
-        tc_fence_after();
+      const uint32_t cbase = smem_u32(smem + kOutOffC), hbase = smem_u32(smem + kOutOffH);
+      int k = 0, kg = 0;
+      bool ok = true;
+      for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x, ++kg) {
+        for (int h = 0; h < nh; ++h, ++k) {
+          const int buf = k & 1, use = k >> 1, acc = k & 1;
+          const uint32_t xb = smem_u32(smem + buf * kOutXBuf);
+          const uint32_t ybase = tmem + 128 + acc * 192;
+          ok = mbar_wait(&y_empty[acc], (use & 1) ^ 1) && mbar_wait(&m_full[0], k & 1);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < 8; ++q)   // Yd = M x, first K half (M in TMEM, 8 columns per 16 elements)
-          mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, q > 0);
-        mma_commit(&m_empty[0]);
-        if (!mbar_wait(ch_full, k & 1)) break;
-        tc_fence_after();
+          for (int q = 0; q < 8; ++q)   // Yd = M x, first K half (M in TMEM, 8 columns per 16 elements)
+            mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, q > 0);
+          mma_commit(&m_empty[0]);
+          ok = mbar_wait(h_full, k & 1) && (h > 0 || mbar_wait(c_full, kg & 1));
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < 8; ++q)   // [Yf | Yb] = C [Hf | Hb]^T, K = N_state = 128
-          mma_bf16_ss(ybase + 64, desc_sw128(cbase + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
-                      desc_sw128(hbase + q * 2048, 16384, 1024), idesc_h, q > 0);
-        mma_commit(ch_empty);
-        if (!mbar_wait(&m_full[1], k & 1)) break;
-        tc_fence_after();
+          for (int q = 0; q < 8; ++q)   // [Yf | Yb] = C [Hf | Hb]^T, K = N_state = 128
+            mma_bf16_ss(ybase + 64, desc_sw128(cbase + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
+                        desc_sw128(hbase + q * 2048, 16384, 1024), idesc_h, q > 0);
+          mma_commit(h_empty);
+          if (h == nh - 1) mma_commit(c_empty);
+          ok = mbar_wait(&m_full[1], k & 1);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int q = 8; q < 16; ++q)   // Yd, second K half
-          mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, true);
-        mma_commit(&m_empty[1]);
-        mma_commit(&y_full[acc]);
-        mma_commit(&x_empty[buf]);
+          for (int q = 8; q < 16; ++q)   // Yd, second K half
+            mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, true);
+          mma_commit(&m_empty[1]);
+          mma_commit(&y_full[acc]);
+          mma_commit(&x_empty[buf]);
+        }
       }
     }
     __syncwarp();
@@ -731,147 +729,153 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
     const int xw = warp - kOutFirstXformWarp;
     const int quad = warp & 3, half = xw >> 2;
     const int r = quad * 32 + lane;
-    int k = 0;
-    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
-      const int buf = k & 1, use = k >> 1;
-      int b, v, h, t;
-      decode(it, b, v, h, t);
+    const uint32_t tm_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 4;
+    int k = 0, kg = 0;
+    bool ok = true;
+    for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x, ++kg) {
+      const int t = g & 1;
       const int i = t * 128 + r, ib = i >> 6;
-      bool ok = true;
-      // every exit decision below is warp-uniform (a lane leaving alone would strand __syncwarp)
-      if (__any_sync(0xffffffffu, !mbar_wait(&x_full[buf], use & 1))) break;
-      const OutTables& tb = *reinterpret_cast<const OutTables*>(smem + buf * kOutXBuf + kOutOffTbl);
-      const float ufi = tb.uf[r], ubi = tb.ub[r];
-      const float si2 = tb.ss[i] * kLog2e, sxi2 = tb.ssx[i] * kLog2e;
-      const float* wfr = tb.wf[ib - 2 * t];
-      const float* wbr = tb.wb[ib - 2 * t];
-      const uint32_t tm_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 4;
+      for (int h = 0; h < nh && ok; ++h, ++k) {
+        const int buf = k & 1, use = k >> 1;
+        if (!wait_all(&x_full[buf], use & 1)) { ok = false; break; }
+        const float* tb = reinterpret_cast<const float*>(smem + buf * kOutXBuf + kOutOffTbl);
+        const float ufi = tb[kTUf + r], ubi = tb[kTUb + r];
+        const float si2 = tb[kTSi + r], sxi2 = tb[kTSx + r];
+        const float* wfr = tb + kTWf + (ib - 2 * t) * 256;
+        const float* wbr = tb + kTWb + (ib - 2 * t) * 256;
 #pragma unroll 1
-      for (int cb = 0; cb < 4; ++cb) {
-        const int hh = cb >> 1;
-        if ((cb & 1) == 0) {
-          if (__any_sync(0xffffffffu, !mbar_wait(&m_empty[hh], (k & 1) ^ 1))) { ok = false; break; }
-          tc_fence_after();
-        }
-        if (__any_sync(0xffffffffu, !mbar_wait(&g_full[cb], k & 1))) { ok = false; break; }
-        const uint8_t* grow = smem + kOutOffG + cb * 16384 + r * 128;
-        const uint32_t tcol = tm_row + cb * 32;
-        if (cb != ib) {
-          const float u = cb < ib ? ufi : ubi;
-          const float* w = (cb < ib ? wfr : wbr) + cb * 64 + half * 8;
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const int ch = 2 * qq + half;
-            const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
-            const float4 wa = *reinterpret_cast<const float4*>(w + qq * 16);
-            const float4 wc = *reinterpret_cast<const float4*>(w + qq * 16 + 4);
-            const float2 g0 = unpack_bf16x2(gc.x), g1 = unpack_bf16x2(gc.y);
-            const float2 g2 = unpack_bf16x2(gc.z), g3 = unpack_bf16x2(gc.w);
-            tmem_st4(tcol + qq * 8, pack_bf16x2(g0.x * (u * wa.x), g0.y * (u * wa.y)),
-                     pack_bf16x2(g1.x * (u * wa.z), g1.y * (u * wa.w)),
-                     pack_bf16x2(g2.x * (u * wc.x), g2.y * (u * wc.y)),
-                     pack_bf16x2(g3.x * (u * wc.z), g3.y * (u * wc.w)));
+        for (int cb = 0; cb < 4; ++cb) {
+          const int hh = cb >> 1;
+          if ((cb & 1) == 0) {
+            if (!wait_all(&m_empty[hh], (k & 1) ^ 1)) { ok = false; break; }
+            tc_fence_after();
           }
-        } else {
-          // one exponential per element, in the log2 domain with delta_j folded into the column
-          // tables: delta_j exp(s_i - s_j) = 2^(s_i log2e + lf_j) below the diagonal,
-          // delta_j exp(s'_j - s'_i) = 2^(lb_j - s'_i log2e) above it; the diagonal itself is added in
-          // fp32 in the epilogue
+          if (h == 0 && !wait_all(&g_full[cb], kg & 1)) { ok = false; break; }
+          const uint8_t* grow = smem + kOutOffG + cb * 16384 + r * 128;
+          const uint32_t tcol = tm_row + cb * 32;
+          if (cb != ib) {
+            const float u = cb < ib ? ufi : ubi;
+            const float* w = (cb < ib ? wfr : wbr) + cb * 64 + half * 8;
 #pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const int ch = 2 * qq + half;
-            const int j0 = cb * 64 + ch * 8;
-            const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
-            const float4 f0 = *reinterpret_cast<const float4*>(tb.lf + j0);
-            const float4 f1 = *reinterpret_cast<const float4*>(tb.lf + j0 + 4);
-            const float4 b0 = *reinterpret_cast<const float4*>(tb.lb + j0);
-            const float4 b1 = *reinterpret_cast<const float4*>(tb.lb + j0 + 4);
-            const float lf8[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-            const float lb8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gc);
-            float m[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int jj = j0 + e;
-              const float w = ex2_approx(jj < i ? si2 + lf8[e] : lb8[e] - sxi2);
-              m[e] = jj == i ? 0.f : w;
+            for (int qq = 0; qq < 4; ++qq) {
+              const int ch = 2 * qq + half;
+              const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
+              const float4 wa = *reinterpret_cast<const float4*>(w + qq * 16);
+              const float4 wc = *reinterpret_cast<const float4*>(w + qq * 16 + 4);
+              const float2 g0 = unpack_bf16x2(gc.x), g1 = unpack_bf16x2(gc.y);
+              const float2 g2 = unpack_bf16x2(gc.z), g3 = unpack_bf16x2(gc.w);
+              tmem_st4(tcol + qq * 8, pack_bf16x2(g0.x * (u * wa.x), g0.y * (u * wa.y)),
+                       pack_bf16x2(g1.x * (u * wa.z), g1.y * (u * wa.w)),
+                       pack_bf16x2(g2.x * (u * wc.x), g2.y * (u * wc.y)),
+                       pack_bf16x2(g3.x * (u * wc.z), g3.y * (u * wc.w)));
             }
-            uint32_t pk[4];
+          } else {
+            // one exponential per element in the log2 domain; the diagonal itself is added in fp32 in
+            // the epilogue
+            const float* lfr = tb + kTLf - 128 * t;
+            const float* lbr = tb + kTLb - 128 * t;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 gf = unpack_bf16x2(gu[e]);
-              pk[e] = pack_bf16x2(gf.x * m[2 * e], gf.y * m[2 * e + 1]);
+            for (int qq = 0; qq < 4; ++qq) {
+              const int ch = 2 * qq + half;
+              const int j0 = cb * 64 + ch * 8;
+              const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
+              const float4 f0 = *reinterpret_cast<const float4*>(lfr + j0);
+              const float4 f1 = *reinterpret_cast<const float4*>(lfr + j0 + 4);
+              const float4 b0 = *reinterpret_cast<const float4*>(lbr + j0);
+              const float4 b1 = *reinterpret_cast<const float4*>(lbr + j0 + 4);
+              const float lf8[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+              const float lb8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+              const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gc);
+              float m[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int jj = j0 + e;
+                const float wv = ex2_approx(jj < i ? si2 + lf8[e] : lb8[e] - sxi2);
+                m[e] = jj == i ? 0.f : wv;
+              }
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 gf = unpack_bf16x2(gu[e]);
+                pk[e] = pack_bf16x2(gf.x * m[2 * e], gf.y * m[2 * e + 1]);
+              }
+              tmem_st4(tcol + qq * 8, pk[0], pk[1], pk[2], pk[3]);
             }
-            tmem_st4(tcol + qq * 8, pk[0], pk[1], pk[2], pk[3]);
           }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&g_empty[cb]);
-        if (cb & 1) {
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&m_full[hh]);
+          if (h == nh - 1) {   // the group's last head has read this G slot
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&g_empty[cb]);
+          }
+          if (cb & 1) {
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&m_full[hh]);
+          }
         }
       }
-      if (!ok) break;
     }
   } else {
     // ------------------------------------------------------------------------------ epilogue
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     int k = 0;
-    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++k) {
-      const int buf = k & 1, acc = k & 1, use = k >> 1;
-      int b, v, h, t;
-      decode(it, b, v, h, t);
+    bool ok = true;
+    for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x) {
+      int b, v, t;
+      decode(g, b, v, t);
       const int i = t * 128 + r;
       const int len = min(kSsdQ, p.s.n - v * kSsdQ);
-      const bool ok = i < len;
-      __nv_bfloat16* yrow = p.y + (b * p.y_bstride + p.s.map(v * kSsdQ + (ok ? i : 0))) * p.ldy + h * kSsdP;
-      if (__any_sync(0xffffffffu, !mbar_wait(&y_full[acc], use & 1))) break;
-      tc_fence_after();
-      const uint8_t* XB = smem + buf * kOutXBuf;
-      const OutTables& tb = *reinterpret_cast<const OutTables*>(XB + kOutOffTbl);
-      const float si = tb.ss[i], sxi = tb.ssx[i], slast = tb.ss[255], dli = tb.sdl[i];
-      const float D2 = 2.f * (tb.D + (ok ? tb.gd[r] * dli : 0.f));
-      // x row of this token (packed bf16 pairs) for the skip and diagonal terms
-      uint32_t xw[32];
+      const bool valid = i < len;
+      const float gdi = p.Gd[(static_cast<long long>(b) * p.nVc + v) * kSsdQ + i];
+      const long long yrow = b * p.y_bstride + p.s.map(v * kSsdQ + (valid ? i : 0));
+      for (int h = 0; h < nh; ++h, ++k) {
+        const int buf = k & 1, acc = k & 1, use = k >> 1;
+        const float Dh = p.Dp[h];
+        if (!wait_all(&y_full[acc], use & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint8_t* XB = smem + buf * kOutXBuf;
+        const float* tb = reinterpret_cast<const float*>(XB + kOutOffTbl);
+        const float ef = tb[kTEf + r], eb = tb[kTEb + r], dli = tb[kTDl + r];
+        const float D2 = 2.f * (Dh + (valid ? gdi * dli : 0.f));
+        // x row of this token (packed bf16 pairs) for the skip and diagonal terms
+        uint32_t xw[32];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(XB + sw128_mnmajor_offset(i, q * 8, 32768));
-        xw[q * 4 + 0] = xv.x; xw[q * 4 + 1] = xv.y; xw[q * 4 + 2] = xv.z; xw[q * 4 + 3] = xv.w;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&x_empty[buf]);
-      const float ef = __expf(si);
-      const float eb = __expf(slast - sxi);
-      const uint32_t ybase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128 + acc * 192;
-#pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {   // 16 columns at a time
-        uint32_t yd[16], yf[16], yb[16];
-        tmem_ld16(ybase + pc * 16, yd);
-        tmem_ld16(ybase + 64 + pc * 16, yf);
-        tmem_ld16(ybase + 128 + pc * 16, yb);
-        tmem_wait_ld();
-        if (ok) {
-          uint32_t ou[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 xf = unpack_bf16x2(xw[pc * 8 + e]);
-            const int k0 = 2 * e;
-            const float y0 = __uint_as_float(yd[k0]) + ef * __uint_as_float(yf[k0]) + eb * __uint_as_float(yb[k0]) + D2 * xf.x;
-            const float y1 = __uint_as_float(yd[k0 + 1]) + ef * __uint_as_float(yf[k0 + 1]) +
-                             eb * __uint_as_float(yb[k0 + 1]) + D2 * xf.y;
-            ou[e] = pack_bf16x2(y0, y1);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(yrow + pc * 16);
-          dst[0] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
-          dst[1] = make_uint4(ou[4], ou[5], ou[6], ou[7]);
+        for (int q = 0; q < 8; ++q) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(XB + sw128_mnmajor_offset(i, q * 8, 32768));
+          xw[q * 4 + 0] = xv.x; xw[q * 4 + 1] = xv.y; xw[q * 4 + 2] = xv.z; xw[q * 4 + 3] = xv.w;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&x_empty[buf]);
+        __nv_bfloat16* ydst = p.y + yrow * p.ldy + h * kSsdP;
+        const uint32_t ybase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128 + acc * 192;
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {   // 16 columns at a time
+          uint32_t yd[16], yf[16], yb[16];
+          tmem_ld16(ybase + pc * 16, yd);
+          tmem_ld16(ybase + 64 + pc * 16, yf);
+          tmem_ld16(ybase + 128 + pc * 16, yb);
+          tmem_wait_ld();
+          if (valid) {
+            uint32_t ou[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float2 xf = unpack_bf16x2(xw[pc * 8 + e]);
+              const int k0 = 2 * e;
+              const float y0 = __uint_as_float(yd[k0]) + ef * __uint_as_float(yf[k0]) +
+                               eb * __uint_as_float(yb[k0]) + D2 * xf.x;
+              const float y1 = __uint_as_float(yd[k0 + 1]) + ef * __uint_as_float(yf[k0 + 1]) +
+                               eb * __uint_as_float(yb[k0 + 1]) + D2 * xf.y;
+              ou[e] = pack_bf16x2(y0, y1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(ydst + pc * 16);
+            dst[0] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+            dst[1] = make_uint4(ou[4], ou[5], ou[6], ou[7]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&y_empty[acc]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&y_empty[acc]);
     }
   }
   tc_fence_before();
