@@ -415,6 +415,7 @@ mate_status run_tesa(const mate_config* c, const void* qkv, int ldq, int qcol, i
   p.O = static_cast<__nv_bfloat16*>(O);
   p.ldo = ldo;
   p.ocol = ocol;
+  p.B = c->B;
   p.T = c->T;
   p.H = c->H;
   p.W = c->W;
@@ -427,11 +428,11 @@ mate_status run_tesa(const mate_config* c, const void* qkv, int ldq, int qcol, i
   p.sw = sft ? c->sw : 0;
   p.shifted = sft;
   p.scale_log2 = 1.4426950408889634f / std::sqrt(static_cast<float>(c->tp));
-  const size_t smem = 1024 + 196608 + 2048 + 1024 + 2048 + 64;
+  const size_t smem = 1024 + kTesaSmem;
   if (!set_smem(tesa_bf16_kernel, smem)) return MATE_ERR_CUDA;
-  const int nwin = (c->T / c->wt) * (c->H / c->wh) * (c->W / c->ww);
+  const int nitems = (c->T / c->wt) * (c->H / c->wh) * (c->W / c->ww) * c->B * c->th;
   trace_begin(MATE_K_TESA, st);
-  tesa_bf16_kernel<<<dim3(nwin, c->B, c->th), kTesaThreads, smem, st>>>(p);
+  tesa_bf16_kernel<<<std::min(nitems, device_sms()), kTesaThreads, smem, st>>>(p);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }
