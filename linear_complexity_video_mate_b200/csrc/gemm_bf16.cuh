@@ -5,9 +5,10 @@
 // [y | O] x [W_out | W_o]^T, so Out = MA + TE falls out of the K reduction).  The projections are the
 // in/out maps around the bidirectional Mamba2 block and the attention (abstract: MATE = MA + TE).
 //
-// Design (one CTA per SM, 6 warps):
+// Design (clusters of 2 CTAs, one CTA per SM, 6 warps each; see the two-SM section below):
 //   warp 0      TMA producer: A and B tiles (BK = 64, 128-byte swizzle) into an S-stage ring;
-//   warp 1      MMA issuer: 128 x BN x 16 tcgen05.mma into one of two TMEM accumulators;
+//   warp 1      MMA issuer (leader CTA): 256 x BN x 16 tcgen05.mma.cta_group::2 into one of two TMEM
+//               accumulators;
 //   warps 2..5  epilogue: tcgen05.ld the finished accumulator, convert, store; the other accumulator
 //               is being filled meanwhile.
 // Optional epilogue side output: columns [dt_col0, dt_col0 + dt_cols) also produce
@@ -38,146 +39,6 @@ constexpr int kGemmThreads = 192;
 __host__ __device__ inline uint32_t gemm_stage_bytes(int bn) { return kGemmBM * 128 + bn * 128; }
 
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(__expf(v)); }
-
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t stage_bytes = gemm_stage_bytes(p.bn);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.stages * stage_bytes);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + p.stages;
-  uint64_t* tfull = bars + 2 * p.stages;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int nk = p.K / kGemmBK;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < p.stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
-    }
-    mbar_fence_init();
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int mb = tile / p.num_n_tiles, nb = tile % p.num_n_tiles;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-          uint8_t* sa = smem + stage * stage_bytes;
-          mbar_arrive_expect_tx(&full[stage], stage_bytes);
-          tma_load_2d(&tmA, &full[stage], sa, kb * kGemmBK, mb * kGemmBM);
-          tma_load_2d(&tmB, &full[stage], sa + kGemmBM * 128, kb * kGemmBK, nb * p.bn);
-          if (++stage == (uint32_t)p.stages) { stage = 0; phase ^= 1; }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kGemmBM, p.bn, 0, 0);
-      uint32_t stage = 0, phase = 0;
-      int it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_par = (it >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], acc_par ^ 1)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * 256;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * stage_bytes);
-          const uint32_t sb = sa + kGemmBM * 128;
-#pragma unroll
-          for (int k = 0; k < kGemmBK / 16; ++k) {
-            mma_bf16_ss(d_tmem, desc_sw128(sa + k * 32, 16, 1024), desc_sw128(sb + k * 32, 16, 1024), idesc,
-                        (kb | k) != 0);
-          }
-          mma_commit(&empty[stage]);
-          if (++stage == (uint32_t)p.stages) { stage = 0; phase ^= 1; }
-        }
-        mma_commit(&tfull[acc]);
-      }
-    }
-  } else {
-    // epilogue warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1
-    const int quad = warp & 3;
-    int it = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
-      const int mb = tile / p.num_n_tiles, nb = tile % p.num_n_tiles;
-      const int acc = it & 1;
-      const uint32_t acc_par = (it >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], acc_par)) break;
-      tc_fence_after();
-      const int row = mb * kGemmBM + quad * 32 + lane;
-      const bool row_ok = row < p.M;
-      __nv_bfloat16* crow = p.C + static_cast<size_t>(row) * p.ldc;
-      for (int c0 = 0; c0 < p.bn; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256 + c0, r);
-        tmem_wait_ld();
-        const int col0 = nb * p.bn + c0;
-        // columns of this tile only: the last 32-column slice of a tile with bn % 32 != 0 is partial
-        const int col_end = min(p.N, nb * p.bn + p.bn);
-        if (!row_ok || col0 >= col_end) continue;
-        if (col0 + 32 <= col_end) {
-          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 pk;
-            pk.x = pack_bf16x2(__uint_as_float(r[v * 8 + 0]), __uint_as_float(r[v * 8 + 1]));
-            pk.y = pack_bf16x2(__uint_as_float(r[v * 8 + 2]), __uint_as_float(r[v * 8 + 3]));
-            pk.z = pack_bf16x2(__uint_as_float(r[v * 8 + 4]), __uint_as_float(r[v * 8 + 5]));
-            pk.w = pack_bf16x2(__uint_as_float(r[v * 8 + 6]), __uint_as_float(r[v * 8 + 7]));
-            dst[v] = pk;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < col_end) crow[col0 + j] = __float2bfloat16_rn(__uint_as_float(r[j]));
-        }
-        if (p.delta != nullptr && col0 < p.dt_col0 + p.dt_cols && col0 + 32 > p.dt_col0) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int c = col0 + j - p.dt_col0;
-            if (c >= 0 && c < p.dt_cols && col0 + j < col_end)
-              p.delta[static_cast<size_t>(row) * p.ld_delta + c] = softplus_f(__uint_as_float(r[j]) + p.dt_bias[c]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
-  }
-}
 
 // ---------------------------------------------------------------------------------------------------
 // Two-SM variant: a cluster of 2 CTAs computes a 256 x BN tile with tcgen05.mma.cta_group::2.  Each CTA

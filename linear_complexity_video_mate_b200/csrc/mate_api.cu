@@ -249,9 +249,6 @@ mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const
   p.K = K;
   p.bn = choose_bn(N);
   p.num_n_tiles = ceil_div(N, p.bn);
-  p.num_tiles = ceil_div(M, kGemmBM) * p.num_n_tiles;
-  const uint32_t sb = gemm_stage_bytes(p.bn);
-  p.stages = std::min<int>(8, static_cast<int>((kSmemLimit - 1024 - 256) / sb));
   p.C = static_cast<__nv_bfloat16*>(C);
   p.ldc = ldc;
   p.delta = delta;
