@@ -110,6 +110,32 @@ def measured_peaks():
         return 6650.0, 1400.0, "fallback (bf16 sustained)"
 
 
+# DRAM bytes per launch measured with ncu (dram__bytes_read.sum + dram__bytes_write.sum), scaled to the
+# bench workload as the profile summary explains; valid only while the kernel source is the one captured.
+MEASURED_TRAFFIC = {
+    "in_projection": {"bytes": 2.639e9, "source": "linear_complexity_video_mate_b200/csrc/gemm_bf16.cuh",
+                      "sha1": "f7a250cbda08da22dcec652ea86f7ef23fe682ae",
+                      "profile": "profiles/gemm_bf16_pair_in_projection_bf16_64x32x32.md",
+                      "workload": "bf16_256x32x32"},
+}
+
+
+def measured_traffic(kernel, workload):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu capture, or None if there is none for
+    this workload or the kernel source changed since it was taken."""
+    import hashlib
+    m = MEASURED_TRAFFIC.get(kernel)
+    if m is None or m["workload"] != workload:
+        return None
+    try:
+        with open(os.path.join(ROOT, m["source"]), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != m["sha1"]:
+                return None
+    except OSError:
+        return None
+    return m["bytes"]
+
+
 def kernel_work(cfg):
     """Algorithmic work per launch of the kernels the roofline can name: (bound, amount, unit)."""
     nin = cfg.nh * cfg.P + 2 * cfg.N + cfg.nh
@@ -287,7 +313,8 @@ def main():
         "block_tflops": total_flops / (ms * 1e-3) / 1e12,
         "block_frac_of_bf16_peak": total_flops / (ms * 1e-3) / 1e12 / tf_peak,
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": tf_peak, "unit": runit,
-                     "frac": achieved / tf_peak, "traffic": None, "peak_source": peak_src,
+                     "frac": achieved / tf_peak, "traffic": measured_traffic(dom, args.config),
+                     "traffic_unit": "bytes per launch", "peak_source": peak_src,
                      "kernel_ms": dom_ms, "launches_timed": per[dom][0],
                      "timing": "CUDA events around each launch inside the timed region (library trace)"},
         "kernels": kernels,
