@@ -176,6 +176,30 @@ def run_oracle_sample(cfg, frames, steps, warmup):
     return tokens / dt, dt, cores, scfg
 
 
+# ------------------------------------------------------------------------------ multi-rank plumbing
+# One process per GPU, each running its own block on its own seeded inputs (replicas: the block has no
+# data-path collective); the job's time is the slowest rank's.
+
+def replica_seed(cfg, rank: int) -> int:
+    return cfg.seed + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of x over all ranks (x itself when world == 1)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job tokens/s: the tokens every rank processed in one step over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms * 1e-3)
+
+
 def reference_arm(args, rank):
     if rank != 0:
         return 0
@@ -223,7 +247,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     cfg = mi.CONFIGS[args.config]
-    w = mi.make_inputs(cfg, seed=cfg.seed + 1000 * rank)   # every rank runs its own block (weak scaling)
+    w = mi.make_inputs(cfg, seed=replica_seed(cfg, rank))   # every rank runs its own block (weak scaling)
     blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
     X = torch.as_tensor(w["X"]).to(device="cuda", dtype=torch.bfloat16)
     out = torch.empty_like(X)
@@ -254,11 +278,7 @@ def main():
     barrier()
     clocks = sampler.stop()
     records = trace.read()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, "cuda")
     status = M.device_status()
 
     # per-kernel device times over the timed region; the roofline names the kernel with the largest total
@@ -290,15 +310,11 @@ def main():
         blk.forward_host(xh, s % 4, oh)
     h1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = h0.elapsed_time(h1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.e2e_steps, world, "cuda")
     nbytes = X.numel() * X.element_size()
 
     tokens_per_step = cfg.B * cfg.n
-    value = tokens_per_step * world / (ms * 1e-3)
+    value = job_value(tokens_per_step, world, ms)
     fl = flops_per_block(cfg)
     total_flops = sum(fl.values())
     line = {
@@ -318,7 +334,7 @@ def main():
                      "kernel_ms": dom_ms, "launches_timed": per[dom][0],
                      "timing": "CUDA events around each launch inside the timed region (library trace)"},
         "kernels": kernels,
-        "e2e": {"value": tokens_per_step * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": nbytes,
+        "e2e": {"value": job_value(tokens_per_step, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": nbytes,
                 "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms, "api": "mate_forward_host"},
         "gpu_launches": len(records),
         "clocks": clocks,
