@@ -755,6 +755,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           const uint32_t tcol = tm_row + cb * 32;
           if (cb != ib) {
             const float u = cb < ib ? ufi : ubi;
+            const float2 uu = make_float2(u, u);
             const float* w = (cb < ib ? wfr : wbr) + cb * 64 + half * 8;
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
@@ -762,12 +763,13 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
               const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
               const float4 wa = *reinterpret_cast<const float4*>(w + qq * 16);
               const float4 wc = *reinterpret_cast<const float4*>(w + qq * 16 + 4);
-              const float2 g0 = unpack_bf16x2(gc.x), g1 = unpack_bf16x2(gc.y);
-              const float2 g2 = unpack_bf16x2(gc.z), g3 = unpack_bf16x2(gc.w);
-              tmem_st4(tcol + qq * 8, pack_bf16x2(g0.x * (u * wa.x), g0.y * (u * wa.y)),
-                       pack_bf16x2(g1.x * (u * wa.z), g1.y * (u * wa.w)),
-                       pack_bf16x2(g2.x * (u * wc.x), g2.y * (u * wc.y)),
-                       pack_bf16x2(g3.x * (u * wc.z), g3.y * (u * wc.w)));
+              // the same products as g * (u * w) elementwise, two per instruction
+              const float2 m0 = mul_f32x2(unpack_bf16x2(gc.x), mul_f32x2(uu, make_float2(wa.x, wa.y)));
+              const float2 m1 = mul_f32x2(unpack_bf16x2(gc.y), mul_f32x2(uu, make_float2(wa.z, wa.w)));
+              const float2 m2 = mul_f32x2(unpack_bf16x2(gc.z), mul_f32x2(uu, make_float2(wc.x, wc.y)));
+              const float2 m3 = mul_f32x2(unpack_bf16x2(gc.w), mul_f32x2(uu, make_float2(wc.z, wc.w)));
+              tmem_st4(tcol + qq * 8, pack_bf16x2(m0.x, m0.y), pack_bf16x2(m1.x, m1.y), pack_bf16x2(m2.x, m2.y),
+                       pack_bf16x2(m3.x, m3.y));
             }
           } else {
             // one exponential per element in the log2 domain; the diagonal itself is added in fp32 in
@@ -796,8 +798,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
               uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const float2 gf = unpack_bf16x2(gu[e]);
-                pk[e] = pack_bf16x2(gf.x * m[2 * e], gf.y * m[2 * e + 1]);
+                const float2 gm = mul_f32x2(unpack_bf16x2(gu[e]), make_float2(m[2 * e], m[2 * e + 1]));
+                pk[e] = pack_bf16x2(gm.x, gm.y);
               }
               tmem_st4(tcol + qq * 8, pk[0], pk[1], pk[2], pk[3]);
             }
