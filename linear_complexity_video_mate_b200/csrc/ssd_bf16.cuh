@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
     const long long ci = (static_cast<long long>(b) * nC + c) * p.nh + h;
     step(p.gl[ci], __ldg(reinterpret_cast<const uint4*>(p.Sf + ci * PN) + e8));
   }
-  constexpr int U = 4;
+  constexpr int U = 16;   // chunks in flight per thread (4: 0.30 ms, 8: 0.27 ms, 16: 0.22 ms at 1024 chunks)
   for (int k0 = 0; k0 < p.nVc; k0 += U) {
     uint4 sv[U];
     float gv[U];
