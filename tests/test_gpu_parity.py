@@ -31,7 +31,8 @@ def cast(cfg, a):
     return mi.round_to_bf16(a) if cfg.dtype == "bf16" else np.asarray(a, np.float32)
 
 
-SMALL = ["tiny_f32_4x8x8", "f32_b2_4x8x12", "bf16_small_8x16x16", "bf16_ragged_12x16x24", "bf16_b2_20x16x16_d512"]
+SMALL = ["tiny_f32_4x8x8", "f32_b2_4x8x12", "bf16_small_8x16x16", "bf16_ragged_12x16x24", "bf16_b2_20x16x16_d512",
+         "bf16_onechunk_4x8x8", "bf16_noreview_b2_8x16x16"]
 
 
 # ------------------------------------------------------------------ Rotary Major Scan + review tokens

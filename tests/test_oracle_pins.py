@@ -350,3 +350,74 @@ def test_config_shapes_are_consistent():
         assert cfg.T % cfg.wt == 0 and cfg.H % cfg.wh == 0 and cfg.W % cfg.ww == 0
         O.review_grid(cfg.T, cfg.H, cfg.W, cfg.R)   # pool factors integral
         assert 0 < cfg.st < cfg.wt and 0 < cfg.sh < cfg.wh and 0 < cfg.sw < cfg.ww
+
+
+# ------------------------------------------------------------------ scan locality (news article, RMS paragraphs)
+
+from oracle import scan_locality as SL  # noqa: E402
+
+
+def _axis_pairs(T, H, W):
+    return {"T": (T - 1) * H * W, "H": T * (H - 1) * W, "W": T * H * (W - 1)}
+
+
+@pytest.mark.parametrize("grid", [(4, 8, 8), (3, 5, 7), (16, 4, 2), (1, 6, 5)])
+@pytest.mark.parametrize("order", range(4))
+def test_locality_of_scan_orders_closed_form(grid, order):
+    """Along the fastest axis of an order neighbours are 1 apart, along the second the size of the fastest,
+    along the slowest the product of the two faster sizes."""
+    T, H, W = grid
+    size = {"T": T, "H": H, "W": W}
+    a1, a2, a3 = O.SCAN_ORDERS[order]
+    stride = {a1: 1, a2: size[a1], a3: size[a1] * size[a2]}
+    pairs = _axis_pairs(T, H, W)
+    total, n, largest = SL.scan_locality(T, H, W, order)
+    assert n == sum(pairs.values())
+    assert total == sum(pairs[a] * stride[a] for a in "THW")
+    assert largest == max(stride[a] for a in "THW" if pairs[a] > 0)
+
+
+@pytest.mark.parametrize("grid", [(4, 8, 8), (3, 5, 7), (1, 1, 9)])
+def test_locality_of_rms_rotation_is_one_per_pair(grid):
+    """Every axis is the fastest axis of one of the four orders, so over a rotation cycle every adjacent
+    pair is once consecutive in the sequence."""
+    total, n, largest = SL.scan_locality(*grid, 6)
+    assert total == n and largest == 1
+
+
+@pytest.mark.parametrize("kind,grid", [(4, (3, 4, 5)), (4, (2, 2, 2)), (5, (4, 4, 4)), (5, (8, 2, 2)), (5, (16, 8, 8))])
+def test_zigzag_and_hilbert_are_unit_step_bijections(kind, grid):
+    """Both maps visit every token once; consecutive positions are grid neighbours (for Hilbert, inside
+    each cube), which is the defining property of the two paths."""
+    T, H, W = grid
+    pos = SL.positions(T, H, W, kind)
+    n = T * H * W
+    assert np.array_equal(np.sort(pos.ravel()), np.arange(n))
+    coords = np.empty((n, 3), dtype=np.int64)
+    coords[pos.ravel()] = np.stack(np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij"), -1).reshape(-1, 3)
+    steps = np.abs(np.diff(coords, axis=0)).sum(1)
+    if kind == 5:
+        cube = H ** 3
+        inside = (np.arange(1, n) % cube) != 0
+        assert np.all(steps[inside] == 1)
+        assert np.all(coords[::cube] % H == 0)           # each cube's curve starts at its origin corner
+    else:
+        assert np.all(steps == 1)
+
+
+@pytest.mark.parametrize("kind", range(7))
+def test_locality_against_brute_force(kind):
+    """All token pairs, adjacency decided from the coordinates."""
+    T, H, W = (4, 4, 4)
+    if kind == 6:
+        pos = [SL.positions(T, H, W, o) for o in range(4)]
+    else:
+        pos = [SL.positions(T, H, W, kind)]
+    pts = [(t, h, w) for t in range(T) for h in range(H) for w in range(W)]
+    total = n = largest = 0
+    for i, a in enumerate(pts):
+        for b in pts[i + 1:]:
+            if sum(abs(x - y) for x, y in zip(a, b)) == 1:
+                d = min(abs(int(p[a]) - int(p[b])) for p in pos)
+                total, n, largest = total + d, n + 1, max(largest, d)
+    assert SL.scan_locality(T, H, W, kind) == (total, n, largest)
