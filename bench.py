@@ -313,6 +313,21 @@ def main():
     e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.e2e_steps, world, "cuda")
     nbytes = X.numel() * X.element_size()
 
+    # scan locality of the workload's grid (outside the timed region): mean sequence distance of
+    # grid-adjacent tokens per index map, computed by the library's kernel
+    locality = {}
+    l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0.record(stream)
+    for kind, name in enumerate(M.LOCALITY_MAPS):
+        if kind == 5 and (cfg.H != cfg.W or cfg.H & (cfg.H - 1) or cfg.T % cfg.H):
+            continue
+        sm, npairs, mx = M.scan_locality(cfg.T, cfg.H, cfg.W, kind)
+        locality[name] = {"mean": sm / npairs, "max": mx}
+    l1.record(stream)
+    torch.cuda.synchronize()
+    locality["pairs"] = npairs
+    locality["ms_all_maps"] = l0.elapsed_time(l1)
+
     tokens_per_step = cfg.B * cfg.n
     value = job_value(tokens_per_step, world, ms)
     fl = flops_per_block(cfg)
@@ -337,6 +352,7 @@ def main():
         "e2e": {"value": job_value(tokens_per_step, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": nbytes,
                 "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms, "api": "mate_forward_host"},
         "gpu_launches": len(records),
+        "scan_locality": locality,
         "clocks": clocks,
         "device_status": status,
     }

@@ -185,6 +185,21 @@ MATE_API mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const
 MATE_API mate_status tesa_forward(const void* qkv, void* O, int shifted, const mate_config* cfg, mate_stream_t stream);
 
 /*
+ * Scan locality ([NEWS] method, Rotary Major Scan paragraphs; [FEAT] 功能特色 / RMS: the alternating
+ * orders bring the average distance, after the scan, between originally adjacent tokens down to the level
+ * of Zigzag and Hilbert scans).  Over all pairs of tokens of a T x H x W grid that differ by one step along
+ * one axis, the distance of their positions in the sequence of index map `map`:
+ *   0..3  the Rotary Major Scan orders (as rms_permute);
+ *   4     Zigzag: 3D boustrophedon (w fastest, reversing on every (t, h) line; h reversing on every t plane);
+ *   5     Hilbert: cubes of side H = W stacked along t, each along the 3D Hilbert curve; needs H = W a power
+ *         of two dividing T (MATE_ERR_UNSUPPORTED otherwise);
+ *   6     the four orders' rotation: per pair the smallest distance over the four orders.
+ * out: DEVICE array of 3 unsigned long long (8-byte aligned), overwritten on `stream` with the sum of the
+ * distances, the number of pairs and the largest distance.  Integer arithmetic: exact.
+ */
+MATE_API mate_status mate_scan_locality(int T, int H, int W, int map, unsigned long long* out, mate_stream_t stream);
+
+/*
  * Tensor-core projection used by the block's in/out maps: C[M, N] = A[M, K] W[N, K]^T in bf16 with
  * fp32 accumulation (row strides lda, ldw, ldc in elements, multiples of 8; K a multiple of 64).
  * bf16 only (cfg is not needed); MATE_ERR_UNSUPPORTED otherwise.
@@ -250,7 +265,8 @@ typedef enum {
   MATE_K_TESA_F32 = 11,
   MATE_K_OUT_PROJ = 12,        /* fused out-projection [y | O] [W_out | W_o]^T (the branch sum) */
   MATE_K_RMS_GATHER = 13,
-  MATE_K_PROJECT = 14          /* mate_project_bf16 */
+  MATE_K_PROJECT = 14,         /* mate_project_bf16 */
+  MATE_K_SCAN_LOCALITY = 15    /* mate_scan_locality */
 } mate_kernel;
 
 typedef struct {

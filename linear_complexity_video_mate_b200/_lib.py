@@ -16,6 +16,7 @@ EXPORTS = (
     "rms_unpermute", "review_pool", "ssd_scan_bidir", "tesa_forward", "mate_forward", "mate_forward_host",
     "mate_forward_host_workspace_bytes", "mate_device_status", "mate_last_launch_count", "mate_project_bf16",
     "ssd_scan_bidir_noalloc", "mate_trace_start", "mate_trace_stop", "mate_trace_read", "mate_kernel_name",
+    "mate_scan_locality",
 )
 
 _CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp", "wt", "wh", "ww", "st", "sh", "sw")
@@ -68,6 +69,7 @@ def load():
         "mate_trace_stop": (ci, []),
         "mate_trace_read": (ci, [ctypes.POINTER(CTraceRecord), ci]),
         "mate_kernel_name": (ctypes.c_char_p, [ci]),
+        "mate_scan_locality": (ci, [ci, ci, ci, ci, vp, vp]),
         "tesa_forward": (ci, [vp, vp, ci, cfgp, vp]),
         "mate_forward": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
         "mate_forward_host": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),

@@ -18,6 +18,7 @@
 #include "simt.cuh"
 #include "ssd_bf16.cuh"
 #include "tesa_bf16.cuh"
+#include "locality.cuh"
 
 using namespace mate;
 
@@ -657,6 +658,29 @@ mate_status tesa_forward(const void* qkv, void* O, int shifted, const mate_confi
   return run_tesa(cfg, qkv, 3 * a, 0, a, 2 * a, O, a, 0, shifted, reinterpret_cast<cudaStream_t>(stream));
 }
 
+mate_status mate_scan_locality(int T, int H, int W, int map, unsigned long long* out, mate_stream_t stream) {
+  if (out == nullptr || T <= 0 || H <= 0 || W <= 0 || map < 0 || map > 6 || (reinterpret_cast<uintptr_t>(out) & 7))
+    return MATE_ERR_ARG;
+  if (static_cast<long long>(T) * H * W >= (1LL << 31)) return MATE_ERR_SHAPE;
+  int bits = 1;
+  if (map == 5) {
+    if (H != W || (H & (H - 1)) != 0 || T % H != 0) return MATE_ERR_UNSUPPORTED;
+    while ((1 << bits) < H) ++bits;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  if (cudaMemsetAsync(out, 0, 3 * sizeof(unsigned long long), st) != cudaSuccess) {
+    cudaGetLastError();
+    return MATE_ERR_CUDA;
+  }
+  const long long n = static_cast<long long>(T) * H * W;
+  const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, (long long)device_sms() * 8));
+  trace_begin(MATE_K_SCAN_LOCALITY, st);
+  scan_locality_kernel<<<blocks, 256, 0, st>>>(T, H, W, map, bits, out);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
 mate_status mate_project_bf16(const void* A, int lda, long long M, int K, const void* Wt, int ldw, int N, void* C,
                               int ldc, mate_stream_t stream) {
   if (A == nullptr || Wt == nullptr || C == nullptr || M < 0 || K <= 0 || N <= 0) return MATE_ERR_ARG;
@@ -764,6 +788,7 @@ const char* mate_kernel_name(int kernel) {
     case MATE_K_OUT_PROJ: return "out_projection";
     case MATE_K_RMS_GATHER: return "rms_gather";
     case MATE_K_PROJECT: return "project";
+    case MATE_K_SCAN_LOCALITY: return "scan_locality";
   }
   return "unknown";
 }

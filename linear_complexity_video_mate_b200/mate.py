@@ -210,3 +210,16 @@ class KernelTrace:
         if n < 0:
             raise _lib.MateError(_lib.MATE_ERR_CUDA, "mate_trace_read")
         return [(lib.mate_kernel_name(recs[r].kernel).decode(), float(recs[r].ms)) for r in range(n)]
+
+
+LOCALITY_MAPS = ("rms_order0", "rms_order1", "rms_order2", "rms_order3", "zigzag", "hilbert", "rms_rotation")
+
+
+def scan_locality(T: int, H: int, W: int, kind: int, stream=None):
+    """(sum of sequence distances, number of grid-adjacent pairs, largest distance) of index map `kind`
+    over a T x H x W grid, computed on the GPU (see mate_scan_locality)."""
+    out = torch.zeros(3, dtype=torch.int64, device="cuda")
+    _lib.check(_lib.load().mate_scan_locality(int(T), int(H), int(W), int(kind), _p(out), _s(stream)),
+               "mate_scan_locality")
+    s, n, m = (int(v) for v in out.cpu().tolist())
+    return s, n, m

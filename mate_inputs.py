@@ -105,12 +105,6 @@ TEST_CONFIGS: Dict[str, MateConfig] = {
                                   (4, 8, 8), "bf16", 13),
     "f32_b2_4x8x12": _cfg("f32_b2_4x8x12", 2, 4, 8, 12, 64, 2, 32, 16, 64, 32, 2, 32, (2, 4, 4), "f32", 14,
                           shift=(1, 2, 2)),
-    # edge cases: a grid that is exactly one scan chunk and one attention window (its shifted layers mask
-    # every region pair inside the single window), and a batch of two without review tokens
-    "bf16_onechunk_4x8x8": _cfg("bf16_onechunk_4x8x8", 1, 4, 8, 8, 512, 8, 64, 128, 256, 16, 4, 128, (4, 8, 8),
-                                "bf16", 15),
-    "bf16_noreview_b2_8x16x16": _cfg("bf16_noreview_b2_8x16x16", 2, 8, 16, 16, 512, 8, 64, 128, 256, 0, 4, 128,
-                                     (4, 8, 8), "bf16", 16),
 }
 
 

@@ -113,7 +113,18 @@ def test_noalloc_scan_rejects_problems_beyond_its_scratch(lib):
 
 
 def test_kernel_names_are_distinct(lib):
-    names = [lib.mate_kernel_name(k).decode() for k in range(15)]
-    assert len(set(names)) == 15 and "unknown" not in names, names
+    names = [lib.mate_kernel_name(k).decode() for k in range(16)]
+    assert len(set(names)) == 16 and "unknown" not in names, names
     assert lib.mate_kernel_name(99).decode() == "unknown"
     assert lib.mate_trace_start(-1) == _lib.MATE_ERR_ARG
+
+
+def test_scan_locality_argument_checks(lib):
+    """Rejected before any device work: bad map, null or misaligned output, Hilbert on a grid it does not tile."""
+    assert lib.mate_scan_locality(4, 8, 8, 7, 64, None) == _lib.MATE_ERR_ARG
+    assert lib.mate_scan_locality(4, 8, 8, 0, None, None) == _lib.MATE_ERR_ARG
+    assert lib.mate_scan_locality(4, 8, 8, 0, 68, None) == _lib.MATE_ERR_ARG
+    assert lib.mate_scan_locality(0, 8, 8, 0, 64, None) == _lib.MATE_ERR_ARG
+    assert lib.mate_scan_locality(64, 48, 48, 5, 64, None) == _lib.MATE_ERR_UNSUPPORTED   # 48 is not a power of two
+    assert lib.mate_scan_locality(12, 8, 8, 5, 64, None) == _lib.MATE_ERR_UNSUPPORTED     # 8 does not divide 12
+    assert lib.mate_scan_locality(8, 8, 4, 5, 64, None) == _lib.MATE_ERR_UNSUPPORTED      # H != W

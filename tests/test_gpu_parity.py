@@ -7,6 +7,7 @@ import pytest
 from helpers import assert_close, assert_close_elementwise, oracle_cached, requires_gpu
 from bf16_floor import bf16_storage_forward, elementwise_err, rms_normalised_max_err, ssd_bf16_storage_emulation
 import mate_inputs as mi
+from edge_configs import all_test_configs
 from oracle import mate_oracle as O
 
 pytestmark = [pytest.mark.gpu, requires_gpu]
@@ -39,7 +40,7 @@ SMALL = ["tiny_f32_4x8x8", "f32_b2_4x8x12", "bf16_small_8x16x16", "bf16_ragged_1
 
 @pytest.mark.parametrize("name", SMALL + ["bf16_16x32x32", "bf16_256x32x32", "bf16_2x64x48x48_d2048"])
 def test_rms_permute_unpermute_bitexact(name):
-    cfg = mi.all_configs()[name]
+    cfg = all_test_configs()[name]
     X = mi.make_x_only(cfg, 100)
     Xd = dev(X, tdt(cfg))
     for order in range(4):
@@ -57,7 +58,7 @@ def test_rms_permute_unpermute_bitexact(name):
 
 @pytest.mark.parametrize("name", SMALL + ["bf16_256x32x32"])
 def test_review_pool(name):
-    cfg = mi.all_configs()[name]
+    cfg = all_test_configs()[name]
     X = mi.make_x_only(cfg, 101)
     Xd = dev(X, tdt(cfg))
     for order in range(4):
@@ -113,7 +114,7 @@ def _ssd_oracle(cfg, x, Bm, Cm, dt, dt_bias, A_log, D, heads=None):
 @pytest.mark.parametrize("long_memory", [False, True])
 @pytest.mark.parametrize("name", SMALL)
 def test_ssd_scan_bidir(name, long_memory):
-    cfg = mi.all_configs()[name]
+    cfg = all_test_configs()[name]
     args = _ssd_inputs(cfg, long_memory, 7)
     x, Bm, Cm, dt, dt_bias, A_log, D = args
     td = tdt(cfg)
@@ -156,7 +157,7 @@ def _tesa_inputs(cfg, seed):
 @pytest.mark.parametrize("shifted", [False, True])
 @pytest.mark.parametrize("name", SMALL + ["bf16_16x32x32"])
 def test_tesa_forward(name, shifted):
-    cfg = mi.all_configs()[name]
+    cfg = all_test_configs()[name]
     qkv = _tesa_inputs(cfg, 8)
     got = host(M.tesa_forward(dev(qkv, tdt(cfg)), shifted, cfg))
     ref = oracle_cached(f"tesa-{name}-{shifted}", lambda: np.stack([
@@ -206,7 +207,7 @@ def _check_block(cfg, w, layer, variant, out):
 @pytest.mark.parametrize("layer", [0, 1, 2, 3])
 @pytest.mark.parametrize("name", SMALL + ["bf16_16x32x32"])
 def test_mate_forward(name, layer, variant):
-    cfg = mi.all_configs()[name]
+    cfg = all_test_configs()[name]
     w = _block(cfg, variant)
     blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
     out = host(blk.forward(dev(w["X"], tdt(cfg)), layer))
@@ -219,7 +220,7 @@ def test_mate_forward(name, layer, variant):
 def test_mate_forward_single_branch(name, branch, layer):
     """Each branch alone (the other branch's output projection zeroed).  The TE branch's output is not
     heavy-tailed, so its bf16-storage floor stays below 2e-2 and the strict bound applies."""
-    cfg = mi.all_configs()[name]
+    cfg = all_test_configs()[name]
     w = dict(_block(cfg, "default"))
     zero = "W_out" if branch == "te" else "W_o"
     w[zero] = np.zeros_like(w[zero])
@@ -277,3 +278,20 @@ def test_ssd_full_size_sampled_head():
     key = "ssd-full-bf16_256x32x32-h5-every16"
     ref = oracle_cached(key, lambda: _ssd_oracle(cfg, *args, heads=[5])[:, rows])
     assert_close_elementwise(got, ref, "bf16", "ssd full size head 5", _ssd_floor(cfg, args, ref, key, [5], rows))
+
+
+# ------------------------------------------------------------------ scan locality
+
+from oracle import scan_locality as SL  # noqa: E402
+
+
+@pytest.mark.parametrize("grid", [(4, 8, 8), (12, 16, 24), (16, 32, 32), (256, 32, 32), (64, 48, 48)])
+@pytest.mark.parametrize("kind", range(7))
+def test_scan_locality_exact(grid, kind):
+    """Integer sums over all grid-adjacent pairs: bit-exact against the oracle, up to the workload grids."""
+    T, H, W = grid
+    if kind == 5 and (H != W or H & (H - 1) or T % H):
+        pytest.skip("Hilbert map needs H = W a power of two dividing T")
+    got = M.scan_locality(T, H, W, kind)
+    ref = SL.scan_locality(T, H, W, kind)   # exact integers (not through the float cache)
+    assert got == ref, (grid, kind, got, ref)
