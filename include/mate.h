@@ -266,7 +266,8 @@ typedef enum {
   MATE_K_OUT_PROJ = 12,        /* fused out-projection [y | O] [W_out | W_o]^T (the branch sum) */
   MATE_K_RMS_GATHER = 13,
   MATE_K_PROJECT = 14,         /* mate_project_bf16 */
-  MATE_K_SCAN_LOCALITY = 15    /* mate_scan_locality */
+  MATE_K_SCAN_LOCALITY = 15,   /* mate_scan_locality */
+  MATE_K_Y_TO_GRID = 16        /* scan-order y rows back to grid order (time-fastest scan orders) */
 } mate_kernel;
 
 typedef struct {

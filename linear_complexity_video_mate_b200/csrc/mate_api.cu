@@ -196,7 +196,7 @@ SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh) {
 
 struct ForwardPlan {
   int NIn, NI, KO;
-  void *Wi, *Wo, *Rv, *Zv, *Zr, *YO;
+  void *Wi, *Wo, *Rv, *Zv, *Zr, *YO, *Ys;
   float *Dv, *Dr;
   SsdScratch ssd;
   size_t bytes;
@@ -218,6 +218,8 @@ ForwardPlan plan_forward(const mate_config* c, void* ws) {
   p.Dv = cv.take<float>((size_t)c->B * n * c->nh);
   p.Dr = cv.take<float>((size_t)c->B * c->R * c->nh);
   p.YO = cv.take<char>((size_t)c->B * n * p.KO * es);
+  // y in scan order, for the time-fastest orders (their grid-order y rows are 1024s of rows apart)
+  p.Ys = c->dtype == MATE_BF16 ? cv.take<char>((size_t)c->B * n * c->nh * c->P * es) : nullptr;
   if (c->dtype == MATE_BF16) p.ssd = carve_ssd(cv, c->B, n, c->R, c->nh);
   else p.ssd = SsdScratch{};
   p.bytes = cv.off + 256;
@@ -498,7 +500,24 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   rows.H = c->H;
   rows.W = c->W;
   rows.order = order;
-  MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.YO, KO, n, pl.ssd, st));
+  // Orders 2 and 3 run time fastest: grid-order rows of one chunk lie in 256 different time planes, and
+  // writing each head's 128-byte y piece there costs more than writing y in scan order and moving whole
+  // rows back to grid order afterwards (measured on the B200).
+  const bool y_in_scan_order = c->dtype == MATE_BF16 && order >= 2;
+  rows.y_order = y_in_scan_order ? -1 : order;
+  if (y_in_scan_order) {
+    MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.Ys, dI, n, pl.ssd, st));
+    const int vec = static_cast<int>(dI * es / 16);
+    const long long total = (long long)c->B * n;
+    const int blocks = static_cast<int>(std::min<long long>((total + 7) / 8, (long long)device_sms() * 16));
+    trace_begin(MATE_K_Y_TO_GRID, st);
+    scan_rows_to_grid_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(pl.Ys), vec,
+                                                    static_cast<uint4*>(pl.YO), static_cast<long long>(KO * es / 16),
+                                                    vec, total, static_cast<int>(n), c->T, c->H, c->W, order);
+    MATE_LAUNCH_CHECK();
+  } else {
+    MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.YO, KO, n, pl.ssd, st));
+  }
   // TE: window attention on the q | k | v columns of Zv, output into YO[:, dI:]
   const int qc = NIn, ac = c->th * c->tp;
   MATE_TRY(run_tesa(c, pl.Zv, NI, qc, qc + ac, qc + 2 * ac, pl.YO, KO, dI, shifted, st));
@@ -608,6 +627,7 @@ mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const 
   rows.H = cfg->H;
   rows.W = cfg->W;
   rows.order = -1;
+  rows.y_order = -1;
   return run_ssd(cfg, rows, A_log, D, y, cfg->nh * cfg->P, n, sc, st);
 }
 
@@ -789,6 +809,7 @@ const char* mate_kernel_name(int kernel) {
     case MATE_K_RMS_GATHER: return "rms_gather";
     case MATE_K_PROJECT: return "project";
     case MATE_K_SCAN_LOCALITY: return "scan_locality";
+    case MATE_K_Y_TO_GRID: return "y_to_grid";
   }
   return "unknown";
 }

@@ -28,6 +28,23 @@ __global__ void rms_gather_rows_kernel(const uint4* __restrict__ src, uint4* __r
   }
 }
 
+// Rows stored in scan order (src, row stride ld_src vectors) back to grid order (dst, row stride ld_dst
+// vectors): dst row b*n + r = src row b*n + raster_to_scan(r).  One warp per row, 16-byte vectors.
+__global__ void scan_rows_to_grid_kernel(const uint4* __restrict__ src, long long ld_src, uint4* __restrict__ dst,
+                                         long long ld_dst, int vec_per_row, long long total_rows, int n, int T, int H,
+                                         int W, int order) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < total_rows;
+       row += warps) {
+    const long long b = row / n;
+    const int r = static_cast<int>(row - b * n);
+    const uint4* s = src + (b * n + raster_to_scan(r, T, H, W, order)) * ld_src;
+    uint4* d = dst + row * ld_dst;
+    for (int v = lane; v < vec_per_row; v += 32) d[v] = __ldg(s + v);
+  }
+}
+
 // ---------------------------------------------------------------------------------------------------
 // Review tokens: block mean of X over each cell of the Tr x 4 x 4 pooling grid, written in scan order
 // of that grid.  One CTA per review token; each thread owns one 16-byte vector of channels.
@@ -144,11 +161,16 @@ struct SeqRows {
   int ldxv, ldbv, ldcv, lddv;
   int ldxr, ldbr, ldcr, lddr;
   long long v_bstride, v_off, r_bstride, r_off;
-  int n, R, T, H, W, order;
+  int n, R, T, H, W;
+  int order;     // scan order of the video input rows (row of scan position q: scan_to_raster(q)); -1: identity
+  int y_order;   // scan order of the output rows (y of scan position q goes to row map(q)); -1: identity
   __host__ __device__ __forceinline__ int map(int q) const {
+    return y_order < 0 ? q : scan_to_raster(q, T, H, W, y_order);
+  }
+  __host__ __device__ __forceinline__ int in_map(int q) const {
     return order < 0 ? q : scan_to_raster(q, T, H, W, order);
   }
-  __host__ __device__ __forceinline__ long long vrow(int b, int q) const { return b * v_bstride + v_off + map(q); }
+  __host__ __device__ __forceinline__ long long vrow(int b, int q) const { return b * v_bstride + v_off + in_map(q); }
   __host__ __device__ __forceinline__ long long rrow(int b, int i) const { return b * r_bstride + r_off + i; }
 };
 

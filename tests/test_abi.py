@@ -113,8 +113,8 @@ def test_noalloc_scan_rejects_problems_beyond_its_scratch(lib):
 
 
 def test_kernel_names_are_distinct(lib):
-    names = [lib.mate_kernel_name(k).decode() for k in range(16)]
-    assert len(set(names)) == 16 and "unknown" not in names, names
+    names = [lib.mate_kernel_name(k).decode() for k in range(17)]
+    assert len(set(names)) == 17 and "unknown" not in names, names
     assert lib.mate_kernel_name(99).decode() == "unknown"
     assert lib.mate_trace_start(-1) == _lib.MATE_ERR_ARG
 
