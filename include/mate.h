@@ -220,9 +220,13 @@ MATE_API mate_status mate_forward(const void* X, const mate_weights* w, int laye
 
 /*
  * mate_forward with HOST input and output: copies X_host (B*T*H*W*d elements) to the device part of
- * the workspace, runs the block and copies Out back to Out_host, all on `stream` (page-locked host
- * buffers give full-speed asynchronous copies).  The host buffers must stay valid until the stream
- * reaches the end of the call.  ws: at least mate_workspace_bytes(cfg) + 2 * B*T*H*W*d*elem bytes.
+ * the workspace, runs the block and copies Out back to Out_host (page-locked host buffers give
+ * full-speed asynchronous copies).  For bf16 blocks the copies go in four row chunks on two copy streams
+ * of the library's own (one pair per device, created on the first call): the in-projection of a chunk
+ * starts as soon as it has landed, and each chunk of Out leaves as soon as its out-projection is done.
+ * The copies start after all earlier work on `stream`, and the call ends on `stream` only when the last
+ * chunk has reached Out_host.  The host buffers must stay valid until the stream reaches the end of the
+ * call.  ws: at least mate_workspace_bytes(cfg) + 2 * B*T*H*W*d*elem bytes.
  */
 MATE_API mate_status mate_forward_host(const void* X_host, const mate_weights* w, int layer_idx, void* Out_host,
                               const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream);

@@ -437,8 +437,62 @@ mate_status run_tesa(const mate_config* c, const void* qkv, int ldq, int qcol, i
   return MATE_OK;
 }
 
+// Host input and output of mate_forward_host, moved in row chunks on two copy streams so that the
+// host-to-device copy overlaps the in-projection of the chunks already landed and the device-to-host copy
+// overlaps the out-projection of the later chunks.  One set per device; the mutex keeps one call's
+// sequence of event records and waits together.
+constexpr int kIoChunks = 4;
+struct HostIo {
+  std::mutex mu;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr, in_ready[kIoChunks] = {}, out_ready[kIoChunks] = {};
+  bool ready = false, failed = false;
+};
+HostIo g_io[kMaxDevices];
+
+HostIo* host_io() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  HostIo& io = g_io[dev];
+  std::lock_guard<std::mutex> lock(io.mu);
+  if (!io.ready && !io.failed) {
+    bool ok = cudaStreamCreateWithFlags(&io.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&io.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&io.start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&io.done, cudaEventDisableTiming) == cudaSuccess;
+    for (int k = 0; ok && k < kIoChunks; ++k)
+      ok = cudaEventCreateWithFlags(&io.in_ready[k], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&io.out_ready[k], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      io.failed = true;
+    } else {
+      io.ready = true;
+    }
+  }
+  return io.ready ? &io : nullptr;
+}
+
+// The chunked host transfers of one mate_forward_host call (null for device-buffer calls).
+struct IoPlan {
+  HostIo* io;
+  const char* x_host;
+  char* out_host;
+  long long rows, chunk_rows;   // chunk c covers rows [c * chunk_rows, min(rows, (c + 1) * chunk_rows))
+  size_t row_bytes;
+};
+
+bool cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return true;
+  cudaGetLastError();
+  return false;
+}
+
 mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, void* Out, const mate_config* c,
-                         void* ws, size_t ws_bytes, cudaStream_t st) {
+                         void* ws, size_t ws_bytes, cudaStream_t st, const IoPlan* iop = nullptr) {
   MATE_TRY(check_config(c));
   if (X == nullptr || w == nullptr || Out == nullptr || ws == nullptr || layer_idx < 0) return MATE_ERR_ARG;
   if (w->W_in == nullptr || w->dt_bias == nullptr || w->A_log == nullptr || w->D == nullptr || w->W_out == nullptr ||
@@ -465,11 +519,24 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   MATE_TRY(copy_block(w->W_out, pl.Wo, c->d, dI, KO, 0, 0, es, st));
   MATE_TRY(copy_block(w->W_o, pl.Wo, c->d, c->th * c->tp, KO, 0, dI, es, st));
   // review tokens, then the projections of the video rows (grid order) and of the review rows
-  MATE_TRY(pool(X, pl.Rv, c, order, st));
-  if (c->dtype == MATE_BF16) {
+  if (c->dtype == MATE_BF16 && iop != nullptr) {
+    // host input: project each row chunk as soon as it has landed; the review pool needs all of X
+    for (int k = 0; k < kIoChunks; ++k) {
+      const long long r0 = k * iop->chunk_rows, r1 = std::min(iop->rows, r0 + iop->chunk_rows);
+      if (!cuda_ok(cudaStreamWaitEvent(st, iop->io->in_ready[k], 0))) return MATE_ERR_CUDA;
+      if (r1 <= r0) continue;
+      MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, static_cast<const char*>(X) + r0 * c->d * es, c->d, r1 - r0, c->d, pl.Wi,
+                         c->d, NI, static_cast<char*>(pl.Zv) + r0 * NI * es, NI, pl.Dv + r0 * c->nh, c->nh, dt0,
+                         c->nh, w->dt_bias, st));
+    }
+    MATE_TRY(pool(X, pl.Rv, c, order, st));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
+  } else if (c->dtype == MATE_BF16) {
+    MATE_TRY(pool(X, pl.Rv, c, order, st));
     MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, X, c->d, Mv, c->d, pl.Wi, c->d, NI, pl.Zv, NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
     MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
   } else {
+    MATE_TRY(pool(X, pl.Rv, c, order, st));
     MATE_TRY(gemm_f32(MATE_K_IN_PROJ, static_cast<const float*>(X), c->d, Mv, c->d, static_cast<const float*>(pl.Wi), c->d, NI,
                       static_cast<float*>(pl.Zv), NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
     MATE_TRY(gemm_f32(MATE_K_IN_PROJ_REVIEW, static_cast<const float*>(pl.Rv), c->d, Mr, c->d, static_cast<const float*>(pl.Wi), c->d, NIn,
@@ -522,7 +589,22 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   const int qc = NIn, ac = c->th * c->tp;
   MATE_TRY(run_tesa(c, pl.Zv, NI, qc, qc + ac, qc + 2 * ac, pl.YO, KO, dI, shifted, st));
   // Out = [y | O] [W_out | W_o]^T = MA + TE
-  if (c->dtype == MATE_BF16)
+  if (c->dtype == MATE_BF16 && iop != nullptr) {
+    // host output: each row chunk goes back to the host while the later chunks are projected
+    for (int k = 0; k < kIoChunks; ++k) {
+      const long long r0 = k * iop->chunk_rows, r1 = std::min(iop->rows, r0 + iop->chunk_rows);
+      if (r1 > r0)
+        MATE_TRY(gemm_bf16(MATE_K_OUT_PROJ, static_cast<const char*>(pl.YO) + r0 * KO * es, KO, r1 - r0, KO, pl.Wo,
+                           KO, c->d, static_cast<char*>(Out) + r0 * c->d * es, c->d, nullptr, 0, 0, 0, nullptr, st));
+      if (!cuda_ok(cudaEventRecord(iop->io->out_ready[k], st)) ||
+          !cuda_ok(cudaStreamWaitEvent(iop->io->d2h, iop->io->out_ready[k], 0)))
+        return MATE_ERR_CUDA;
+      if (r1 > r0 && !cuda_ok(cudaMemcpyAsync(iop->out_host + r0 * iop->row_bytes,
+                                              static_cast<const char*>(Out) + r0 * iop->row_bytes,
+                                              (r1 - r0) * iop->row_bytes, cudaMemcpyDeviceToHost, iop->io->d2h)))
+        return MATE_ERR_CUDA;
+    }
+  } else if (c->dtype == MATE_BF16)
     MATE_TRY(gemm_bf16(MATE_K_OUT_PROJ, pl.YO, KO, Mv, KO, pl.Wo, KO, c->d, Out, c->d, nullptr, 0, 0, 0, nullptr, st));
   else
     MATE_TRY(gemm_f32(MATE_K_OUT_PROJ, static_cast<const float*>(pl.YO), KO, Mv, KO, static_cast<const float*>(pl.Wo), KO, c->d,
@@ -729,9 +811,36 @@ mate_status mate_forward_host(const void* X_host, const mate_weights* w, int lay
   char* xdev = static_cast<char*>(ws) + ((fw + 255) & ~size_t(255));
   char* odev = xdev + ((xb + 255) & ~size_t(255));
   t_launches = 0;
-  if (cudaMemcpyAsync(xdev, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MATE_ERR_CUDA;
-  MATE_TRY(forward_impl(xdev, w, layer_idx, odev, cfg, ws, fw, st));
-  if (cudaMemcpyAsync(Out_host, odev, xb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MATE_ERR_CUDA;
+  HostIo* io = cfg->dtype == MATE_BF16 ? host_io() : nullptr;
+  if (io == nullptr) {   // one copy each way on `stream`
+    if (cudaMemcpyAsync(xdev, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MATE_ERR_CUDA;
+    MATE_TRY(forward_impl(xdev, w, layer_idx, odev, cfg, ws, fw, st));
+    if (cudaMemcpyAsync(Out_host, odev, xb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MATE_ERR_CUDA;
+    return MATE_OK;
+  }
+  std::lock_guard<std::mutex> lock(io->mu);
+  IoPlan iop;
+  iop.io = io;
+  iop.x_host = static_cast<const char*>(X_host);
+  iop.out_host = static_cast<char*>(Out_host);
+  iop.rows = (long long)cfg->B * cfg->T * cfg->H * cfg->W;
+  iop.row_bytes = (size_t)cfg->d * elem_size(cfg);
+  iop.chunk_rows = ((iop.rows + kIoChunks - 1) / kIoChunks + 255) / 256 * 256;
+  // both copy streams start after all earlier work on `stream` (the workspace may still be in use)
+  if (!cuda_ok(cudaEventRecord(io->start, st)) || !cuda_ok(cudaStreamWaitEvent(io->h2d, io->start, 0)) ||
+      !cuda_ok(cudaStreamWaitEvent(io->d2h, io->start, 0)))
+    return MATE_ERR_CUDA;
+  for (int k = 0; k < kIoChunks; ++k) {
+    const long long r0 = k * iop.chunk_rows, r1 = std::min(iop.rows, r0 + iop.chunk_rows);
+    if (r1 > r0 && !cuda_ok(cudaMemcpyAsync(xdev + r0 * iop.row_bytes, iop.x_host + r0 * iop.row_bytes,
+                                            (r1 - r0) * iop.row_bytes, cudaMemcpyHostToDevice, io->h2d)))
+      return MATE_ERR_CUDA;
+    if (!cuda_ok(cudaEventRecord(io->in_ready[k], io->h2d))) return MATE_ERR_CUDA;
+  }
+  MATE_TRY(forward_impl(xdev, w, layer_idx, odev, cfg, ws, fw, st, &iop));
+  // the call ends on `stream` only when the last chunk has reached the host
+  if (!cuda_ok(cudaEventRecord(io->done, io->d2h)) || !cuda_ok(cudaStreamWaitEvent(st, io->done, 0)))
+    return MATE_ERR_CUDA;
   return MATE_OK;
 }
 
