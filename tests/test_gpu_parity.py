@@ -260,15 +260,19 @@ def test_mate_forward_single_branch(name, branch, layer):
     _check_block(cfg, w, layer, f"{branch}only", out)
 
 
-def test_mate_forward_host_matches_device_path():
-    cfg = mi.TEST_CONFIGS["bf16_small_8x16x16"]
+@pytest.mark.parametrize("name,layer", [("bf16_small_8x16x16", 3), ("bf16_b2_20x16x16_d512", 2),
+                                        ("bf16_onechunk_4x8x8", 1), ("bf16_noreview_b2_8x16x16", 0)])
+def test_mate_forward_host_matches_device_path(name, layer):
+    """Host buffers (row-chunked copies overlapped with the projections, including chunks that are empty or
+    cross a sample boundary) give the same bits as the device-buffer call."""
+    cfg = all_test_configs()[name]
     w = _block(cfg, "default")
     blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
     Xd = dev(w["X"], torch.bfloat16)
-    ref = blk.forward(Xd, 3)
+    ref = blk.forward(Xd, layer)
     xh = Xd.cpu().pin_memory()
     oh = torch.empty_like(xh).pin_memory()
-    blk.forward_host(xh, 3, oh)
+    blk.forward_host(xh, layer, oh)
     torch.cuda.synchronize()
     assert torch.equal(oh, ref.cpu())
 
