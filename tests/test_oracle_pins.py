@@ -421,3 +421,50 @@ def test_locality_against_brute_force(kind):
                 d = min(abs(int(p[a]) - int(p[b])) for p in pos)
                 total, n, largest = total + d, n + 1, max(largest, d)
     assert SL.scan_locality(T, H, W, kind) == (total, n, largest)
+
+
+# ------------------------------------------------------------------ per-direction scan parameters
+
+from oracle import per_direction as PD  # noqa: E402
+
+
+def _pd_case(seed=3, L=40, R=6, nh=2, P=3, N=4):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((L, nh, P))
+    Bm, Cm = rng.standard_normal((L, N)), rng.standard_normal((L, N))
+    delta_f = O.softplus(rng.standard_normal((L, nh)))
+    delta_b = O.softplus(rng.standard_normal((L, nh)) - 0.5)
+    A_f, A_b = -np.exp(rng.uniform(-1, 1, nh)), -np.exp(rng.uniform(-1, 1, nh))
+    D_f, D_b = rng.standard_normal(nh), rng.standard_normal(nh)
+    return x, Bm, Cm, delta_f, A_f, D_f, delta_b, A_b, D_b, R
+
+
+def test_per_direction_without_backward_is_the_forward_recurrence():
+    """Backward step sizes and skip zero: the backward scan adds nothing."""
+    x, Bm, Cm, df, Af, Df, db, Ab, Db, R = _pd_case()
+    y = PD.ssd_bidirectional_per_direction(x, Bm, Cm, df, Af, Df, np.zeros_like(db), Ab, np.zeros_like(Db), R)
+    np.testing.assert_allclose(y, O.ssd_recurrence(x, Bm, Cm, df, Af, Df)[R:], rtol=1e-13, atol=1e-13)
+
+
+def test_per_direction_without_forward_is_the_reversed_backward_recurrence():
+    x, Bm, Cm, df, Af, Df, db, Ab, Db, R = _pd_case()
+    y = PD.ssd_bidirectional_per_direction(x, Bm, Cm, np.zeros_like(df), Af, np.zeros_like(Df), db, Ab, Db, R)
+    flip = np.concatenate([np.arange(R), np.arange(x.shape[0] - 1, R - 1, -1)])
+    yb = O.ssd_recurrence(x[flip], Bm[flip], Cm[flip], db[flip], Ab, Db)[R:][::-1]
+    np.testing.assert_allclose(y, yb, rtol=1e-13, atol=1e-13)
+
+
+def test_per_direction_fast_decay_closed_form():
+    """Every decay underflows: y_t = (D_f + D_b + C_t . B_t (delta_f + delta_b)) x_t, written out directly."""
+    x, Bm, Cm, df, Af, Df, db, Ab, Db, R = _pd_case()
+    Af, Ab = np.full_like(Af, -1e4), np.full_like(Ab, -1e4)
+    y = PD.ssd_bidirectional_per_direction(x, Bm, Cm, df, Af, Df, db, Ab, Db, R)
+    cb = np.einsum("ln,ln->l", Cm, Bm)[R:]
+    want = (Df + Db + cb[:, None] * (df + db)[R:])[:, :, None] * x[R:]
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
+
+
+def test_per_direction_with_shared_parameters_is_the_shared_oracle():
+    x, Bm, Cm, df, Af, Df, db, Ab, Db, R = _pd_case()
+    np.testing.assert_allclose(PD.ssd_bidirectional_per_direction(x, Bm, Cm, df, Af, Df, df, Af, Df, R),
+                               O.ssd_bidirectional(x, Bm, Cm, df, Af, Df, R), rtol=0, atol=0)
