@@ -87,6 +87,11 @@ typedef struct {
   const void* W_out;    /* [d, nh*P]  MA out-projection                                              */
   const void* W_qkv;    /* [3*th*tp, d] output features q | k | v, head-major inside each            */
   const void* W_o;      /* [d, th*tp]  TE out-projection                                             */
+  /* Optional separate parameters of the backward scan direction (all three or none; null: the backward
+   * scan uses dt_bias, A_log and D above).  The pages do not say whether the directions share them. */
+  const float* dt_bias_b; /* [nh] */
+  const float* A_log_b;   /* [nh] */
+  const float* D_b;       /* [nh] */
 } mate_weights;
 
 /* Human-readable name of a status code (static string). */
@@ -100,6 +105,10 @@ MATE_API size_t mate_workspace_bytes(const mate_config* cfg);
 
 /* Workspace bytes needed by ssd_scan_bidir for this shape with `prefix_len` prefix rows. */
 MATE_API size_t mate_ssd_workspace_bytes(const mate_config* cfg, int prefix_len);
+
+/* Workspace bytes needed by ssd_scan_bidir_pd (separate backward-scan parameters): the backward step
+ * sizes, log-decays and review-chunk states come on top of what ssd_scan_bidir needs. */
+MATE_API size_t mate_ssd_pd_workspace_bytes(const mate_config* cfg, int prefix_len);
 
 /*
  * Rotary Major Scan reorder ([NEWS] RMS paragraphs; [FEAT] RMS modes).
@@ -139,6 +148,23 @@ MATE_API mate_status review_pool(const void* X, void* Rv, int order, const mate_
 MATE_API mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const float* dt, const float* dt_bias,
                            const float* A_log, const float* D, int prefix_len, void* y, const mate_config* cfg,
                            void* ws, size_t ws_bytes, mate_stream_t stream);
+
+/*
+ * ssd_scan_bidir with separate parameters for the backward scan direction ([ABS] "bidirectional Mamba2
+ * block"; the pages leave open whether the two directions share A, D and the step-size bias).  The
+ * forward scan uses dt_bias, A_log, D; the backward scan (over [prefix rows; video rows reversed]) uses
+ * delta_b = softplus(dt + dt_bias_b[h]), A_b = -exp(A_log_b[h]) and D_b, with the same x, Bm, Cm and raw
+ * dt.  y = y_forward + (y_backward reversed back), each direction including its own D x skip term.
+ * With dt_bias_b = dt_bias, A_log_b = A_log, D_b = D it computes what ssd_scan_bidir computes.
+ *   dt_bias_b, A_log_b, D_b  [nh] float, device; ws at least mate_ssd_pd_workspace_bytes(cfg, prefix_len)
+ *   bytes; every other argument as for ssd_scan_bidir.  MATE_ERR_ARG if any of the three is null;
+ *   otherwise the statuses of ssd_scan_bidir.
+ */
+MATE_API mate_status ssd_scan_bidir_pd(const void* x, const void* Bm, const void* Cm, const float* dt,
+                                       const float* dt_bias, const float* A_log, const float* D,
+                                       const float* dt_bias_b, const float* A_log_b, const float* D_b,
+                                       int prefix_len, void* y, const mate_config* cfg, void* ws, size_t ws_bytes,
+                                       mate_stream_t stream);
 
 /* Size of the fixed device scratch buffer behind ssd_scan_bidir_noalloc: 32 MiB. */
 #define MATE_SSD_NOALLOC_SCRATCH_BYTES (32u << 20)

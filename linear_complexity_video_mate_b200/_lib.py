@@ -16,7 +16,7 @@ EXPORTS = (
     "rms_unpermute", "review_pool", "ssd_scan_bidir", "tesa_forward", "mate_forward", "mate_forward_host",
     "mate_forward_host_workspace_bytes", "mate_device_status", "mate_last_launch_count", "mate_project_bf16",
     "ssd_scan_bidir_noalloc", "mate_trace_start", "mate_trace_stop", "mate_trace_read", "mate_kernel_name",
-    "mate_scan_locality",
+    "mate_scan_locality", "ssd_scan_bidir_pd", "mate_ssd_pd_workspace_bytes",
 )
 
 _CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp", "wt", "wh", "ww", "st", "sh", "sw")
@@ -29,7 +29,8 @@ class CConfig(ctypes.Structure):
 class CWeights(ctypes.Structure):
     _fields_ = [("W_in", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
                 ("D", ctypes.c_void_p), ("W_out", ctypes.c_void_p), ("W_qkv", ctypes.c_void_p),
-                ("W_o", ctypes.c_void_p)]
+                ("W_o", ctypes.c_void_p), ("dt_bias_b", ctypes.c_void_p), ("A_log_b", ctypes.c_void_p),
+                ("D_b", ctypes.c_void_p)]
 
 
 class CTraceRecord(ctypes.Structure):
@@ -60,11 +61,13 @@ def load():
         "mate_check_config": (ci, [cfgp]),
         "mate_workspace_bytes": (sz, [cfgp]),
         "mate_ssd_workspace_bytes": (sz, [cfgp, ci]),
+        "mate_ssd_pd_workspace_bytes": (sz, [cfgp, ci]),
         "rms_permute": (ci, [vp, vp, ci, cfgp, vp]),
         "rms_unpermute": (ci, [vp, vp, ci, cfgp, vp]),
         "review_pool": (ci, [vp, vp, ci, cfgp, vp]),
         "ssd_scan_bidir": (ci, [vp, vp, vp, vp, vp, vp, vp, ci, vp, cfgp, vp, sz, vp]),
         "ssd_scan_bidir_noalloc": (ci, [vp, vp, vp, vp, vp, vp, vp, ci, vp, cfgp, vp]),
+        "ssd_scan_bidir_pd": (ci, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, cfgp, vp, sz, vp]),
         "mate_trace_start": (ci, [ci]),
         "mate_trace_stop": (ci, []),
         "mate_trace_read": (ci, [ctypes.POINTER(CTraceRecord), ci]),

@@ -30,6 +30,7 @@ struct GemmParams {
   int ld_delta;
   int dt_col0, dt_cols;
   const float* dt_bias;
+  const float* dt_bias2;   // optional: a second side output softplus(acc + dt_bias2) at column offset dt_cols
 };
 
 constexpr int kGemmBM = 128;
@@ -183,8 +184,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int c = col0 + j - p.dt_col0;
-            if (c >= 0 && c < p.dt_cols && col0 + j < col_end)
+            if (c >= 0 && c < p.dt_cols && col0 + j < col_end) {
               p.delta[static_cast<size_t>(row) * p.ld_delta + c] = softplus_f(__uint_as_float(r[j]) + p.dt_bias[c]);
+              if (p.dt_bias2 != nullptr)
+                p.delta[static_cast<size_t>(row) * p.ld_delta + p.dt_cols + c] =
+                    softplus_f(__uint_as_float(r[j]) + p.dt_bias2[c]);
+            }
           }
         }
       }

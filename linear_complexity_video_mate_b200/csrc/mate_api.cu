@@ -172,13 +172,15 @@ struct Carver {
 
 struct SsdScratch {
   __nv_bfloat16 *Gm, *Sf, *Sb, *Hf, *Hb;
-  float *gl, *Gd, *tbl;
+  float *gl, *glb, *Gd, *tbl;
+  __nv_bfloat16* Srb;
   int* crow;
 };
 
 int ceil_div(long long a, int b) { return static_cast<int>((a + b - 1) / b); }
 
-SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh) {
+// per_dir: also the backward scan's own decays and review-chunk states (separate backward parameters)
+SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh, bool per_dir) {
   SsdScratch s;
   const int nRc = ceil_div(R, kSsdQ), nVc = ceil_div(n, kSsdQ);
   const size_t PN = (size_t)kSsdP * kSsdN;
@@ -188,6 +190,8 @@ SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh) {
   s.Hf = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
   s.Hb = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
   s.gl = cv.take<float>((size_t)B * (nRc + nVc) * nh);
+  s.glb = per_dir ? cv.take<float>((size_t)B * (nRc + nVc) * nh) : nullptr;
+  s.Srb = per_dir ? cv.take<__nv_bfloat16>((size_t)B * nRc * nh * PN) : nullptr;
   s.Gd = cv.take<float>((size_t)B * nVc * kSsdQ);
   s.tbl = cv.take<float>((size_t)B * nVc * nh * 2 * kOutTbl);
   s.crow = cv.take<int>((size_t)B * nVc * kSsdQ);
@@ -215,23 +219,23 @@ ForwardPlan plan_forward(const mate_config* c, void* ws) {
   p.Rv = cv.take<char>((size_t)c->B * c->R * c->d * es);
   p.Zv = cv.take<char>((size_t)c->B * n * p.NI * es);
   p.Zr = cv.take<char>((size_t)c->B * c->R * p.NI * es);
-  p.Dv = cv.take<float>((size_t)c->B * n * c->nh);
-  p.Dr = cv.take<float>((size_t)c->B * c->R * c->nh);
+  p.Dv = cv.take<float>((size_t)c->B * n * 2 * c->nh);      // [rows][nh forward | nh backward]
+  p.Dr = cv.take<float>((size_t)c->B * c->R * 2 * c->nh);
   p.YO = cv.take<char>((size_t)c->B * n * p.KO * es);
   // y in scan order, for the time-fastest orders (their grid-order y rows are 1024s of rows apart)
   p.Ys = c->dtype == MATE_BF16 ? cv.take<char>((size_t)c->B * n * c->nh * c->P * es) : nullptr;
-  if (c->dtype == MATE_BF16) p.ssd = carve_ssd(cv, c->B, n, c->R, c->nh);
+  if (c->dtype == MATE_BF16) p.ssd = carve_ssd(cv, c->B, n, c->R, c->nh, true);
   else p.ssd = SsdScratch{};
   p.bytes = cv.off + 256;
   return p;
 }
 
-size_t ssd_ws_bytes(const mate_config* c, int prefix_len, float** delta, SsdScratch* s, void* ws) {
+size_t ssd_ws_bytes(const mate_config* c, int prefix_len, bool per_dir, float** delta, SsdScratch* s, void* ws) {
   Carver cv{static_cast<char*>(ws)};
   const long long n = (long long)c->T * c->H * c->W;
-  float* d = cv.take<float>((size_t)c->B * (n + prefix_len) * c->nh);
+  float* d = cv.take<float>((size_t)c->B * (n + prefix_len) * (per_dir ? 2 : 1) * c->nh);
   if (delta) *delta = d;
-  SsdScratch sc = c->dtype == MATE_BF16 ? carve_ssd(cv, c->B, n, prefix_len, c->nh) : SsdScratch{};
+  SsdScratch sc = c->dtype == MATE_BF16 ? carve_ssd(cv, c->B, n, prefix_len, c->nh, per_dir) : SsdScratch{};
   if (s) *s = sc;
   return cv.off + 256;
 }
@@ -243,7 +247,7 @@ int choose_bn(int N) { return N >= 256 ? 256 : ((N + 15) / 16) * 16; }
 
 mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const void* Bw, int ldb, int N, void* C,
                       int ldc, float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias,
-                      cudaStream_t st) {
+                      cudaStream_t st, const float* dt_bias2 = nullptr) {
   if (M <= 0) return MATE_OK;
   if (K % kGemmBK) return MATE_ERR_UNSUPPORTED;
   GemmParams p;
@@ -259,6 +263,7 @@ mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const
   p.dt_col0 = dt_col0;
   p.dt_cols = dt_cols;
   p.dt_bias = dt_bias;
+  p.dt_bias2 = dt_bias2;
   // 256-row tiles computed by 2-CTA clusters (tcgen05 cta_group::2)
   p.num_tiles = ceil_div(M, 256) * p.num_n_tiles;
   const uint32_t psb = gemm_pair_stage_bytes(p.bn);
@@ -276,12 +281,12 @@ mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const
 
 mate_status gemm_f32(int kid, const float* A, int lda, long long M, int K, const float* Bw, int ldb, int N, float* C,
                      int ldc, float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias,
-                     cudaStream_t st) {
+                     cudaStream_t st, const float* dt_bias2 = nullptr) {
   if (M <= 0) return MATE_OK;
   dim3 grid(ceil_div(N, 64), ceil_div(M, 64));
   trace_begin(kid, st);
   gemm_f32_kernel<<<grid, 256, 0, st>>>(A, lda, Bw, ldb, C, ldc, static_cast<int>(M), N, K, delta, ld_delta, dt_col0,
-                                        dt_cols, dt_bias);
+                                        dt_cols, dt_bias, dt_bias2);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }
@@ -329,13 +334,14 @@ mate_status copy_block(const void* src, void* dst, int rows, int cols, int ld_ds
 
 // Scan over sequences described by `rows`; y row = b*y_bstride + map(q), ldy.  bf16 or fp32 path.
 mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_log, const float* Dp, void* y, int ldy,
-                    long long y_bstride, const SsdScratch& sc, cudaStream_t st) {
+                    long long y_bstride, const SsdScratch& sc, cudaStream_t st, const float* A_log_b = nullptr,
+                    const float* Dp_b = nullptr) {
   const long long n = (long long)c->T * c->H * c->W;
   if (c->dtype == MATE_F32) {
     const int threads = ((c->P * c->N) + 31) / 32 * 32;
     trace_begin(MATE_K_SSD_F32, st);
     ssd_f32_kernel<<<dim3(c->nh, c->B), threads, c->P * c->N * sizeof(float), st>>>(
-        rows, A_log, Dp, c->P, c->N, static_cast<float*>(y), ldy, y_bstride);
+        rows, A_log, Dp, A_log_b, Dp_b, c->P, c->N, static_cast<float*>(y), ldy, y_bstride);
     MATE_LAUNCH_CHECK();
     return MATE_OK;
   }
@@ -356,6 +362,10 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   p.Hb = sc.Hb;
   p.crow = sc.crow;
   p.tbl = sc.tbl;
+  p.A_log_b = A_log_b;
+  p.Dp_b = Dp_b;
+  p.glb = sc.glb;
+  p.Srb = sc.Srb;
   p.y = static_cast<__nv_bfloat16*>(y);
   p.ldy = ldy;
   p.y_bstride = y_bstride;
@@ -498,6 +508,10 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   if (w->W_in == nullptr || w->dt_bias == nullptr || w->A_log == nullptr || w->D == nullptr || w->W_out == nullptr ||
       w->W_qkv == nullptr || w->W_o == nullptr)
     return MATE_ERR_ARG;
+  // separate backward-scan parameters: all three or none
+  const int n_bwd = (w->dt_bias_b != nullptr) + (w->A_log_b != nullptr) + (w->D_b != nullptr);
+  if (n_bwd != 0 && n_bwd != 3) return MATE_ERR_ARG;
+  const bool per_dir = n_bwd == 3;
   if (!aligned16(X) || !aligned16(Out) || !aligned16(ws) || !aligned16(w->W_in) || !aligned16(w->W_out) ||
       !aligned16(w->W_qkv) || !aligned16(w->W_o))
     return MATE_ERR_ARG;
@@ -512,6 +526,8 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   const int dI = c->nh * c->P;
   const int NIn = pl.NIn, NI = pl.NI, KO = pl.KO;
   const int dt0 = dI + 2 * c->N;
+  const int ldd = per_dir ? 2 * c->nh : c->nh;                     // delta rows: forward | backward
+  const float* dtb2 = per_dir ? w->dt_bias_b : nullptr;
 
   // packed weights: Wi = [W_in; W_qkv] (NI x d), Wo = [W_out | W_o] (d x KO)
   MATE_TRY(copy_block(w->W_in, pl.Wi, NIn, c->d, c->d, 0, 0, es, st));
@@ -526,21 +542,21 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
       if (!cuda_ok(cudaStreamWaitEvent(st, iop->io->in_ready[k], 0))) return MATE_ERR_CUDA;
       if (r1 <= r0) continue;
       MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, static_cast<const char*>(X) + r0 * c->d * es, c->d, r1 - r0, c->d, pl.Wi,
-                         c->d, NI, static_cast<char*>(pl.Zv) + r0 * NI * es, NI, pl.Dv + r0 * c->nh, c->nh, dt0,
-                         c->nh, w->dt_bias, st));
+                         c->d, NI, static_cast<char*>(pl.Zv) + r0 * NI * es, NI, pl.Dv + r0 * ldd, ldd, dt0,
+                         c->nh, w->dt_bias, st, dtb2));
     }
     MATE_TRY(pool(X, pl.Rv, c, order, st));
-    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
   } else if (c->dtype == MATE_BF16) {
     MATE_TRY(pool(X, pl.Rv, c, order, st));
-    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, X, c->d, Mv, c->d, pl.Wi, c->d, NI, pl.Zv, NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
-    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, X, c->d, Mv, c->d, pl.Wi, c->d, NI, pl.Zv, NI, pl.Dv, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
   } else {
     MATE_TRY(pool(X, pl.Rv, c, order, st));
     MATE_TRY(gemm_f32(MATE_K_IN_PROJ, static_cast<const float*>(X), c->d, Mv, c->d, static_cast<const float*>(pl.Wi), c->d, NI,
-                      static_cast<float*>(pl.Zv), NI, pl.Dv, c->nh, dt0, c->nh, w->dt_bias, st));
+                      static_cast<float*>(pl.Zv), NI, pl.Dv, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
     MATE_TRY(gemm_f32(MATE_K_IN_PROJ_REVIEW, static_cast<const float*>(pl.Rv), c->d, Mr, c->d, static_cast<const float*>(pl.Wi), c->d, NIn,
-                      static_cast<float*>(pl.Zr), NI, pl.Dr, c->nh, dt0, c->nh, w->dt_bias, st));
+                      static_cast<float*>(pl.Zr), NI, pl.Dr, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
   }
   // MA: scan over [review rows; video rows in scan order], y written at grid-order rows of YO[:, :dI]
   SeqRows rows;
@@ -556,7 +572,8 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   rows.dr = pl.Dr;
   rows.ldxv = rows.ldbv = rows.ldcv = NI;
   rows.ldxr = rows.ldbr = rows.ldcr = NI;
-  rows.lddv = rows.lddr = c->nh;
+  rows.lddv = rows.lddr = ldd;
+  rows.db_off = per_dir ? c->nh : 0;
   rows.v_bstride = n;
   rows.v_off = 0;
   rows.r_bstride = c->R;
@@ -573,7 +590,7 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   const bool y_in_scan_order = c->dtype == MATE_BF16 && order >= 2;
   rows.y_order = y_in_scan_order ? -1 : order;
   if (y_in_scan_order) {
-    MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.Ys, dI, n, pl.ssd, st));
+    MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.Ys, dI, n, pl.ssd, st, w->A_log_b, w->D_b));
     const int vec = static_cast<int>(dI * es / 16);
     const long long total = (long long)c->B * n;
     const int blocks = static_cast<int>(std::min<long long>((total + 7) / 8, (long long)device_sms() * 16));
@@ -583,7 +600,7 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
                                                     vec, total, static_cast<int>(n), c->T, c->H, c->W, order);
     MATE_LAUNCH_CHECK();
   } else {
-    MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.YO, KO, n, pl.ssd, st));
+    MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.YO, KO, n, pl.ssd, st, w->A_log_b, w->D_b));
   }
   // TE: window attention on the q | k | v columns of Zv, output into YO[:, dI:]
   const int qc = NIn, ac = c->th * c->tp;
@@ -639,7 +656,12 @@ size_t mate_workspace_bytes(const mate_config* cfg) {
 
 size_t mate_ssd_workspace_bytes(const mate_config* cfg, int prefix_len) {
   if (check_config(cfg) != MATE_OK || prefix_len < 0) return 0;
-  return ssd_ws_bytes(cfg, prefix_len, nullptr, nullptr, nullptr);
+  return ssd_ws_bytes(cfg, prefix_len, false, nullptr, nullptr, nullptr);
+}
+
+size_t mate_ssd_pd_workspace_bytes(const mate_config* cfg, int prefix_len) {
+  if (check_config(cfg) != MATE_OK || prefix_len < 0) return 0;
+  return ssd_ws_bytes(cfg, prefix_len, true, nullptr, nullptr, nullptr);
 }
 
 size_t mate_forward_host_workspace_bytes(const mate_config* cfg) {
@@ -670,26 +692,30 @@ mate_status review_pool(const void* X, void* Rv, int order, const mate_config* c
   return pool(X, Rv, cfg, order, reinterpret_cast<cudaStream_t>(stream));
 }
 
-mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const float* dt, const float* dt_bias,
-                           const float* A_log, const float* D, int prefix_len, void* y, const mate_config* cfg,
-                           void* ws, size_t ws_bytes, mate_stream_t stream) {
+mate_status scan_impl(const void* x, const void* Bm, const void* Cm, const float* dt, const float* dt_bias,
+                      const float* A_log, const float* D, const float* dt_bias_b, const float* A_log_b,
+                      const float* D_b, int prefix_len, void* y, const mate_config* cfg, void* ws, size_t ws_bytes,
+                      mate_stream_t stream) {
   MATE_TRY(check_config(cfg));
   if (x == nullptr || Bm == nullptr || Cm == nullptr || dt == nullptr || dt_bias == nullptr || A_log == nullptr ||
       D == nullptr || y == nullptr || ws == nullptr || prefix_len < 0)
     return MATE_ERR_ARG;
   if (!aligned16(x) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(y) || !aligned16(ws)) return MATE_ERR_ARG;
-  if (ws_bytes < ssd_ws_bytes(cfg, prefix_len, nullptr, nullptr, nullptr)) return MATE_ERR_WORKSPACE;
+  const int n_bwd = (dt_bias_b != nullptr) + (A_log_b != nullptr) + (D_b != nullptr);
+  if (n_bwd != 0 && n_bwd != 3) return MATE_ERR_ARG;
+  const bool per_dir = n_bwd == 3;
+  if (ws_bytes < ssd_ws_bytes(cfg, prefix_len, per_dir, nullptr, nullptr, nullptr)) return MATE_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   t_launches = 0;
   float* delta = nullptr;
   SsdScratch sc;
-  ssd_ws_bytes(cfg, prefix_len, &delta, &sc, ws);
+  ssd_ws_bytes(cfg, prefix_len, per_dir, &delta, &sc, ws);
   const long long n = (long long)cfg->T * cfg->H * cfg->W;
   const long long L = n + prefix_len;
   const long long total = (long long)cfg->B * L * cfg->nh;
   trace_begin(MATE_K_SOFTPLUS, st);
-  softplus_kernel<<<static_cast<int>(std::min<long long>((total + 255) / 256, 4096)), 256, 0, st>>>(dt, dt_bias, delta,
-                                                                                                   total, cfg->nh);
+  softplus_kernel<<<static_cast<int>(std::min<long long>((total + 255) / 256, 4096)), 256, 0, st>>>(
+      dt, dt_bias, per_dir ? dt_bias_b : nullptr, delta, total, cfg->nh);
   MATE_LAUNCH_CHECK();
   SeqRows rows;
   rows.xv = rows.xr = x;
@@ -698,7 +724,8 @@ mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const 
   rows.dv = rows.dr = delta;
   rows.ldxv = rows.ldxr = cfg->nh * cfg->P;
   rows.ldbv = rows.ldbr = rows.ldcv = rows.ldcr = cfg->N;
-  rows.lddv = rows.lddr = cfg->nh;
+  rows.lddv = rows.lddr = per_dir ? 2 * cfg->nh : cfg->nh;
+  rows.db_off = per_dir ? cfg->nh : 0;
   rows.v_bstride = L;
   rows.v_off = prefix_len;
   rows.r_bstride = L;
@@ -710,7 +737,24 @@ mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const 
   rows.W = cfg->W;
   rows.order = -1;
   rows.y_order = -1;
-  return run_ssd(cfg, rows, A_log, D, y, cfg->nh * cfg->P, n, sc, st);
+  return run_ssd(cfg, rows, A_log, D, y, cfg->nh * cfg->P, n, sc, st, per_dir ? A_log_b : nullptr,
+                 per_dir ? D_b : nullptr);
+}
+
+mate_status ssd_scan_bidir(const void* x, const void* Bm, const void* Cm, const float* dt, const float* dt_bias,
+                           const float* A_log, const float* D, int prefix_len, void* y, const mate_config* cfg,
+                           void* ws, size_t ws_bytes, mate_stream_t stream) {
+  return scan_impl(x, Bm, Cm, dt, dt_bias, A_log, D, nullptr, nullptr, nullptr, prefix_len, y, cfg, ws, ws_bytes,
+                   stream);
+}
+
+mate_status ssd_scan_bidir_pd(const void* x, const void* Bm, const void* Cm, const float* dt, const float* dt_bias,
+                              const float* A_log, const float* D, const float* dt_bias_b, const float* A_log_b,
+                              const float* D_b, int prefix_len, void* y, const mate_config* cfg, void* ws,
+                              size_t ws_bytes, mate_stream_t stream) {
+  if (dt_bias_b == nullptr || A_log_b == nullptr || D_b == nullptr) return MATE_ERR_ARG;
+  return scan_impl(x, Bm, Cm, dt, dt_bias, A_log, D, dt_bias_b, A_log_b, D_b, prefix_len, y, cfg, ws, ws_bytes,
+                   stream);
 }
 
 // Fixed scratch behind ssd_scan_bidir_noalloc.  In host code this name is only a stand-in for the
@@ -728,7 +772,7 @@ mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const void* Cm
                                    const mate_config* cfg, mate_stream_t stream) {
   MATE_TRY(check_config(cfg));
   if (prefix_len < 0) return MATE_ERR_ARG;
-  if (ssd_ws_bytes(cfg, prefix_len, nullptr, nullptr, nullptr) > MATE_SSD_NOALLOC_SCRATCH_BYTES)
+  if (ssd_ws_bytes(cfg, prefix_len, false, nullptr, nullptr, nullptr) > MATE_SSD_NOALLOC_SCRATCH_BYTES)
     return MATE_ERR_TOO_LARGE;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) {

@@ -96,11 +96,20 @@ __global__ void copy_block_kernel(const uint4* __restrict__ src, uint4* __restri
 }
 
 // delta = softplus(dt + dt_bias) for [rows, nh] raw step sizes.
-__global__ void softplus_kernel(const float* __restrict__ dt, const float* __restrict__ bias, float* __restrict__ out,
-                                long long total, int nh) {
+// out[row][c] = softplus(dt[row][c] + bias[c]); with bias2, rows of out hold 2 nh values and
+// out[row][nh + c] = softplus(dt[row][c] + bias2[c]).
+__global__ void softplus_kernel(const float* __restrict__ dt, const float* __restrict__ bias,
+                                const float* __restrict__ bias2, float* __restrict__ out, long long total, int nh) {
+  const int ld = bias2 != nullptr ? 2 * nh : nh;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
-    const float v = dt[i] + bias[i % nh];
-    out[i] = v > 20.f ? v : log1pf(expf(v));
+    const long long row = i / nh;
+    const int c = static_cast<int>(i - row * nh);
+    const float v = dt[i] + bias[c];
+    out[row * ld + c] = v > 20.f ? v : log1pf(expf(v));
+    if (bias2 != nullptr) {
+      const float v2 = dt[i] + bias2[c];
+      out[row * ld + nh + c] = v2 > 20.f ? v2 : log1pf(expf(v2));
+    }
   }
 }
 
@@ -113,7 +122,8 @@ __global__ void softplus_kernel(const float* __restrict__ dt, const float* __res
 __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A, int lda, const float* __restrict__ Bm,
                                                        int ldb, float* __restrict__ C, int ldc, int M, int N, int K,
                                                        float* __restrict__ delta, int ld_delta, int dt_col0,
-                                                       int dt_cols, const float* __restrict__ dt_bias) {
+                                                       int dt_cols, const float* __restrict__ dt_bias,
+                                                       const float* __restrict__ dt_bias2) {
   __shared__ float As[16][65];
   __shared__ float Bs[16][65];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -146,6 +156,10 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
       if (delta != nullptr && col >= dt_col0 && col < dt_col0 + dt_cols) {
         const float v = acc[a][c] + dt_bias[col - dt_col0];
         delta[(long long)r * ld_delta + col - dt_col0] = v > 20.f ? v : log1pf(expf(v));
+        if (dt_bias2 != nullptr) {   // the backward scan's step size, dt_cols columns further on
+          const float v2 = acc[a][c] + dt_bias2[col - dt_col0];
+          delta[(long long)r * ld_delta + dt_cols + col - dt_col0] = v2 > 20.f ? v2 : log1pf(expf(v2));
+        }
       }
     }
   }
@@ -162,6 +176,7 @@ struct SeqRows {
   int ldxr, ldbr, ldcr, lddr;
   long long v_bstride, v_off, r_bstride, r_off;
   int n, R, T, H, W;
+  int db_off;    // column offset of the backward direction's delta in the delta rows (0: shared delta)
   int order;     // scan order of the video input rows (row of scan position q: scan_to_raster(q)); -1: identity
   int y_order;   // scan order of the output rows (y of scan position q goes to row map(q)); -1: identity
   __host__ __device__ __forceinline__ int map(int q) const {
@@ -177,16 +192,19 @@ struct SeqRows {
 // fp32 selective scan, one CTA per (head, sample); thread (p, n) owns state element h[p][n].  Runs the
 // recurrence over [prefix; video] and then over [prefix; video reversed], adding both video outputs
 // into y at row b*y_bstride + map(q) (so the video rows land back in grid order when map is a scan).
-__global__ void ssd_f32_kernel(SeqRows s, const float* __restrict__ A_log, const float* __restrict__ Dp, int P, int N,
+__global__ void ssd_f32_kernel(SeqRows s, const float* __restrict__ A_log, const float* __restrict__ Dp,
+                               const float* __restrict__ A_log_b, const float* __restrict__ Dp_b, int P, int N,
                                float* __restrict__ y, int ldy, long long y_bstride) {
   extern __shared__ float red[];  // [P*N]
   const int h = blockIdx.x, b = blockIdx.y;
   const int p = threadIdx.x / N, nn = threadIdx.x % N;
   const bool active = threadIdx.x < P * N;
-  const float A = -expf(A_log[h]);
-  const float Dh = Dp[h];
   const int L = s.R + s.n;
   for (int dir = 0; dir < 2; ++dir) {
+    // the backward scan may have its own parameters and its delta at column offset db_off
+    const float A = -expf((dir == 1 && A_log_b != nullptr ? A_log_b : A_log)[h]);
+    const float Dh = (dir == 1 && Dp_b != nullptr ? Dp_b : Dp)[h];
+    const int dcol = (dir == 1 ? s.db_off : 0) + h;
     float hs = 0.f;
     for (int i = 0; i < L; ++i) {
       const float *xrow, *brow, *crow;
@@ -197,7 +215,7 @@ __global__ void ssd_f32_kernel(SeqRows s, const float* __restrict__ A_log, const
         xrow = static_cast<const float*>(s.xr) + r * s.ldxr;
         brow = static_cast<const float*>(s.br) + r * s.ldbr;
         crow = static_cast<const float*>(s.cr) + r * s.ldcr;
-        dl = s.dr[r * s.lddr + h];
+        dl = s.dr[r * s.lddr + dcol];
       } else {
         const int q = dir == 0 ? i - s.R : s.n - 1 - (i - s.R);
         const long long r = s.vrow(b, q);
@@ -205,7 +223,7 @@ __global__ void ssd_f32_kernel(SeqRows s, const float* __restrict__ A_log, const
         xrow = static_cast<const float*>(s.xv) + r * s.ldxv;
         brow = static_cast<const float*>(s.bv) + r * s.ldbv;
         crow = static_cast<const float*>(s.cv) + r * s.ldcv;
-        dl = s.dv[r * s.lddv + h];
+        dl = s.dv[r * s.lddv + dcol];
       }
       float xp = 0.f;
       if (active) {

@@ -63,6 +63,14 @@ struct SsdBf16Params {
   __nv_bfloat16* Hb;  // [B][nVc][nh][N][P]  state entering video chunk v, backward traversal
   int* crow;          // [B][nVc][Q]     source row of each video-chunk row (-1 past the end)
   float* tbl;         // [B][nVc][nh][2][kOutTbl]  decay tables of each 128-row tile (layout below)
+  // Optional separate parameters of the backward scan (null: shared with the forward scan).  With them,
+  // the backward delta sits at column s.db_off of the delta rows, glb holds the backward log-decays and
+  // Srb the review chunks' states under the backward parameters (the backward scan also runs over the
+  // review prefix first, in its stored order).
+  const float* A_log_b;
+  const float* Dp_b;
+  float* glb;           // [B][nRc + nVc][nh]
+  __nv_bfloat16* Srb;   // [B][nRc][nh][N][P]
   __nv_bfloat16* y;   // row b*y_bstride + map(q), column h*P
   int ldy;
   long long y_bstride;
@@ -302,21 +310,35 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
                       : make_uint4(0, 0, 0, 0);
     }
   };
+  const bool per_dir = p.A_log_b != nullptr;   // backward scan with its own A, D and delta
   load_x(blockIdx.z * heads_per_cta);
   float dl_next = myrw >= 0 ? cb.d[myrw * cb.ldd + blockIdx.z * heads_per_cta] : 0.f;
+  float dlb_next = per_dir ? (myrw >= 0 ? cb.d[myrw * cb.ldd + p.s.db_off + blockIdx.z * heads_per_cta] : 0.f)
+                           : dl_next;
 
   for (int hh = 0; hh < heads_per_cta; ++hh) {
     const int h = blockIdx.z * heads_per_cta + hh;
     const float A = -__expf(p.A_log[h]);
-    const float dl = dl_next;
+    const float dl = dl_next, dlb = dlb_next;
     const float a = dl * A;
     const float s = block_scan_256(a, wtot);
-    const float sx = s - a;
     if (j == 255) wtot[8 - 1] = s;  // reuse slot 7 for s_last after the scan finished with wtot
     if ((j & 63) == 63 && j < 255) bnd[j >> 6] = s;          // bnd[ib - 1] = s_{64 ib - 1}, ib = 1..3
-    if ((j & 63) == 0 && j > 0) bnd[4 + (j >> 6) - 1] = sx;  // bnd[4 + ib] = s'_{64 ib + 64}, ib = 0..2
     __syncthreads();
     const float s_last = wtot[7];
+    // backward scan quantities: the same as the forward ones unless the backward parameters differ
+    float ab = a, sbk = s, sb_last = s_last;
+    if (per_dir) {
+      ab = dlb * -__expf(p.A_log_b[h]);
+      __syncthreads();   // every thread has read s_last before the second scan reuses wtot
+      sbk = block_scan_256(ab, wtot);
+      if (j == 255) wtot[8 - 1] = sbk;
+      __syncthreads();
+      sb_last = wtot[7];
+    }
+    const float sx = sbk - ab;   // exclusive backward cumulative sum s'
+    if ((j & 63) == 0 && j > 0) bnd[4 + (j >> 6) - 1] = sx;  // bnd[4 + ib] = s'_{64 ib + 64}, ib = 0..2
+    __syncthreads();
     if (video) {
       // decay tables of the output kernel (see kOutTbl); thread j is token j of the chunk
       const long long cv = static_cast<long long>(b) * p.nVc + (c - p.nRc);
@@ -329,20 +351,24 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
       T[kTSi + r] = s * kLog2e;
       T[kTSx + r] = sx * kLog2e;
       T[kTEf + r] = __expf(s);
-      T[kTEb + r] = __expf(s_last - sx);
-      T[kTDl + r] = dl;
+      T[kTEb + r] = __expf(sb_last - sx);
+      T[kTDl + r] = 0.5f * (dl + dlb);   // the output epilogue's diagonal term uses 2 (D + G_ii dl)
       const float l2d = dl > 0.f ? __log2f(dl) : -INFINITY;
+      const float l2db = dlb > 0.f ? __log2f(dlb) : -INFINITY;
       T[kTLf + r] = l2d - s * kLog2e;
-      T[kTLb + r] = l2d + sx * kLog2e;
+      T[kTLb + r] = l2db + sx * kLog2e;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {   // column factors of row block q (stored with the tile holding it)
         float* W = T0 + (q >> 1) * kOutTbl + (q & 1) * 256 + j;
         W[kTWf] = (q > 0 && j < 64 * q) ? dl * __expf(bnd[q - 1] - s) : 0.f;
-        W[kTWb] = (q < 3 && j >= 64 * q + 64) ? dl * __expf(sx - bnd[4 + q]) : 0.f;
+        W[kTWb] = (q < 3 && j >= 64 * q + 64) ? dlb * __expf(sx - bnd[4 + q]) : 0.f;
       }
     }
+    if (threadIdx.x == 0 && per_dir) p.glb[(static_cast<long long>(b) * nC + c) * p.nh + h] = sb_last;
     sWf[j] = __expf(s_last - s) * dl;
-    sWb[j] = __expf(s - a) * dl;
+    // second product: the backward state of a video chunk (decay to its start); for a review chunk under
+    // separate backward parameters, its state at the chunk end under those parameters
+    sWb[j] = (video || !per_dir) ? __expf(sx) * dlb : __expf(sb_last - sbk) * dlb;
     __syncthreads();
     // weighted x tiles, 8 bf16 (one 16-byte chunk) per item; 8 items per row
 #pragma unroll
@@ -375,23 +401,25 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
       for (int k = 0; k < 16; ++k) {
         const uint64_t ad = desc_sw128(ab + k * 2048, 32768, 1024);
         mma_bf16_ss(tmem, ad, desc_sw128(xf + k * 2048, 32768, 1024), idesc, k > 0);
-        if (video) mma_bf16_ss(tmem + 64, ad, desc_sw128(xb + k * 2048, 32768, 1024), idesc, k > 0);
+        if (video || per_dir) mma_bf16_ss(tmem + 64, ad, desc_sw128(xb + k * 2048, 32768, 1024), idesc, k > 0);
       }
       mma_commit(bar);
     }
     if (hh + 1 < heads_per_cta) {
       load_x(h + 1);
       dl_next = myrw >= 0 ? cb.d[myrw * cb.ldd + h + 1] : 0.f;
+      dlb_next = per_dir ? (myrw >= 0 ? cb.d[myrw * cb.ldd + p.s.db_off + h + 1] : 0.f) : dl_next;
     }
     mbar_wait(bar, phase);
     phase ^= 1;
     tc_fence_after();
     const int dir = warp >> 2, quad = warp & 3;
     const int nidx = quad * 32 + lane;
-    if (dir == 0 || video) {
+    if (dir == 0 || video || per_dir) {
       __nv_bfloat16* dst = dir == 0
           ? p.Sf + ((static_cast<long long>(b) * nC + c) * p.nh + h) * (kSsdP * kSsdN)
-          : p.Sb + ((static_cast<long long>(b) * p.nVc + (c - p.nRc)) * p.nh + h) * (kSsdP * kSsdN);
+          : (video ? p.Sb + ((static_cast<long long>(b) * p.nVc + (c - p.nRc)) * p.nh + h) * (kSsdP * kSsdN)
+                   : p.Srb + ((static_cast<long long>(b) * p.nRc + c) * p.nh + h) * (kSsdP * kSsdN));
       // lane = state row n: its 64 p values are one contiguous 128-byte row of the [N][P] state
       for (int pc = 0; pc < 2; ++pc) {
         uint32_t r[32];
@@ -451,9 +479,13 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
     for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(H[2 * e], H[2 * e + 1]);
     *reinterpret_cast<uint4*>(base + e8 * 8) = o;
   };
+  const bool bwd_own = dir == 1 && p.A_log_b != nullptr;   // backward scan with its own parameters
+  const float* gld = bwd_own ? p.glb : p.gl;
   for (int c = 0; c < p.nRc; ++c) {
     const long long ci = (static_cast<long long>(b) * nC + c) * p.nh + h;
-    step(p.gl[ci], __ldg(reinterpret_cast<const uint4*>(p.Sf + ci * PN) + e8));
+    const __nv_bfloat16* S = bwd_own ? p.Srb + ((static_cast<long long>(b) * p.nRc + c) * p.nh + h) * PN
+                                     : p.Sf + ci * PN;
+    step(gld[ci], __ldg(reinterpret_cast<const uint4*>(S) + e8));
   }
   constexpr int U = 16;   // chunks in flight per thread (4: 0.30 ms, 8: 0.27 ms, 16: 0.22 ms at 1024 chunks)
   for (int k0 = 0; k0 < p.nVc; k0 += U) {
@@ -466,7 +498,7 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
         const int v = dir == 0 ? k : p.nVc - 1 - k;
         const long long ci = (static_cast<long long>(b) * nC + p.nRc + v) * p.nh + h;
         const long long vi = (static_cast<long long>(b) * p.nVc + v) * p.nh + h;
-        gv[u] = p.gl[ci];
+        gv[u] = gld[ci];
         sv[u] = __ldg(reinterpret_cast<const uint4*>((dir == 0 ? p.Sf + ci * PN : p.Sb + vi * PN)) + e8);
       }
     }
@@ -832,7 +864,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
       const long long yrow = b * p.y_bstride + p.s.map(v * kSsdQ + (valid ? i : 0));
       for (int h = 0; h < nh; ++h, ++k) {
         const int buf = k & 1, acc = k & 1, use = k >> 1;
-        const float Dh = p.Dp[h];
+        const float Dh = p.Dp_b != nullptr ? 0.5f * (p.Dp[h] + p.Dp_b[h]) : p.Dp[h];
         if (!wait_all(&y_full[acc], use & 1)) { ok = false; break; }
         tc_fence_after();
         const uint8_t* XB = smem + buf * kOutXBuf;

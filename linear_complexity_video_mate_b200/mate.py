@@ -13,7 +13,8 @@ import torch
 
 from . import _lib
 
-__all__ = ["MateBlock", "rms_permute", "rms_unpermute", "review_pool", "ssd_scan_bidir", "tesa_forward",
+__all__ = ["MateBlock", "rms_permute", "rms_unpermute", "review_pool", "ssd_scan_bidir", "ssd_scan_bidir_pd",
+           "tesa_forward",
            "project_bf16", "device_status", "torch_dtype", "weights_to_device"]
 
 
@@ -42,8 +43,9 @@ def weights_to_device(w: Dict, cfg, device="cuda") -> Dict[str, torch.Tensor]:
     out = {}
     for k in ("W_in", "W_out", "W_qkv", "W_o"):
         out[k] = torch.as_tensor(w[k]).to(device=device, dtype=dt).contiguous()
-    for k in ("dt_bias", "A_log", "D"):
-        out[k] = torch.as_tensor(w[k]).to(device=device, dtype=torch.float32).contiguous()
+    for k in ("dt_bias", "A_log", "D", "dt_bias_b", "A_log_b", "D_b"):
+        if k in w:   # the last three are the optional backward-scan parameters
+            out[k] = torch.as_tensor(w[k]).to(device=device, dtype=torch.float32).contiguous()
     return out
 
 
@@ -65,8 +67,14 @@ class MateBlock:
         _need(weights["W_o"], self.dtype, cfg.d * cfg.th * cfg.tp, "W_o")
         for k in ("dt_bias", "A_log", "D"):
             _need(weights[k], torch.float32, cfg.nh, k)
-        self.cw = _lib.CWeights(*(weights[k].data_ptr() for k in
-                                  ("W_in", "dt_bias", "A_log", "D", "W_out", "W_qkv", "W_o")))
+        bwd = [k for k in ("dt_bias_b", "A_log_b", "D_b") if k in weights]
+        if bwd and len(bwd) != 3:
+            raise ValueError(f"backward-scan parameters: give dt_bias_b, A_log_b and D_b together, got {bwd}")
+        for k in bwd:
+            _need(weights[k], torch.float32, cfg.nh, k)
+        self.cw = _lib.CWeights(*(weights[k].data_ptr() if k in weights else None for k in
+                                  ("W_in", "dt_bias", "A_log", "D", "W_out", "W_qkv", "W_o", "dt_bias_b", "A_log_b",
+                                   "D_b")))
         self.ws_bytes = lib.mate_workspace_bytes(ctypes.byref(self.ccfg))
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
         self.ws_host = None
@@ -148,6 +156,24 @@ def ssd_scan_bidir(x, Bm, Cm, dt, dt_bias, A_log, D, prefix_len: int, cfg, out=N
     st = lib.ssd_scan_bidir(_p(x), _p(Bm), _p(Cm), _p(dt), _p(dt_bias), _p(A_log), _p(D), int(prefix_len), _p(out),
                             ctypes.byref(c), _p(ws), ws.numel(), _s(stream))
     _lib.check(st, "ssd_scan_bidir")
+    return out
+
+
+def ssd_scan_bidir_pd(x, Bm, Cm, dt, dt_bias, A_log, D, dt_bias_b, A_log_b, D_b, prefix_len: int, cfg, out=None,
+                      ws=None, stream=None):
+    """ssd_scan_bidir with the backward scan's own step-size bias, A_log and D ([nh] fp32 each)."""
+    lib = _lib.load()
+    c = _cfg(cfg)
+    n = cfg.T * cfg.H * cfg.W
+    if out is None:
+        out = torch.empty((cfg.B, n, cfg.nh * cfg.P), dtype=x.dtype, device=x.device)
+    nb = lib.mate_ssd_pd_workspace_bytes(ctypes.byref(c), int(prefix_len))
+    if ws is None or ws.numel() < nb:
+        ws = torch.empty(nb, dtype=torch.uint8, device=x.device)
+    st = lib.ssd_scan_bidir_pd(_p(x), _p(Bm), _p(Cm), _p(dt), _p(dt_bias), _p(A_log), _p(D), _p(dt_bias_b),
+                               _p(A_log_b), _p(D_b), int(prefix_len), _p(out), ctypes.byref(c), _p(ws), ws.numel(),
+                               _s(stream))
+    _lib.check(st, "ssd_scan_bidir_pd")
     return out
 
 

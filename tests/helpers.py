@@ -64,9 +64,9 @@ def assert_close(got, ref, dtype, what="", floor=0.0):
     return rel, rms_abs
 
 
-def _oracle_digest():
+def _oracle_digest(extra=()):
     h = hashlib.sha256()
-    for f in ("oracle/mate_oracle.py", "mate_inputs.py"):
+    for f in ("oracle/mate_oracle.py", "mate_inputs.py") + tuple(extra):
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -76,10 +76,11 @@ CACHE_BIG = os.path.join(ROOT, ".oracle_cache_big")
 BIG_BYTES = 8 << 20
 
 
-def oracle_cached(key: str, fn):
+def oracle_cached(key: str, fn, extra=()):
     """fn() -> np.ndarray, cached on disk (as float32: far below every tolerance) under a key that includes
-    the oracle's source digest.  Small results and large ones are kept in separate folders."""
-    name = f"{key}-{_oracle_digest()}.npy"
+    the oracle's source digest (plus the files `extra` names).  Small results and large ones are kept in
+    separate folders."""
+    name = f"{key}-{_oracle_digest(extra)}.npy"
     for d in (CACHE, CACHE_BIG):
         if os.path.exists(os.path.join(d, name)):
             return np.load(os.path.join(d, name)).astype(np.float64)

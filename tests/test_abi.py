@@ -85,6 +85,15 @@ def test_null_and_misaligned_arguments_are_rejected_before_launch(lib):
     nss = lib.mate_ssd_workspace_bytes(cp, 256)
     assert lib.ssd_scan_bidir(fake, fake, fake, fake, fake, fake, fake, 256, fake, cp, fake, nss - 1, None) == \
         _lib.MATE_ERR_WORKSPACE
+    # separate backward-scan parameters: all three or none
+    wp = _lib.CWeights(*([1 << 20] * 8))
+    assert lib.mate_forward(fake, ctypes.byref(wp), 0, fake, cp, fake, 1 << 40, None) == _lib.MATE_ERR_ARG
+    assert lib.ssd_scan_bidir_pd(fake, fake, fake, fake, fake, fake, fake, fake, None, fake, 256, fake, cp, fake,
+                                 1 << 40, None) == _lib.MATE_ERR_ARG
+    npd = lib.mate_ssd_pd_workspace_bytes(cp, 256)
+    assert npd > nss   # the backward scan's own step sizes, decays and review states
+    assert lib.ssd_scan_bidir_pd(fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, 256, fake, cp, fake,
+                                 npd - 1, None) == _lib.MATE_ERR_WORKSPACE
     assert lib.mate_project_bf16(fake, 512, 128, 1024, fake, 1024, 256, fake, 256, None) == _lib.MATE_ERR_ARG
     assert lib.mate_project_bf16(fake, 1000, 128, 1000, fake, 1000, 256, fake, 256, None) == \
         _lib.MATE_ERR_UNSUPPORTED
