@@ -468,3 +468,108 @@ def test_per_direction_with_shared_parameters_is_the_shared_oracle():
     x, Bm, Cm, df, Af, Df, db, Ab, Db, R = _pd_case()
     np.testing.assert_allclose(PD.ssd_bidirectional_per_direction(x, Bm, Cm, df, Af, Df, df, Af, Df, R),
                                O.ssd_bidirectional(x, Bm, Cm, df, Af, Df, R), rtol=0, atol=0)
+
+
+# ------------------------------------------------------------------ Mamba2 block extras (conv, gate, norm)
+
+from oracle import mamba2_extras as MX  # noqa: E402
+
+
+def test_silu_values_and_identities():
+    assert MX.silu(np.array([0.0]))[0] == 0.0
+    assert abs(MX.silu(np.array([1.0]))[0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+    v = np.linspace(-30, 30, 121)
+    np.testing.assert_allclose(MX.silu(v) - MX.silu(-v), v, rtol=0, atol=1e-12)   # v s(v) - (-v) s(-v) = v
+    assert abs(MX.silu(np.array([60.0]))[0] - 60.0) < 1e-12
+    assert abs(MX.silu(np.array([-60.0]))[0]) < 1e-20
+
+
+def test_causal_conv_equals_library_convolution():
+    """Per channel, the causal convolution is numpy's full convolution with the taps reversed, truncated
+    to the first L outputs, plus the bias."""
+    rng = np.random.default_rng(11)
+    L, C, K = 37, 5, MX.CONV_K
+    u, w, b = rng.standard_normal((L, C)), rng.standard_normal((C, K)), rng.standard_normal(C)
+    got = MX.causal_conv(u, w, b)
+    for c in range(C):
+        np.testing.assert_allclose(got[:, c], np.convolve(u[:, c], w[c, ::-1])[:L] + b[c], rtol=1e-13, atol=1e-13)
+
+
+def test_causal_conv_impulse_response_is_causal():
+    """A unit impulse at row t0 of channel c reaches rows t0 .. t0 + 3 only, with taps K-1, K-2, ... in turn."""
+    rng = np.random.default_rng(12)
+    L, C, t0, c = 12, 3, 5, 1
+    w, b = rng.standard_normal((C, MX.CONV_K)), np.zeros(C)
+    u = np.zeros((L, C))
+    u[t0, c] = 1.0
+    got = MX.causal_conv(u, w, b)
+    want = np.zeros(L)
+    for j in range(MX.CONV_K):
+        want[t0 + j] = w[c, MX.CONV_K - 1 - j]
+    np.testing.assert_array_equal(got[:, c], want)
+    assert not got[:, [0, 2]].any()
+
+
+def test_gated_rmsnorm_normalises_after_the_gate():
+    """With weight 1 and eps 0 every row of the result has root-mean-square 1 whatever z is (the norm
+    comes after the gate), and scaling y leaves it unchanged; a 2-channel row has a closed form."""
+    rng = np.random.default_rng(13)
+    y, z = rng.standard_normal((9, 16)), rng.standard_normal((9, 16))
+    out = MX.gated_rmsnorm(y, z, np.ones(16), eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(out ** 2, axis=1)), 1.0, rtol=1e-13)
+    np.testing.assert_allclose(MX.gated_rmsnorm(7.5 * y, z, np.ones(16), eps=0.0), out, rtol=1e-12, atol=1e-13)
+    row = MX.gated_rmsnorm(np.array([[3.0, 4.0]]), np.array([[50.0, 50.0]]), np.array([2.0, -1.0]), eps=0.0)
+    np.testing.assert_allclose(row, [[2.0 * 3.0 / math.sqrt(12.5), -4.0 / math.sqrt(12.5)]], rtol=1e-12)
+    # eps enters under the root: a zero row stays zero, a tiny row is damped
+    assert not MX.gated_rmsnorm(np.zeros((1, 4)), np.ones((1, 4)), np.ones(4)).any()
+
+
+def _extras_weights(cfg, seed):
+    rng = np.random.default_rng(seed)
+    nP, C = cfg.nh * cfg.P, cfg.nh * cfg.P + 2 * cfg.N
+    return dict(W_z=rng.standard_normal((nP, cfg.d)) / math.sqrt(cfg.d),
+                conv_w=rng.uniform(-0.5, 0.5, (C, MX.CONV_K)), conv_b=rng.uniform(-0.5, 0.5, C),
+                norm_w=1.0 + 0.1 * rng.standard_normal(nP))
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+def test_extras_branch_fast_decay_closed_form(layer):
+    """Decays that all underflow and a convolution that only delays by one row: the MA branch reduces to
+    y_i = 2 (D + C'_i . B'_i delta_i) x'_i with x', B', C' = silu(bias + the previous sequence row's
+    projection), then gate, norm and out-projection, written out here directly.  The delay runs along the
+    scan sequence [review; video in scan order], so a wrong axis or direction of the convolution fails."""
+    cfg = _small_cfg()
+    w = dict(make_inputs(cfg, dt_bias=2.0))
+    w.update(_extras_weights(cfg, 14))
+    w["A_log"] = np.full(cfg.nh, 12.0)
+    conv_w = np.zeros_like(w["conv_w"])
+    conv_w[:, MX.CONV_K - 2] = 1.0
+    w["conv_w"] = conv_w
+    X3 = np.asarray(w["X"][0], np.float64)
+    order = layer % 4
+    nP, N = cfg.nh * cfg.P, cfg.N
+    Xp = O.rms_permute(X3, order)
+    S = np.concatenate([O.review_tokens(X3, cfg.R, order), Xp], axis=0)
+    Z = S @ np.asarray(w["W_in"], np.float64).T
+    prev = np.concatenate([np.zeros((1, nP + 2 * N)), Z[:-1, :nP + 2 * N]], axis=0)
+    v = prev + w["conv_b"][None, :]
+    act = v / (1.0 + np.exp(-v))
+    x, Bm, Cm = act[:, :nP].reshape(-1, cfg.nh, cfg.P), act[:, nP:nP + N], act[:, nP + N:]
+    delta = np.log1p(np.exp(Z[:, nP + 2 * N:] + 2.0))
+    cb = np.einsum("ln,ln->l", Cm, Bm)
+    y = (2.0 * (np.asarray(w["D"], np.float64)[None, :] + cb[:, None] * delta)[:, :, None] * x)[cfg.R:]
+    zz = Xp @ w["W_z"].T
+    g = y.reshape(cfg.n, nP) * zz / (1.0 + np.exp(-zz))
+    yn = g / np.sqrt(np.mean(g * g, axis=1, keepdims=True) + 1e-5) * w["norm_w"]
+    want = O.rms_unpermute(yn @ np.asarray(w["W_out"], np.float64).T, order, cfg.T, cfg.H, cfg.W)
+    np.testing.assert_allclose(MX.ma_branch_extras(X3, w, cfg, layer), want, rtol=1e-10, atol=1e-10)
+
+
+def test_extras_block_is_sum_of_branches():
+    cfg = _small_cfg()
+    w = dict(make_inputs(cfg))
+    w.update(_extras_weights(cfg, 15))
+    full = MX.mate_forward_extras(w["X"], w, cfg, 1)
+    ma = np.stack([MX.ma_branch_extras(w["X"][0], w, cfg, 1)])
+    te = O.mate_forward(w["X"], dict(w, W_out=np.zeros_like(w["W_out"])), cfg, 1)
+    np.testing.assert_allclose(full, ma + te, rtol=1e-12, atol=1e-12)
