@@ -68,6 +68,12 @@ typedef enum { MATE_BF16 = 0, MATE_F32 = 1 } mate_dtype;
  * bf16 tensor-core path additionally: d % 64 == 0, nh % 8 == 0, P == 64, N == 128, Q == 256,
  * tp == 128, wt*wh*ww == 256.  fp32 path (CUDA-core kernels, for small blocks): P*N <= 1024, tp <= 128.
  * B * (T*H*W + R) < 2^31.
+ * mamba_extras = 1 gives the MA branch the rest of a Mamba2 block around the scan: a causal depthwise
+ * convolution of width 4 with bias + SiLU on x | B | C (along [review rows; video rows in scan order],
+ * zero before each sample's first row, one pass feeding both scan directions), the gate z = W_z X of the
+ * video rows and gated RMSNorm  y <- (y silu(z)) / sqrt(mean((y silu(z))^2) + 1e-5) * norm_w  over each
+ * row's nh*P channels before the out-projection.  The pages name a Mamba2 block without listing its
+ * parts; these are the standard ones.  0 (default): projections and scan only.
  */
 typedef struct {
   int B, T, H, W, d;
@@ -76,6 +82,7 @@ typedef struct {
   int wt, wh, ww;
   int st, sh, sw;
   mate_dtype dtype;
+  int mamba_extras; /* 0 or 1 */
 } mate_config;
 
 /* Block weights, device pointers, caller-owned.  Element type cfg->dtype except the fp32 vectors. */
@@ -92,6 +99,11 @@ typedef struct {
   const float* dt_bias_b; /* [nh] */
   const float* A_log_b;   /* [nh] */
   const float* D_b;       /* [nh] */
+  /* Required when cfg->mamba_extras = 1, ignored otherwise. */
+  const void* W_z;        /* [nh*P, d]  gate projection                                              */
+  const float* conv_w;    /* [nh*P + 2N, 4] depthwise taps per channel of x | B | C, tap 3 on the current row */
+  const float* conv_b;    /* [nh*P + 2N]  convolution bias                                           */
+  const float* norm_w;    /* [nh*P]   gated RMSNorm weight                                           */
 } mate_weights;
 
 /* Human-readable name of a status code (static string). */
@@ -297,7 +309,9 @@ typedef enum {
   MATE_K_RMS_GATHER = 13,
   MATE_K_PROJECT = 14,         /* mate_project_bf16 */
   MATE_K_SCAN_LOCALITY = 15,   /* mate_scan_locality */
-  MATE_K_Y_TO_GRID = 16        /* scan-order y rows back to grid order (time-fastest scan orders) */
+  MATE_K_Y_TO_GRID = 16,       /* scan-order y rows back to grid order (time-fastest scan orders) */
+  MATE_K_CONV_SILU = 17,       /* causal depthwise convolution + SiLU on x | B | C (mamba_extras) */
+  MATE_K_GATE_NORM = 18        /* y silu(z) and gated RMSNorm (mamba_extras) */
 } mate_kernel;
 
 typedef struct {

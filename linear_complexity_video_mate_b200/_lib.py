@@ -23,14 +23,15 @@ _CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp",
 
 
 class CConfig(ctypes.Structure):
-    _fields_ = [(f, ctypes.c_int) for f in _CONFIG_FIELDS] + [("dtype", ctypes.c_int)]
+    _fields_ = [(f, ctypes.c_int) for f in _CONFIG_FIELDS] + [("dtype", ctypes.c_int), ("mamba_extras", ctypes.c_int)]
 
 
 class CWeights(ctypes.Structure):
     _fields_ = [("W_in", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
                 ("D", ctypes.c_void_p), ("W_out", ctypes.c_void_p), ("W_qkv", ctypes.c_void_p),
                 ("W_o", ctypes.c_void_p), ("dt_bias_b", ctypes.c_void_p), ("A_log_b", ctypes.c_void_p),
-                ("D_b", ctypes.c_void_p)]
+                ("D_b", ctypes.c_void_p), ("W_z", ctypes.c_void_p), ("conv_w", ctypes.c_void_p),
+                ("conv_b", ctypes.c_void_p), ("norm_w", ctypes.c_void_p)]
 
 
 class CTraceRecord(ctypes.Structure):
@@ -98,10 +99,12 @@ def check(status: int, where: str):
         raise MateError(status, where)
 
 
-def make_config(cfg) -> CConfig:
-    """C config from any object with the block's shape attributes (e.g. mate_inputs.MateConfig)."""
+def make_config(cfg, mamba_extras: bool = False) -> CConfig:
+    """C config from any object with the block's shape attributes (e.g. mate_inputs.MateConfig);
+    mamba_extras adds the convolution, gate and gated norm of a full Mamba2 block."""
     c = CConfig()
     for f in _CONFIG_FIELDS:
         setattr(c, f, int(getattr(cfg, f)))
     c.dtype = MATE_BF16 if cfg.dtype == "bf16" else MATE_F32
+    c.mamba_extras = 1 if mamba_extras else 0
     return c

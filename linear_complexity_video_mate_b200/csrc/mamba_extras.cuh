@@ -1,0 +1,158 @@
+// The rest of a Mamba2 block around the bidirectional scan (optional part of the MATE block's MA branch;
+// the pages name the branch's core a bidirectional Mamba2 block without listing its internals):
+//   * conv_silu_kernel     causal depthwise convolution (width 4, bias) + SiLU over the x | B | C channels,
+//                          along each sample's scan sequence [review rows; video rows in scan order];
+//   * gate_rmsnorm_kernel  y <- (y * silu(z)) / sqrt(mean((y * silu(z))^2) + eps) * norm_w, per row, in place.
+// Both are HBM-bound streams of whole rows: coalesced 16-byte vectors where the row strides allow, fp32
+// arithmetic, the storage type's rounding on the way out.
+#pragma once
+#include "common.cuh"
+#include "simt.cuh"
+
+namespace mate {
+
+constexpr int kConvK = 4;          // taps of the causal convolution; tap kConvK - 1 is the current row
+constexpr int kConvRun = 16;       // sequence positions per thread (the window slides in registers)
+constexpr float kNormEps = 1e-5f;  // epsilon of the gated RMSNorm
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T_> __device__ __forceinline__ T_ from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// V consecutive elements as fp32; one 16-byte access when V elements fill 16 bytes (the caller has
+// checked the alignment), else element by element.
+template <typename T_, int V>
+__device__ __forceinline__ void load_vec(const T_* p, float (&f)[V]) {
+  if constexpr (sizeof(T_) * V == 16) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const T_* e = reinterpret_cast<const T_*>(&u);
+#pragma unroll
+    for (int i = 0; i < V; ++i) f[i] = to_f32(e[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i) f[i] = to_f32(p[i]);
+  }
+}
+
+template <typename T_, int V>
+__device__ __forceinline__ void store_vec(T_* p, const float (&f)[V]) {
+  if constexpr (sizeof(T_) * V == 16) {
+    uint4 u;
+    T_* e = reinterpret_cast<T_*>(&u);
+#pragma unroll
+    for (int i = 0; i < V; ++i) e[i] = from_f32<T_>(f[i]);
+    *reinterpret_cast<uint4*>(p) = u;
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i) p[i] = from_f32<T_>(f[i]);
+  }
+}
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.f + __expf(-v)); }
+
+// Causal depthwise convolution + SiLU.  Sequence position i of sample b reads the source row of s (prefix
+// row rrow(b, i) of s.xr for i < R, else video row vrow(b, i - R) of s.xv, row strides s.ldxr / s.ldxv)
+// and writes the same row of the outputs (out_r / out_v, row stride ldo).  Channels [0, C), C a
+// multiple of V.  Thread g owns channel vector g % nvec and the kConvRun positions of run g / nvec; the
+// kConvK - 1 rows before its run are read again as its window's start (zero before position 0).
+// w: [C][kConvK] fp32, tap kConvK - 1 on the current row; bias: [C].
+template <typename T_, int V>
+__global__ void __launch_bounds__(256) conv_silu_kernel(SeqRows s, int C, const float* __restrict__ w,
+                                                        const float* __restrict__ bias, T_* __restrict__ out_v,
+                                                        T_* __restrict__ out_r, int ldo, int nruns, int B) {
+  const int nvec = C / V;
+  const long long total = (long long)B * nruns * nvec;
+  const int L = s.R + s.n;
+  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+       g += (long long)gridDim.x * blockDim.x) {
+    const int vi = static_cast<int>(g % nvec);
+    const long long rb = g / nvec;
+    const int b = static_cast<int>(rb / nruns);
+    const int i0 = static_cast<int>(rb - (long long)b * nruns) * kConvRun;
+    const int c0 = vi * V;
+    float wt[V][kConvK], bs[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      const float4 t = __ldg(reinterpret_cast<const float4*>(w + (size_t)(c0 + e) * kConvK));
+      wt[e][0] = t.x; wt[e][1] = t.y; wt[e][2] = t.z; wt[e][3] = t.w;
+      bs[e] = __ldg(bias + c0 + e);
+    }
+    // window[k] holds position i - (kConvK - 1) + k
+    float win[kConvK][V];
+#pragma unroll
+    for (int k = 0; k < kConvK - 1; ++k) {
+      const int i = i0 - (kConvK - 1) + k;
+      if (i < 0) {
+#pragma unroll
+        for (int e = 0; e < V; ++e) win[k][e] = 0.f;
+      } else {
+        const T_* src = i < s.R ? static_cast<const T_*>(s.xr) + s.rrow(b, i) * s.ldxr
+                                : static_cast<const T_*>(s.xv) + s.vrow(b, i - s.R) * s.ldxv;
+        load_vec<T_, V>(src + c0, win[k]);
+      }
+    }
+    const int i_end = min(L, i0 + kConvRun);
+    for (int i = i0; i < i_end; ++i) {
+      const bool pre = i < s.R;
+      const long long row = pre ? s.rrow(b, i) : s.vrow(b, i - s.R);
+      const T_* src = pre ? static_cast<const T_*>(s.xr) + row * s.ldxr : static_cast<const T_*>(s.xv) + row * s.ldxv;
+      load_vec<T_, V>(src + c0, win[kConvK - 1]);
+      float o[V];
+#pragma unroll
+      for (int e = 0; e < V; ++e) {
+        float acc = bs[e];
+#pragma unroll
+        for (int k = 0; k < kConvK; ++k) acc = fmaf(wt[e][k], win[k][e], acc);
+        o[e] = silu_f(acc);
+      }
+      store_vec<T_, V>((pre ? out_r : out_v) + row * ldo + c0, o);
+#pragma unroll
+      for (int k = 0; k < kConvK - 1; ++k)
+#pragma unroll
+        for (int e = 0; e < V; ++e) win[k][e] = win[k + 1][e];
+    }
+  }
+}
+
+// Gated RMSNorm in place, one warp per row: g = y * silu(z) over the row's C channels (C a multiple of
+// V), y <- g * rsqrt(mean(g^2) + eps) * norm_w.  The second pass recomputes g from the row, which the
+// first pass left in L1.
+template <typename T_, int V>
+__global__ void __launch_bounds__(256) gate_rmsnorm_kernel(T_* __restrict__ y, long long ldy,
+                                                           const T_* __restrict__ z, long long ldz,
+                                                           const float* __restrict__ norm_w, int C,
+                                                           long long rows) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  const int nvec = C / V;
+  for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    T_* yr = y + r * ldy;
+    const T_* zr = z + r * ldz;
+    float ss = 0.f;
+    for (int v = lane; v < nvec; v += 32) {
+      float a[V], c[V];
+      load_vec<T_, V>(yr + v * V, a);
+      load_vec<T_, V>(zr + v * V, c);
+#pragma unroll
+      for (int e = 0; e < V; ++e) {
+        const float g = a[e] * silu_f(c[e]);
+        ss = fmaf(g, g, ss);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = rsqrtf(ss / static_cast<float>(C) + kNormEps);
+    for (int v = lane; v < nvec; v += 32) {
+      float a[V], c[V];
+      load_vec<T_, V>(yr + v * V, a);
+      load_vec<T_, V>(zr + v * V, c);
+#pragma unroll
+      for (int e = 0; e < V; ++e) a[e] = a[e] * silu_f(c[e]) * inv * __ldg(norm_w + v * V + e);
+      store_vec<T_, V>(yr + v * V, a);
+    }
+  }
+}
+
+}  // namespace mate

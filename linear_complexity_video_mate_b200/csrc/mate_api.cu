@@ -19,6 +19,7 @@
 #include "ssd_bf16.cuh"
 #include "tesa_bf16.cuh"
 #include "locality.cuh"
+#include "mamba_extras.cuh"
 
 using namespace mate;
 
@@ -132,6 +133,7 @@ size_t elem_size(const mate_config* c) { return c->dtype == MATE_BF16 ? 2 : 4; }
 mate_status check_config(const mate_config* c) {
   if (c == nullptr) return MATE_ERR_ARG;
   if (c->dtype != MATE_BF16 && c->dtype != MATE_F32) return MATE_ERR_ARG;
+  if (c->mamba_extras != 0 && c->mamba_extras != 1) return MATE_ERR_ARG;
   if (c->B <= 0 || c->T <= 0 || c->H <= 0 || c->W <= 0 || c->d <= 0 || c->nh <= 0 || c->P <= 0 || c->N <= 0 ||
       c->Q <= 0 || c->R < 0 || c->th <= 0 || c->tp <= 0 || c->wt <= 0 || c->wh <= 0 || c->ww <= 0)
     return MATE_ERR_SHAPE;
@@ -200,7 +202,9 @@ SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh, bool per_dir
 
 struct ForwardPlan {
   int NIn, NI, KO;
+  int zc0;               // first gate column of the video rows' projection (mamba_extras), else -1
   void *Wi, *Wo, *Rv, *Zv, *Zr, *YO, *Ys;
+  void *XBv, *XBr;       // convolved x | B | C rows (mamba_extras), same row order as Zv / Zr
   float *Dv, *Dr;
   SsdScratch ssd;
   size_t bytes;
@@ -213,6 +217,11 @@ ForwardPlan plan_forward(const mate_config* c, void* ws) {
   const long long n = (long long)c->T * c->H * c->W;
   p.NIn = c->nh * c->P + 2 * c->N + c->nh;
   p.NI = p.NIn + 3 * c->th * c->tp;
+  p.zc0 = -1;
+  if (c->mamba_extras) {   // gate columns after q | k | v
+    p.zc0 = p.NI;
+    p.NI += c->nh * c->P;
+  }
   p.KO = c->nh * c->P + c->th * c->tp;
   p.Wi = cv.take<char>((size_t)p.NI * c->d * es);
   p.Wo = cv.take<char>((size_t)c->d * p.KO * es);
@@ -222,6 +231,9 @@ ForwardPlan plan_forward(const mate_config* c, void* ws) {
   p.Dv = cv.take<float>((size_t)c->B * n * 2 * c->nh);      // [rows][nh forward | nh backward]
   p.Dr = cv.take<float>((size_t)c->B * c->R * 2 * c->nh);
   p.YO = cv.take<char>((size_t)c->B * n * p.KO * es);
+  const size_t Cx = (size_t)c->nh * c->P + 2 * c->N;
+  p.XBv = c->mamba_extras ? cv.take<char>((size_t)c->B * n * Cx * es) : nullptr;
+  p.XBr = c->mamba_extras ? cv.take<char>((size_t)c->B * c->R * Cx * es) : nullptr;
   // y in scan order, for the time-fastest orders (their grid-order y rows are 1024s of rows apart)
   p.Ys = c->dtype == MATE_BF16 ? cv.take<char>((size_t)c->B * n * c->nh * c->P * es) : nullptr;
   if (c->dtype == MATE_BF16) p.ssd = carve_ssd(cv, c->B, n, c->R, c->nh, true);
@@ -486,6 +498,64 @@ HostIo* host_io() {
   return io.ready ? &io : nullptr;
 }
 
+// Causal depthwise convolution + SiLU of the Cx channels [0, Cx) of the sequence rows `rows` (source
+// rows rows.xv / rows.xr, strides rows.ldxv / rows.ldxr) into out_v / out_r (row stride Cx).
+mate_status run_conv(const mate_config* c, const SeqRows& rows, int Cx, const float* w, const float* bias, void* out_v,
+                     void* out_r, cudaStream_t st) {
+  const long long L = (long long)rows.R + rows.n;
+  const int nruns = ceil_div(L, kConvRun);
+  const size_t es = elem_size(c);
+  // 16-byte vectors when every row start and the channel count allow them
+  const bool vec = (Cx * es) % 16 == 0 && (rows.ldxv * es) % 16 == 0 && (rows.ldxr * es) % 16 == 0 &&
+                   aligned16(rows.xv) && aligned16(rows.xr);
+  const int V = vec ? static_cast<int>(16 / es) : 1;
+  const long long total = (long long)c->B * nruns * (Cx / V);
+  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, (long long)device_sms() * 16));
+  if (total == 0) return MATE_OK;
+  trace_begin(MATE_K_CONV_SILU, st);
+  if (c->dtype == MATE_BF16) {
+    if (vec)
+      conv_silu_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(rows, Cx, w, bias, static_cast<__nv_bfloat16*>(out_v),
+                                                                static_cast<__nv_bfloat16*>(out_r), Cx, nruns, c->B);
+    else
+      conv_silu_kernel<__nv_bfloat16, 1><<<blocks, 256, 0, st>>>(rows, Cx, w, bias, static_cast<__nv_bfloat16*>(out_v),
+                                                                static_cast<__nv_bfloat16*>(out_r), Cx, nruns, c->B);
+  } else {
+    if (vec)
+      conv_silu_kernel<float, 4><<<blocks, 256, 0, st>>>(rows, Cx, w, bias, static_cast<float*>(out_v),
+                                                         static_cast<float*>(out_r), Cx, nruns, c->B);
+    else
+      conv_silu_kernel<float, 1><<<blocks, 256, 0, st>>>(rows, Cx, w, bias, static_cast<float*>(out_v),
+                                                         static_cast<float*>(out_r), Cx, nruns, c->B);
+  }
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
+// y <- gated RMSNorm(y, z) in place over rows [0, rows) (y row stride ldy, z row stride ldz, elements).
+mate_status run_gate_norm(const mate_config* c, void* y, int ldy, const void* z, int ldz, const float* norm_w,
+                          long long nrows, cudaStream_t st) {
+  if (nrows <= 0) return MATE_OK;
+  const int C = c->nh * c->P;
+  const size_t es = elem_size(c);
+  const bool vec = (C * es) % 16 == 0 && (ldy * es) % 16 == 0 && (ldz * es) % 16 == 0 && aligned16(y) && aligned16(z);
+  const int blocks = static_cast<int>(std::min<long long>((nrows + 7) / 8, (long long)device_sms() * 16));
+  trace_begin(MATE_K_GATE_NORM, st);
+  if (c->dtype == MATE_BF16) {
+    auto* yy = static_cast<__nv_bfloat16*>(y);
+    const auto* zz = static_cast<const __nv_bfloat16*>(z);
+    if (vec) gate_rmsnorm_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
+    else gate_rmsnorm_kernel<__nv_bfloat16, 1><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
+  } else {
+    auto* yy = static_cast<float*>(y);
+    const auto* zz = static_cast<const float*>(z);
+    if (vec) gate_rmsnorm_kernel<float, 4><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
+    else gate_rmsnorm_kernel<float, 1><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
+  }
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
 // The chunked host transfers of one mate_forward_host call (null for device-buffer calls).
 struct IoPlan {
   HostIo* io;
@@ -515,6 +585,10 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   if (!aligned16(X) || !aligned16(Out) || !aligned16(ws) || !aligned16(w->W_in) || !aligned16(w->W_out) ||
       !aligned16(w->W_qkv) || !aligned16(w->W_o))
     return MATE_ERR_ARG;
+  const bool extras = c->mamba_extras == 1;
+  if (extras && (w->W_z == nullptr || w->conv_w == nullptr || w->conv_b == nullptr || w->norm_w == nullptr ||
+                 !aligned16(w->W_z) || !aligned16(w->conv_w)))
+    return MATE_ERR_ARG;
   ForwardPlan pl = plan_forward(c, nullptr);
   if (ws_bytes < pl.bytes) return MATE_ERR_WORKSPACE;
   pl = plan_forward(c, ws);
@@ -532,6 +606,7 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   // packed weights: Wi = [W_in; W_qkv] (NI x d), Wo = [W_out | W_o] (d x KO)
   MATE_TRY(copy_block(w->W_in, pl.Wi, NIn, c->d, c->d, 0, 0, es, st));
   MATE_TRY(copy_block(w->W_qkv, pl.Wi, 3 * c->th * c->tp, c->d, c->d, NIn, 0, es, st));
+  if (extras) MATE_TRY(copy_block(w->W_z, pl.Wi, dI, c->d, c->d, pl.zc0, 0, es, st));
   MATE_TRY(copy_block(w->W_out, pl.Wo, c->d, dI, KO, 0, 0, es, st));
   MATE_TRY(copy_block(w->W_o, pl.Wo, c->d, c->th * c->tp, KO, 0, dI, es, st));
   // review tokens, then the projections of the video rows (grid order) and of the review rows
@@ -584,6 +659,22 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   rows.H = c->H;
   rows.W = c->W;
   rows.order = order;
+  if (extras) {
+    // x | B | C through the causal convolution + SiLU, along [review rows; video rows in scan order];
+    // the scan then reads the convolved rows (same row order, row stride Cx)
+    const int Cx = dI + 2 * c->N;
+    MATE_TRY(run_conv(c, rows, Cx, w->conv_w, w->conv_b, pl.XBv, pl.XBr, st));
+    const char* xbv = static_cast<const char*>(pl.XBv);
+    const char* xbr = static_cast<const char*>(pl.XBr);
+    rows.xv = xbv;
+    rows.bv = xbv + (size_t)dI * es;
+    rows.cv = xbv + (size_t)(dI + c->N) * es;
+    rows.xr = xbr;
+    rows.br = xbr + (size_t)dI * es;
+    rows.cr = xbr + (size_t)(dI + c->N) * es;
+    rows.ldxv = rows.ldbv = rows.ldcv = Cx;
+    rows.ldxr = rows.ldbr = rows.ldcr = Cx;
+  }
   // Orders 2 and 3 run time fastest: grid-order rows of one chunk lie in 256 different time planes, and
   // writing each head's 128-byte y piece there costs more than writing y in scan order and moving whole
   // rows back to grid order afterwards (measured on the B200).
@@ -602,6 +693,9 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   } else {
     MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.YO, KO, n, pl.ssd, st, w->A_log_b, w->D_b));
   }
+  // gate and gated RMSNorm of y in place (grid-order rows of YO[:, :dI]), before the out-projection
+  if (extras) MATE_TRY(run_gate_norm(c, pl.YO, KO, static_cast<const char*>(pl.Zv) + (size_t)pl.zc0 * es, NI, w->norm_w,
+                                     Mv, st));
   // TE: window attention on the q | k | v columns of Zv, output into YO[:, dI:]
   const int qc = NIn, ac = c->th * c->tp;
   MATE_TRY(run_tesa(c, pl.Zv, NI, qc, qc + ac, qc + 2 * ac, pl.YO, KO, dI, shifted, st));
@@ -963,6 +1057,8 @@ const char* mate_kernel_name(int kernel) {
     case MATE_K_PROJECT: return "project";
     case MATE_K_SCAN_LOCALITY: return "scan_locality";
     case MATE_K_Y_TO_GRID: return "y_to_grid";
+    case MATE_K_CONV_SILU: return "conv_silu";
+    case MATE_K_GATE_NORM: return "gate_rmsnorm";
   }
   return "unknown";
 }

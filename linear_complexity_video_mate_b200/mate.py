@@ -41,21 +41,28 @@ def weights_to_device(w: Dict, cfg, device="cuda") -> Dict[str, torch.Tensor]:
     """Host weight arrays (numpy / tensors) -> device tensors in the library's dtypes."""
     dt = torch_dtype(cfg)
     out = {}
-    for k in ("W_in", "W_out", "W_qkv", "W_o"):
-        out[k] = torch.as_tensor(w[k]).to(device=device, dtype=dt).contiguous()
-    for k in ("dt_bias", "A_log", "D", "dt_bias_b", "A_log_b", "D_b"):
-        if k in w:   # the last three are the optional backward-scan parameters
+    for k in ("W_in", "W_out", "W_qkv", "W_o", "W_z"):
+        if k in w:   # W_z: the optional gate projection of the full Mamba2 block
+            out[k] = torch.as_tensor(w[k]).to(device=device, dtype=dt).contiguous()
+    for k in ("dt_bias", "A_log", "D", "dt_bias_b", "A_log_b", "D_b", "conv_w", "conv_b", "norm_w"):
+        if k in w:   # optional: the backward-scan parameters, the convolution and the norm weight
             out[k] = torch.as_tensor(w[k]).to(device=device, dtype=torch.float32).contiguous()
     return out
 
 
 class MateBlock:
-    """One MATE block (MA + TE branches) with its weights resident on the GPU and a reusable workspace."""
+    """One MATE block (MA + TE branches) with its weights resident on the GPU and a reusable workspace.
+    Weights W_z, conv_w, conv_b and norm_w, given together, make the MA branch's core a full Mamba2 block
+    (causal convolution + SiLU on x | B | C, SiLU(z) gate, gated RMSNorm)."""
 
     def __init__(self, cfg, weights: Dict[str, torch.Tensor], device="cuda"):
         lib = _lib.load()
         self.cfg = cfg
-        self.ccfg = _lib.make_config(cfg)
+        ext = [k for k in ("W_z", "conv_w", "conv_b", "norm_w") if k in weights]
+        if ext and len(ext) != 4:
+            raise ValueError(f"Mamba2 extras: give W_z, conv_w, conv_b and norm_w together, got {ext}")
+        self.extras = bool(ext)
+        self.ccfg = _lib.make_config(cfg, self.extras)
         _lib.check(lib.mate_check_config(ctypes.byref(self.ccfg)), "mate_check_config")
         self.device = torch.device(device)
         self.dtype = torch_dtype(cfg)
@@ -72,9 +79,15 @@ class MateBlock:
             raise ValueError(f"backward-scan parameters: give dt_bias_b, A_log_b and D_b together, got {bwd}")
         for k in bwd:
             _need(weights[k], torch.float32, cfg.nh, k)
+        if self.extras:
+            nP, Cx = cfg.nh * cfg.P, cfg.nh * cfg.P + 2 * cfg.N
+            _need(weights["W_z"], self.dtype, nP * cfg.d, "W_z")
+            _need(weights["conv_w"], torch.float32, Cx * 4, "conv_w")
+            _need(weights["conv_b"], torch.float32, Cx, "conv_b")
+            _need(weights["norm_w"], torch.float32, nP, "norm_w")
         self.cw = _lib.CWeights(*(weights[k].data_ptr() if k in weights else None for k in
                                   ("W_in", "dt_bias", "A_log", "D", "W_out", "W_qkv", "W_o", "dt_bias_b", "A_log_b",
-                                   "D_b")))
+                                   "D_b", "W_z", "conv_w", "conv_b", "norm_w")))
         self.ws_bytes = lib.mate_workspace_bytes(ctypes.byref(self.ccfg))
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
         self.ws_host = None

@@ -107,3 +107,33 @@ def elementwise_err(a, ref):
     a, ref = np.asarray(a, np.float64), np.asarray(ref, np.float64)
     rms = np.sqrt(np.mean(ref * ref))
     return float((np.abs(a - ref) / np.maximum(np.abs(ref), rms)).max())
+
+
+def bf16_storage_forward_extras(X, w, cfg, layer):
+    """bf16_storage_forward for the block with the Mamba2 extras: besides the block's own storage points,
+    the convolved x | B | C rows, the gate z and the normalised rows are stored in bf16."""
+    from oracle import mamba2_extras as MX
+    order, shifted = layer % 4, layer % 2 == 1
+    nP, N = cfg.nh * cfg.P, cfg.N
+    outs = []
+    for b in range(X.shape[0]):
+        X3 = np.asarray(X[b], np.float64)
+        T, H, W, d = X3.shape
+        Xp = O.rms_permute(X3, order)
+        Rv = _r(O.review_tokens(X3, cfg.R, order))
+        S = np.concatenate([Rv, Xp], axis=0)
+        x, Bm, Cm, delta = O.in_projection(S, w, cfg)
+        xbc = _r(np.concatenate([x.reshape(-1, nP), Bm, Cm], axis=1))
+        xbc = _r(MX.silu(MX.causal_conv(xbc, w["conv_w"], w["conv_b"])))
+        x, Bm, Cm = xbc[:, :nP].reshape(-1, cfg.nh, cfg.P), xbc[:, nP:nP + N], xbc[:, nP + N:]
+        A = -np.exp(np.asarray(w["A_log"], np.float64))
+        y = _r(O.ssd_bidirectional(x, Bm, Cm, delta, A, w["D"], cfg.R).reshape(T * H * W, -1))
+        z = _r(Xp @ np.asarray(w["W_z"], np.float64).T)
+        yn = _r(MX.gated_rmsnorm(y, z, w["norm_w"]))
+        ma = O.rms_unpermute(yn @ np.asarray(w["W_out"], np.float64).T, order, T, H, W)
+        qkv = _r(X3.reshape(-1, d) @ np.asarray(w["W_qkv"], np.float64).T)
+        Oa = _r(O.tesa_attention(qkv.reshape(T, H, W, -1), cfg.th, cfg.tp, (cfg.wt, cfg.wh, cfg.ww),
+                                 (cfg.st, cfg.sh, cfg.sw), shifted))
+        te = (Oa.reshape(-1, cfg.th * cfg.tp) @ np.asarray(w["W_o"], np.float64).T).reshape(T, H, W, d)
+        outs.append(_r(ma + te))
+    return np.stack(outs)

@@ -85,6 +85,19 @@ def test_null_and_misaligned_arguments_are_rejected_before_launch(lib):
     nss = lib.mate_ssd_workspace_bytes(cp, 256)
     assert lib.ssd_scan_bidir(fake, fake, fake, fake, fake, fake, fake, 256, fake, cp, fake, nss - 1, None) == \
         _lib.MATE_ERR_WORKSPACE
+    # Mamba2 extras: the flag is 0 or 1, and with it the four extra weights are required
+    ce = _cfg()
+    ce.mamba_extras = 2
+    assert lib.mate_check_config(ctypes.byref(ce)) == _lib.MATE_ERR_ARG
+    ce.mamba_extras = 1
+    assert lib.mate_check_config(ctypes.byref(ce)) == _lib.MATE_OK
+    assert lib.mate_workspace_bytes(ctypes.byref(ce)) > lib.mate_workspace_bytes(cp)
+    assert lib.mate_forward(fake, ctypes.byref(w), 0, fake, ctypes.byref(ce), fake, 1 << 40, None) == \
+        _lib.MATE_ERR_ARG
+    we = _lib.CWeights(*([1 << 20] * 14))
+    we.conv_w = (1 << 20) + 4    # the taps are read as 16-byte vectors
+    assert lib.mate_forward(fake, ctypes.byref(we), 0, fake, ctypes.byref(ce), fake, 1 << 40, None) == \
+        _lib.MATE_ERR_ARG
     # separate backward-scan parameters: all three or none
     wp = _lib.CWeights(*([1 << 20] * 8))
     assert lib.mate_forward(fake, ctypes.byref(wp), 0, fake, cp, fake, 1 << 40, None) == _lib.MATE_ERR_ARG
@@ -122,8 +135,8 @@ def test_noalloc_scan_rejects_problems_beyond_its_scratch(lib):
 
 
 def test_kernel_names_are_distinct(lib):
-    names = [lib.mate_kernel_name(k).decode() for k in range(17)]
-    assert len(set(names)) == 17 and "unknown" not in names, names
+    names = [lib.mate_kernel_name(k).decode() for k in range(19)]
+    assert len(set(names)) == 19 and "unknown" not in names, names
     assert lib.mate_kernel_name(99).decode() == "unknown"
     assert lib.mate_trace_start(-1) == _lib.MATE_ERR_ARG
 

@@ -61,7 +61,7 @@ def _pd_scan(cfg, args, bwd):
                                dev(D, f32), *(dev(a, f32) for a in bwd), cfg.R, cfg)
 
 
-def video_rows(cfg, stride=8):
+def video_rows(cfg, stride=16):
     """Every stride-th video row plus the last one: the rows whose oracle values are kept on disk (the GPU
     computes all of them; the stored references stay small)."""
     return np.unique(np.append(np.arange(0, cfg.n, stride), cfg.n - 1))
@@ -75,14 +75,14 @@ def scan_reference(name, long_memory):
     cfg = all_test_configs()[name]
     args, bwd = _scan_args(cfg, long_memory)
     rows = video_rows(cfg)
-    key = f"pd-ssd-{name}-{long_memory}-every8"
+    key = f"pd-ssd-{name}-{long_memory}-every16"
     ref = oracle_cached(key, lambda: _pd_oracle(cfg, *args, *bwd)[:, rows], PD_SRC)
     floor = 0.0
     if cfg.dtype == "bf16":
         x, Bm, Cm, dt, dt_bias, A_log, D = args
         for tag, params in (("f", (dt_bias, A_log, D)), ("b", bwd)):
             a2 = (x, Bm, Cm, dt) + tuple(params)
-            k2 = f"pd-ssd-{name}-{long_memory}-every8-shared{tag}"
+            k2 = f"pd-ssd-{name}-{long_memory}-every16-shared{tag}"
             # only the scalar floor is kept on disk
             fl = lambda a2=a2, k2=k2: np.array([_ssd_floor(cfg, a2, _ssd_oracle(cfg, *a2)[:, rows], k2, rows=rows)])
             floor = max(floor, float(oracle_cached(f"pd-floor-{k2}", fl, PD_SRC)[0]))
@@ -126,8 +126,8 @@ def block_reference(name, layer):
     cfg = all_test_configs()[name]
     w = dict(mi.make_inputs(cfg))
     w["dt_bias_b"], w["A_log_b"], w["D_b"] = backward_params(cfg.nh, 29, w["dt_bias"], (0.0, 1.0))
-    rows = np.unique(np.append(np.arange(0, cfg.B * cfg.n, 8), cfg.B * cfg.n - 1))
-    key = f"pd-mate-{name}-{layer}-every8"
+    rows = np.unique(np.append(np.arange(0, cfg.B * cfg.n, 16), cfg.B * cfg.n - 1))
+    key = f"pd-mate-{name}-{layer}-every16"
     ref = oracle_cached(key, lambda: PD.mate_forward_per_direction(w["X"], w, cfg, layer).reshape(
         cfg.B * cfg.n, cfg.d)[rows], PD_SRC)
     floor = 0.0
