@@ -113,8 +113,8 @@ def measured_peaks():
 # DRAM bytes per launch measured with ncu (dram__bytes_read.sum + dram__bytes_write.sum), scaled to the
 # bench workload as the profile summary explains; valid only while the kernel source is the one captured.
 MEASURED_TRAFFIC = {
-    "in_projection": {"bytes": 2.639e9, "source": "linear_complexity_video_mate_b200/csrc/gemm_bf16.cuh",
-                      "sha1": "f7a250cbda08da22dcec652ea86f7ef23fe682ae",
+    "in_projection": {"bytes": 2.640e9, "source": "linear_complexity_video_mate_b200/csrc/gemm_bf16.cuh",
+                      "sha1": "5a3dbaeadb0ece8caaabc8703f84db7e67ad95b9",
                       "profile": "profiles/gemm_bf16_pair_in_projection_bf16_64x32x32.md",
                       "workload": "bf16_256x32x32"},
 }
@@ -148,6 +148,56 @@ def kernel_work(cfg):
         "out_projection": ("tensor", 2.0 * rows * KO * cfg.d, "TFLOP/s"),
         "tesa": ("tensor", 4.0 * rows * cfg.th * win * cfg.tp, "TFLOP/s"),
     }
+
+
+def extras_weights(cfg, seed):
+    """Random-init weights of the rest of a Mamba2 block: gate projection N(0, 1/d), convolution taps and
+    bias U(-1/2, 1/2), norm weight 1 + N(0, 0.1^2)."""
+    rng = np.random.default_rng(seed)
+    nP, Cx = cfg.nh * cfg.P, cfg.nh * cfg.P + 2 * cfg.N
+    return dict(W_z=(rng.standard_normal((nP, cfg.d)) / np.sqrt(cfg.d)).astype(np.float32),
+                conv_w=rng.uniform(-0.5, 0.5, (Cx, 4)).astype(np.float32),
+                conv_b=rng.uniform(-0.5, 0.5, Cx).astype(np.float32),
+                norm_w=(1.0 + 0.1 * rng.standard_normal(nP)).astype(np.float32))
+
+
+def measure_extras(M, torch, cfg, w, X, out, stream, base_ms, hbm_peak, steps=20):
+    """The block with the full Mamba2 core (convolution + SiLU, gate, gated RMSNorm), timed after the
+    headline region: ms per block and the two added kernels against the HBM roofline (algorithmic bytes:
+    the convolution reads and writes the x | B | C rows of the video and review rows, the gated norm reads
+    y and z and writes y)."""
+    we = dict(w)
+    we.update(extras_weights(cfg, 4242))
+    blk = M.MateBlock(cfg, M.weights_to_device(we, cfg))
+    for s in range(3):
+        blk.forward(X, s, out)
+    nl = M.MateBlock.last_launch_count()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    trace = M.KernelTrace(nl * steps).start()
+    e0.record(stream)
+    for s in range(steps):
+        blk.forward(X, s % 4, out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    trace.stop()
+    ms = e0.elapsed_time(e1) / steps
+    per = {}
+    for name, kms in trace.read():
+        a = per.setdefault(name, [0, 0.0])
+        a[0] += 1
+        a[1] += kms
+    es = 2 if cfg.dtype == "bf16" else 4
+    nP, Cx = cfg.nh * cfg.P, cfg.nh * cfg.P + 2 * cfg.N
+    nbytes = {"conv_silu": 2.0 * cfg.B * (cfg.n + cfg.R) * Cx * es, "gate_rmsnorm": 3.0 * cfg.B * cfg.n * nP * es}
+    res = {"ms_per_block": ms, "added_ms": ms - base_ms, "steps": steps}
+    for k, b in nbytes.items():
+        if k in per:
+            kms = per[k][1] / per[k][0]
+            gbs = b / (kms * 1e-3) / 1e9
+            res[k] = {"ms_per_launch": kms, "algorithmic_bytes": b, "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
+    del blk
+    return res
 
 
 def oracle_sample_cfg(cfg, frames):
@@ -227,6 +277,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--oracle-frames", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the full-Mamba2-block side measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -328,6 +379,9 @@ def main():
     locality["pairs"] = npairs
     locality["ms_all_maps"] = l0.elapsed_time(l1)
 
+    # side measurement, outside the headline region: the block with the rest of the Mamba2 block
+    extras = None if args.no_extras else measure_extras(M, torch, cfg, w, X, out, stream, ms, hbm_peak)
+
     tokens_per_step = cfg.B * cfg.n
     value = job_value(tokens_per_step, world, ms)
     fl = flops_per_block(cfg)
@@ -353,6 +407,7 @@ def main():
                 "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms, "api": "mate_forward_host"},
         "gpu_launches": len(records),
         "scan_locality": locality,
+        "mamba_extras": extras,
         "clocks": clocks,
         "device_status": status,
     }
