@@ -178,6 +178,26 @@ MATE_API mate_status ssd_scan_bidir_pd(const void* x, const void* Bm, const void
                                        int prefix_len, void* y, const mate_config* cfg, void* ws, size_t ws_bytes,
                                        mate_stream_t stream);
 
+/*
+ * Backward pass of ssd_scan_bidir (training): given the output gradient dy [B, T*H*W, nh*P] of the video
+ * rows, the gradients of every input.  The adjoint follows from the forward recurrence by the chain rule
+ * (the pages give only the forward computation):
+ *     dx, dB, dC  [B, L, nh*P] / [B, L, N]   same layout as x, Bm, Cm (prefix rows included)
+ *     ddt         [B, L, nh]  gradient of the raw step input dt (delta = softplus(dt + dt_bias))
+ *     ddt_bias, dA_log, dD  [nh]  summed over samples and rows
+ * fp32 blocks only (cfg->dtype = MATE_F32; bf16 gives MATE_ERR_UNSUPPORTED); a CUDA-core kernel that
+ * keeps every state of one direction in the workspace, for small problems.  ws: at least
+ * mate_ssd_backward_workspace_bytes(cfg, prefix_len) bytes.  All gradient outputs are written in full
+ * (the summed ones are zeroed first on `stream`).
+ */
+MATE_API size_t mate_ssd_backward_workspace_bytes(const mate_config* cfg, int prefix_len);
+MATE_API mate_status ssd_scan_bidir_backward(const void* x, const void* Bm, const void* Cm, const float* dt,
+                                             const float* dt_bias, const float* A_log, const float* D,
+                                             int prefix_len, const void* dy, void* dx, void* dB, void* dC,
+                                             float* ddt, float* ddt_bias, float* dA_log, float* dD,
+                                             const mate_config* cfg, void* ws, size_t ws_bytes,
+                                             mate_stream_t stream);
+
 /* Size of the fixed device scratch buffer behind ssd_scan_bidir_noalloc: 32 MiB. */
 #define MATE_SSD_NOALLOC_SCRATCH_BYTES (32u << 20)
 
@@ -311,7 +331,8 @@ typedef enum {
   MATE_K_SCAN_LOCALITY = 15,   /* mate_scan_locality */
   MATE_K_Y_TO_GRID = 16,       /* scan-order y rows back to grid order (time-fastest scan orders) */
   MATE_K_CONV_SILU = 17,       /* causal depthwise convolution + SiLU on x | B | C (mamba_extras) */
-  MATE_K_GATE_NORM = 18        /* y silu(z) and gated RMSNorm (mamba_extras) */
+  MATE_K_GATE_NORM = 18,       /* y silu(z) and gated RMSNorm (mamba_extras) */
+  MATE_K_SSD_BACKWARD = 19     /* ssd_scan_bidir_backward (fp32) */
 } mate_kernel;
 
 typedef struct {

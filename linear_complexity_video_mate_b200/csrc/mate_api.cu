@@ -20,6 +20,7 @@
 #include "tesa_bf16.cuh"
 #include "locality.cuh"
 #include "mamba_extras.cuh"
+#include "ssd_backward.cuh"
 
 using namespace mate;
 
@@ -851,6 +852,65 @@ mate_status ssd_scan_bidir_pd(const void* x, const void* Bm, const void* Cm, con
                    stream);
 }
 
+size_t mate_ssd_backward_workspace_bytes(const mate_config* cfg, int prefix_len) {
+  if (check_config(cfg) != MATE_OK || prefix_len < 0) return 0;
+  const long long L = (long long)cfg->T * cfg->H * cfg->W + prefix_len;
+  return (size_t)cfg->B * cfg->nh * L * cfg->P * cfg->N * sizeof(float) + 256;
+}
+
+mate_status ssd_scan_bidir_backward(const void* x, const void* Bm, const void* Cm, const float* dt,
+                                    const float* dt_bias, const float* A_log, const float* D, int prefix_len,
+                                    const void* dy, void* dx, void* dB, void* dC, float* ddt, float* ddt_bias,
+                                    float* dA_log, float* dD, const mate_config* cfg, void* ws, size_t ws_bytes,
+                                    mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (x == nullptr || Bm == nullptr || Cm == nullptr || dt == nullptr || dt_bias == nullptr || A_log == nullptr ||
+      D == nullptr || dy == nullptr || dx == nullptr || dB == nullptr || dC == nullptr || ddt == nullptr ||
+      ddt_bias == nullptr || dA_log == nullptr || dD == nullptr || ws == nullptr || prefix_len < 0)
+    return MATE_ERR_ARG;
+  if (cfg->dtype != MATE_F32) return MATE_ERR_UNSUPPORTED;
+  if (ws_bytes < mate_ssd_backward_workspace_bytes(cfg, prefix_len)) return MATE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  const long long n = (long long)cfg->T * cfg->H * cfg->W;
+  const long long L = n + prefix_len;
+  if (!cuda_ok(cudaMemsetAsync(dB, 0, (size_t)cfg->B * L * cfg->N * sizeof(float), st)) ||
+      !cuda_ok(cudaMemsetAsync(dC, 0, (size_t)cfg->B * L * cfg->N * sizeof(float), st)) ||
+      !cuda_ok(cudaMemsetAsync(ddt_bias, 0, (size_t)cfg->nh * sizeof(float), st)) ||
+      !cuda_ok(cudaMemsetAsync(dA_log, 0, (size_t)cfg->nh * sizeof(float), st)) ||
+      !cuda_ok(cudaMemsetAsync(dD, 0, (size_t)cfg->nh * sizeof(float), st)))
+    return MATE_ERR_CUDA;
+  SeqRows rows;
+  rows.xv = rows.xr = x;
+  rows.bv = rows.br = Bm;
+  rows.cv = rows.cr = Cm;
+  rows.dv = rows.dr = nullptr;
+  rows.ldxv = rows.ldxr = cfg->nh * cfg->P;
+  rows.ldbv = rows.ldbr = rows.ldcv = rows.ldcr = cfg->N;
+  rows.lddv = rows.lddr = cfg->nh;
+  rows.db_off = 0;
+  rows.v_bstride = L;
+  rows.v_off = prefix_len;
+  rows.r_bstride = L;
+  rows.r_off = 0;
+  rows.n = static_cast<int>(n);
+  rows.R = prefix_len;
+  rows.T = cfg->T;
+  rows.H = cfg->H;
+  rows.W = cfg->W;
+  rows.order = -1;
+  rows.y_order = -1;
+  const int PN = cfg->P * cfg->N;
+  const int threads = (PN + 31) / 32 * 32;
+  const size_t smem = (size_t)(4 * PN + 3 * cfg->P) * sizeof(float);
+  trace_begin(MATE_K_SSD_BACKWARD, st);
+  ssd_backward_f32_kernel<<<dim3(cfg->nh, cfg->B), threads, smem, st>>>(
+      rows, dt, cfg->nh, dt_bias, A_log, D, cfg->P, cfg->N, static_cast<const float*>(dy), static_cast<float*>(dx),
+      static_cast<float*>(dB), static_cast<float*>(dC), ddt, ddt_bias, dA_log, dD, static_cast<float*>(ws));
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
 // Fixed scratch behind ssd_scan_bidir_noalloc.  In host code this name is only a stand-in for the
 // device symbol; its device address comes from cudaGetSymbolAddress, once per device.
 static __device__ __align__(256) unsigned char g_ssd_noalloc_scratch[MATE_SSD_NOALLOC_SCRATCH_BYTES];
@@ -1059,6 +1119,7 @@ const char* mate_kernel_name(int kernel) {
     case MATE_K_Y_TO_GRID: return "y_to_grid";
     case MATE_K_CONV_SILU: return "conv_silu";
     case MATE_K_GATE_NORM: return "gate_rmsnorm";
+    case MATE_K_SSD_BACKWARD: return "ssd_backward_f32";
   }
   return "unknown";
 }

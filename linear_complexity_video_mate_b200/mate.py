@@ -190,6 +190,24 @@ def ssd_scan_bidir_pd(x, Bm, Cm, dt, dt_bias, A_log, D, dt_bias_b, A_log_b, D_b,
     return out
 
 
+def ssd_scan_bidir_backward(x, Bm, Cm, dt, dt_bias, A_log, D, dy, prefix_len: int, cfg, ws=None, stream=None):
+    """Gradients of ssd_scan_bidir (fp32 blocks) given the video rows' output gradient dy [B, T*H*W, nh*P]:
+    a dict with dx, dB, dC (layouts of x, Bm, Cm), ddt (layout of dt) and ddt_bias, dA_log, dD [nh]."""
+    lib = _lib.load()
+    c = _cfg(cfg)
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g = dict(dx=torch.empty_like(x), dB=torch.empty_like(Bm), dC=torch.empty_like(Cm), ddt=torch.empty_like(dt),
+             ddt_bias=torch.empty(cfg.nh, **f32), dA_log=torch.empty(cfg.nh, **f32), dD=torch.empty(cfg.nh, **f32))
+    nb = lib.mate_ssd_backward_workspace_bytes(ctypes.byref(c), int(prefix_len))
+    if ws is None or ws.numel() < nb:
+        ws = torch.empty(nb, dtype=torch.uint8, device=x.device)
+    st = lib.ssd_scan_bidir_backward(_p(x), _p(Bm), _p(Cm), _p(dt), _p(dt_bias), _p(A_log), _p(D), int(prefix_len),
+                                     _p(dy), _p(g["dx"]), _p(g["dB"]), _p(g["dC"]), _p(g["ddt"]), _p(g["ddt_bias"]),
+                                     _p(g["dA_log"]), _p(g["dD"]), ctypes.byref(c), _p(ws), ws.numel(), _s(stream))
+    _lib.check(st, "ssd_scan_bidir_backward")
+    return g
+
+
 def ssd_scan_bidir_noalloc(x, Bm, Cm, dt, dt_bias, A_log, D, prefix_len: int, cfg, out, stream=None):
     """ssd_scan_bidir on the library's fixed device scratch, for callers that may not allocate device memory.
     Nothing is allocated here either: the caller passes the output `out` [B, T*H*W, nh*P]."""

@@ -98,6 +98,18 @@ def test_null_and_misaligned_arguments_are_rejected_before_launch(lib):
     we.conv_w = (1 << 20) + 4    # the taps are read as 16-byte vectors
     assert lib.mate_forward(fake, ctypes.byref(we), 0, fake, ctypes.byref(ce), fake, 1 << 40, None) == \
         _lib.MATE_ERR_ARG
+    # backward scan: fp32 blocks only, every pointer required, workspace checked
+    nbw = lib.mate_ssd_backward_workspace_bytes(cp, 256)
+    assert nbw > 0
+    bargs = [fake] * 7 + [256] + [fake] * 8
+    assert lib.ssd_scan_bidir_backward(*bargs, cp, fake, nbw, None) == _lib.MATE_ERR_UNSUPPORTED   # bf16 config
+    cf = _lib.make_config(mi.CONFIGS["tiny_f32_4x8x8"])
+    nbf = lib.mate_ssd_backward_workspace_bytes(ctypes.byref(cf), 256)
+    assert nbf > 0
+    assert lib.ssd_scan_bidir_backward(*bargs, ctypes.byref(cf), fake, nbf - 1, None) == _lib.MATE_ERR_WORKSPACE
+    nullargs = list(bargs)
+    nullargs[9] = None
+    assert lib.ssd_scan_bidir_backward(*nullargs, ctypes.byref(cf), fake, nbf, None) == _lib.MATE_ERR_ARG
     # separate backward-scan parameters: all three or none
     wp = _lib.CWeights(*([1 << 20] * 8))
     assert lib.mate_forward(fake, ctypes.byref(wp), 0, fake, cp, fake, 1 << 40, None) == _lib.MATE_ERR_ARG
@@ -135,8 +147,8 @@ def test_noalloc_scan_rejects_problems_beyond_its_scratch(lib):
 
 
 def test_kernel_names_are_distinct(lib):
-    names = [lib.mate_kernel_name(k).decode() for k in range(19)]
-    assert len(set(names)) == 19 and "unknown" not in names, names
+    names = [lib.mate_kernel_name(k).decode() for k in range(20)]
+    assert len(set(names)) == 20 and "unknown" not in names, names
     assert lib.mate_kernel_name(99).decode() == "unknown"
     assert lib.mate_trace_start(-1) == _lib.MATE_ERR_ARG
 
