@@ -14,8 +14,8 @@ import torch
 from . import _lib
 
 __all__ = ["MateBlock", "rms_permute", "rms_unpermute", "review_pool", "ssd_scan_bidir", "ssd_scan_bidir_pd",
-           "tesa_forward",
-           "project_bf16", "device_status", "torch_dtype", "weights_to_device"]
+           "ssd_scan_bidir_noalloc", "ssd_scan_bidir_backward", "tesa_forward", "project_bf16", "device_status",
+           "torch_dtype", "weights_to_device", "scan_locality", "KernelTrace"]
 
 
 def torch_dtype(cfg) -> torch.dtype:
@@ -195,6 +195,12 @@ def ssd_scan_bidir_backward(x, Bm, Cm, dt, dt_bias, A_log, D, dy, prefix_len: in
     a dict with dx, dB, dC (layouts of x, Bm, Cm), ddt (layout of dt) and ddt_bias, dA_log, dD [nh]."""
     lib = _lib.load()
     c = _cfg(cfg)
+    L = cfg.n + int(prefix_len)
+    for t, nm, numel in ((x, "x", cfg.B * L * cfg.nh * cfg.P), (Bm, "Bm", cfg.B * L * cfg.N),
+                         (Cm, "Cm", cfg.B * L * cfg.N), (dt, "dt", cfg.B * L * cfg.nh),
+                         (dy, "dy", cfg.B * cfg.n * cfg.nh * cfg.P), (dt_bias, "dt_bias", cfg.nh),
+                         (A_log, "A_log", cfg.nh), (D, "D", cfg.nh)):
+        _need(t, torch.float32, numel, nm)
     f32 = dict(dtype=torch.float32, device=x.device)
     g = dict(dx=torch.empty_like(x), dB=torch.empty_like(Bm), dC=torch.empty_like(Cm), ddt=torch.empty_like(dt),
              ddt_bias=torch.empty(cfg.nh, **f32), dA_log=torch.empty(cfg.nh, **f32), dD=torch.empty(cfg.nh, **f32))
