@@ -161,14 +161,10 @@ def extras_weights(cfg, seed):
                 norm_w=(1.0 + 0.1 * rng.standard_normal(nP)).astype(np.float32))
 
 
-def measure_extras(M, torch, cfg, w, X, out, stream, base_ms, hbm_peak, steps=20):
-    """The block with the full Mamba2 core (convolution + SiLU, gate, gated RMSNorm), timed after the
-    headline region: ms per block and the two added kernels against the HBM roofline (algorithmic bytes:
-    the convolution reads and writes the x | B | C rows of the video and review rows, the gated norm reads
-    y and z and writes y)."""
-    we = dict(w)
-    we.update(extras_weights(cfg, 4242))
-    blk = M.MateBlock(cfg, M.weights_to_device(we, cfg))
+def time_block_variant(M, torch, cfg, wv, X, out, stream, steps):
+    """ms per block of a MateBlock built from weights wv (3 warm-up forwards, `steps` timed ones cycling
+    the layers) and per-kernel [launches, total ms] from the library trace."""
+    blk = M.MateBlock(cfg, M.weights_to_device(wv, cfg))
     for s in range(3):
         blk.forward(X, s, out)
     nl = M.MateBlock.last_launch_count()
@@ -181,12 +177,39 @@ def measure_extras(M, torch, cfg, w, X, out, stream, base_ms, hbm_peak, steps=20
     e1.record(stream)
     torch.cuda.synchronize()
     trace.stop()
-    ms = e0.elapsed_time(e1) / steps
     per = {}
     for name, kms in trace.read():
         a = per.setdefault(name, [0, 0.0])
         a[0] += 1
         a[1] += kms
+    del blk
+    return e0.elapsed_time(e1) / steps, per
+
+
+def measure_per_direction(M, torch, cfg, w, X, out, stream, base_ms, steps=20):
+    """The block with separate backward-scan parameters (dt_bias_b, A_log_b, D_b), timed after the
+    headline region: ms per block and the scan kernels' times."""
+    rng = np.random.default_rng(4343)
+    wp = dict(w)
+    wp["dt_bias_b"] = (np.asarray(w["dt_bias"], np.float64) + rng.uniform(-1.0, 1.0, cfg.nh)).astype(np.float32)
+    wp["A_log_b"] = rng.uniform(0.0, 1.0, cfg.nh).astype(np.float32)
+    wp["D_b"] = rng.standard_normal(cfg.nh).astype(np.float32)
+    ms, per = time_block_variant(M, torch, cfg, wp, X, out, stream, steps)
+    res = {"ms_per_block": ms, "added_ms": ms - base_ms, "steps": steps}
+    for k in ("in_projection", "ssd_state", "ssd_carry", "ssd_output"):
+        if k in per:
+            res[k + "_ms"] = per[k][1] / per[k][0]
+    return res
+
+
+def measure_extras(M, torch, cfg, w, X, out, stream, base_ms, hbm_peak, steps=20):
+    """The block with the full Mamba2 core (convolution + SiLU, gate, gated RMSNorm), timed after the
+    headline region: ms per block and the two added kernels against the HBM roofline (algorithmic bytes:
+    the convolution reads and writes the x | B | C rows of the video and review rows, the gated norm reads
+    y and z and writes y)."""
+    we = dict(w)
+    we.update(extras_weights(cfg, 4242))
+    ms, per = time_block_variant(M, torch, cfg, we, X, out, stream, steps)
     es = 2 if cfg.dtype == "bf16" else 4
     nP, Cx = cfg.nh * cfg.P, cfg.nh * cfg.P + 2 * cfg.N
     nbytes = {"conv_silu": 2.0 * cfg.B * (cfg.n + cfg.R) * Cx * es, "gate_rmsnorm": 3.0 * cfg.B * cfg.n * nP * es}
@@ -196,7 +219,6 @@ def measure_extras(M, torch, cfg, w, X, out, stream, base_ms, hbm_peak, steps=20
             kms = per[k][1] / per[k][0]
             gbs = b / (kms * 1e-3) / 1e9
             res[k] = {"ms_per_launch": kms, "algorithmic_bytes": b, "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
-    del blk
     return res
 
 
@@ -379,8 +401,18 @@ def main():
     locality["pairs"] = npairs
     locality["ms_all_maps"] = l0.elapsed_time(l1)
 
-    # side measurement, outside the headline region: the block with the rest of the Mamba2 block
-    extras = None if args.no_extras else measure_extras(M, torch, cfg, w, X, out, stream, ms, hbm_peak)
+    # side measurements, outside the headline region: the block with the rest of the Mamba2 block, and with
+    # separate backward-scan parameters; a failure is reported in the line instead of ending the run
+    extras = per_direction = None
+    if not args.no_extras:
+        try:
+            extras = measure_extras(M, torch, cfg, w, X, out, stream, ms, hbm_peak)
+        except Exception as e:  # noqa: BLE001
+            extras = {"error": f"{type(e).__name__}: {e}"}
+        try:
+            per_direction = measure_per_direction(M, torch, cfg, w, X, out, stream, ms)
+        except Exception as e:  # noqa: BLE001
+            per_direction = {"error": f"{type(e).__name__}: {e}"}
 
     tokens_per_step = cfg.B * cfg.n
     value = job_value(tokens_per_step, world, ms)
@@ -408,6 +440,7 @@ def main():
         "gpu_launches": len(records),
         "scan_locality": locality,
         "mamba_extras": extras,
+        "per_direction_scan": per_direction,
         "clocks": clocks,
         "device_status": status,
     }
