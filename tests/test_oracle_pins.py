@@ -573,3 +573,79 @@ def test_extras_block_is_sum_of_branches():
     ma = np.stack([MX.ma_branch_extras(w["X"][0], w, cfg, 1)])
     te = O.mate_forward(w["X"], dict(w, W_out=np.zeros_like(w["W_out"])), cfg, 1)
     np.testing.assert_allclose(full, ma + te, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ DiT block around MATE (adaLN-Zero)
+
+from oracle import dit_block as DB  # noqa: E402
+
+
+def test_layer_norm_closed_form_and_moments():
+    np.testing.assert_allclose(DB.layer_norm(np.array([[3.0, 5.0]]), eps=0.0), [[-1.0, 1.0]], rtol=1e-15)
+    rng = np.random.default_rng(30)
+    y = DB.layer_norm(3.0 + 2.0 * rng.standard_normal((7, 64)), eps=0.0)
+    np.testing.assert_allclose(y.mean(axis=1), 0.0, atol=1e-13)
+    np.testing.assert_allclose(y.var(axis=1), 1.0, rtol=1e-12)
+
+
+def test_gelu_tanh_identity_and_error_bound_against_erf_gelu():
+    v = np.linspace(-6, 6, 241)
+    np.testing.assert_allclose(DB.gelu_tanh(v) - DB.gelu_tanh(-v), v, rtol=0, atol=1e-12)
+    exact = np.array([0.5 * t * (1.0 + math.erf(t / math.sqrt(2.0))) for t in v])
+    assert np.abs(DB.gelu_tanh(v) - exact).max() < 1e-3     # the tanh form's published accuracy
+
+
+def _dit_weights(cfg, dc, seed, zero_ada=False):
+    rng = np.random.default_rng(seed)
+    w = dict(make_inputs(cfg))
+    d = cfg.d
+    w.update(W_ada=np.zeros((6 * d, dc)) if zero_ada else rng.standard_normal((6 * d, dc)) / math.sqrt(dc),
+             b_ada=np.zeros(6 * d) if zero_ada else 0.1 * rng.standard_normal(6 * d),
+             W1=rng.standard_normal((4 * d, d)) / math.sqrt(d), b1=0.1 * rng.standard_normal(4 * d),
+             W2=rng.standard_normal((d, 4 * d)) / math.sqrt(4 * d), b2=0.1 * rng.standard_normal(d))
+    c = rng.standard_normal((cfg.B, dc))
+    return w, c
+
+
+def test_dit_block_with_zero_modulation_is_the_identity():
+    """adaLN-Zero: zero modulation weights give zero gates, so the block passes X through unchanged."""
+    cfg = _small_cfg()
+    w, c = _dit_weights(cfg, 8, 31, zero_ada=True)
+    np.testing.assert_array_equal(DB.dit_block(w["X"], c, w, cfg, 1), np.asarray(w["X"], np.float64))
+
+
+def test_dit_block_residual_structure():
+    """Gate_a = 1 with no shift or scale and gate_m = 0 leave X + MATE(LN(X)); a zero second MLP layer with
+    bias beta and gate_m = 1 then adds beta to every token."""
+    cfg = _small_cfg()
+    d = cfg.d
+    w, c = _dit_weights(cfg, 8, 32)
+    w["W_ada"] = np.zeros_like(w["W_ada"])
+    b = np.zeros(6 * d)
+    b[2 * d:3 * d] = 1.0                         # gate_a
+    w["b_ada"] = b
+    X = np.asarray(w["X"], np.float64)
+    ln = DB.layer_norm(X.reshape(-1, d)).reshape(X.shape)
+    want = X + O.mate_forward(ln, w, cfg, 2)
+    np.testing.assert_allclose(DB.dit_block(X, c, w, cfg, 2), want, rtol=1e-12, atol=1e-12)
+    b[5 * d:6 * d] = 1.0                         # gate_m
+    beta = np.linspace(-1, 1, d)
+    w2 = dict(w, b_ada=b, W2=np.zeros_like(w["W2"]), b2=beta)
+    np.testing.assert_allclose(DB.dit_block(X, c, w2, cfg, 2), want + beta, rtol=1e-12, atol=1e-12)
+
+
+def test_dit_block_modulation_enters_as_scale_and_shift():
+    """scale_a = -1 and shift_a = s turn the mixer input into the constant token s: the mixer then sees a
+    spatially constant input, and the result depends on X only through the residual and the MLP path."""
+    cfg = _small_cfg()
+    d = cfg.d
+    w, c = _dit_weights(cfg, 8, 33)
+    w["W_ada"] = np.zeros_like(w["W_ada"])
+    b = np.zeros(6 * d)
+    s = np.linspace(-0.5, 0.5, d)
+    b[0:d], b[d:2 * d], b[2 * d:3 * d] = s, -1.0, 1.0
+    w["b_ada"] = b
+    X = np.asarray(w["X"], np.float64)
+    const = np.broadcast_to(s, X.shape).copy()
+    want = X + O.mate_forward(const, w, cfg, 0)
+    np.testing.assert_allclose(DB.dit_block(X, c, w, cfg, 0), want, rtol=1e-12, atol=1e-12)
