@@ -188,7 +188,9 @@ MATE_API mate_status ssd_scan_bidir_pd(const void* x, const void* Bm, const void
  * fp32 blocks only (cfg->dtype = MATE_F32; bf16 gives MATE_ERR_UNSUPPORTED); a CUDA-core kernel that
  * keeps every state of one direction in the workspace, for small problems.  ws: at least
  * mate_ssd_backward_workspace_bytes(cfg, prefix_len) bytes.  All gradient outputs are written in full
- * (the summed ones are zeroed first on `stream`).
+ * (the summed ones are zeroed first on `stream`).  dB, dC, ddt_bias, dA_log and dD are sums over heads or
+ * rows accumulated with float atomics, so their last bits may differ from run to run; dx and ddt are
+ * reproducible.
  */
 MATE_API size_t mate_ssd_backward_workspace_bytes(const mate_config* cfg, int prefix_len);
 MATE_API mate_status ssd_scan_bidir_backward(const void* x, const void* Bm, const void* Cm, const float* dt,
