@@ -162,3 +162,21 @@ def test_scan_locality_argument_checks(lib):
     assert lib.mate_scan_locality(64, 48, 48, 5, 64, None) == _lib.MATE_ERR_UNSUPPORTED   # 48 is not a power of two
     assert lib.mate_scan_locality(12, 8, 8, 5, 64, None) == _lib.MATE_ERR_UNSUPPORTED     # 8 does not divide 12
     assert lib.mate_scan_locality(8, 8, 4, 5, 64, None) == _lib.MATE_ERR_UNSUPPORTED      # H != W
+
+
+def test_plain_c_consumer_compiles_links_and_validates(tmp_path):
+    """include/mate.h compiles as C99 and libmate.so links into a plain C program whose host-side checks
+    answer as the header states (tests/c_abi_check.c; no device needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.dirname(_lib.LIB_PATH)
+    exe = str(tmp_path / "c_abi_check")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                    os.path.join(root, "tests", "c_abi_check.c"), "-L", pkg, "-lmate", f"-Wl,-rpath,{pkg}",
+                    "-o", exe], check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.startswith("ok"), (r.returncode, r.stdout, r.stderr)
