@@ -106,6 +106,15 @@ typedef struct {
   const float* norm_w;    /* [nh*P]   gated RMSNorm weight                                           */
 } mate_weights;
 
+/*
+ * Self-test of the timeout report (no counterpart in the pages).  Launches one thread that waits on a
+ * device barrier nothing completes, polling at most max_polls times (1 <= max_polls <= 65536), after
+ * which it records a timeout in the device status word and returns, as every bounded wait of the library
+ * does when it runs out.  The next mate_device_status on the stream then returns MATE_ERR_TIMEOUT and
+ * clears the word.  MATE_ERR_ARG if max_polls is out of range.
+ */
+MATE_API mate_status mate_selftest_wait_timeout(unsigned int max_polls, mate_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 MATE_API const char* mate_status_str(mate_status s);
 
@@ -334,7 +343,8 @@ typedef enum {
   MATE_K_Y_TO_GRID = 16,       /* scan-order y rows back to grid order (time-fastest scan orders) */
   MATE_K_CONV_SILU = 17,       /* causal depthwise convolution + SiLU on x | B | C (mamba_extras) */
   MATE_K_GATE_NORM = 18,       /* y silu(z) and gated RMSNorm (mamba_extras) */
-  MATE_K_SSD_BACKWARD = 19     /* ssd_scan_bidir_backward (fp32) */
+  MATE_K_SSD_BACKWARD = 19,    /* ssd_scan_bidir_backward (fp32) */
+  MATE_K_SELFTEST = 20         /* mate_selftest_wait_timeout */
 } mate_kernel;
 
 typedef struct {

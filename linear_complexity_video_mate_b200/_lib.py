@@ -17,7 +17,7 @@ EXPORTS = (
     "mate_forward_host_workspace_bytes", "mate_device_status", "mate_last_launch_count", "mate_project_bf16",
     "ssd_scan_bidir_noalloc", "mate_trace_start", "mate_trace_stop", "mate_trace_read", "mate_kernel_name",
     "mate_scan_locality", "ssd_scan_bidir_pd", "mate_ssd_pd_workspace_bytes", "ssd_scan_bidir_backward",
-    "mate_ssd_backward_workspace_bytes",
+    "mate_ssd_backward_workspace_bytes", "mate_selftest_wait_timeout",
 )
 
 _CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp", "wt", "wh", "ww", "st", "sh", "sw")
@@ -65,6 +65,7 @@ def load():
         "mate_ssd_workspace_bytes": (sz, [cfgp, ci]),
         "mate_ssd_pd_workspace_bytes": (sz, [cfgp, ci]),
         "mate_ssd_backward_workspace_bytes": (sz, [cfgp, ci]),
+        "mate_selftest_wait_timeout": (ci, [ctypes.c_uint, vp]),
         "ssd_scan_bidir_backward": (ci, [vp] * 7 + [ci] + [vp] * 8 + [cfgp, vp, sz, vp]),
         "rms_permute": (ci, [vp, vp, ci, cfgp, vp]),
         "rms_unpermute": (ci, [vp, vp, ci, cfgp, vp]),

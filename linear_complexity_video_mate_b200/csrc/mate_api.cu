@@ -1054,6 +1054,16 @@ mate_status mate_device_status(mate_stream_t stream, unsigned int* flags) {
 
 int mate_last_launch_count(void) { return t_launches; }
 
+mate_status mate_selftest_wait_timeout(unsigned int max_polls, mate_stream_t stream) {
+  if (max_polls < 1 || max_polls > 65536) return MATE_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  trace_begin(MATE_K_SELFTEST, st);
+  wait_timeout_selftest_kernel<<<1, 1, 0, st>>>(max_polls);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
 mate_status mate_trace_start(int capacity) {
   if (capacity < 0) return MATE_ERR_ARG;
   std::lock_guard<std::mutex> lock(g_trace.mu);
@@ -1120,6 +1130,7 @@ const char* mate_kernel_name(int kernel) {
     case MATE_K_CONV_SILU: return "conv_silu";
     case MATE_K_GATE_NORM: return "gate_rmsnorm";
     case MATE_K_SSD_BACKWARD: return "ssd_backward_f32";
+    case MATE_K_SELFTEST: return "selftest_wait_timeout";
   }
   return "unknown";
 }

@@ -114,6 +114,22 @@ __global__ void softplus_kernel(const float* __restrict__ dt, const float* __res
 }
 
 // ---------------------------------------------------------------------------------------------------
+// Self-test of the timeout report: one thread waits on a fresh mbarrier that nothing arrives at, polling
+// at most max_polls times, then records MATE_DEV_TIMEOUT in the device status word and returns, as every
+// bounded wait of the library does when it runs out.
+// ---------------------------------------------------------------------------------------------------
+__global__ void wait_timeout_selftest_kernel(unsigned max_polls) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(&bar, 1);
+  mbar_fence_init();
+  for (unsigned i = 0; i < max_polls; ++i) {
+    if (mbar_try_wait(&bar, 0)) return;   // phase 0 never completes: no thread arrives
+    __nanosleep(64);
+  }
+  flag_status(MATE_DEV_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------------------------------
 // fp32 path
 // ---------------------------------------------------------------------------------------------------
 

@@ -38,7 +38,8 @@ int main(void) {
   if (mate_ssd_pd_workspace_bytes(&c, 256) <= mate_ssd_workspace_bytes(&c, 256))
     return fail(8, "per-direction scan workspace not larger");
   if (strcmp(mate_status_str(MATE_ERR_WORKSPACE), "workspace too small") != 0) return fail(9, "status string");
-  for (int k = 0; k <= MATE_K_SSD_BACKWARD; ++k)
+  if (mate_selftest_wait_timeout(0, NULL) != MATE_ERR_ARG) return fail(11, "zero poll limit accepted");
+  for (int k = 0; k <= MATE_K_SELFTEST; ++k)
     if (mate_kernel_name(k) == NULL || strcmp(mate_kernel_name(k), "unknown") == 0) return fail(10, "kernel name");
   printf("ok %zu\n", ws);
   return 0;

@@ -98,6 +98,9 @@ def test_null_and_misaligned_arguments_are_rejected_before_launch(lib):
     we.conv_w = (1 << 20) + 4    # the taps are read as 16-byte vectors
     assert lib.mate_forward(fake, ctypes.byref(we), 0, fake, ctypes.byref(ce), fake, 1 << 40, None) == \
         _lib.MATE_ERR_ARG
+    # the timeout self-test takes a bounded poll count
+    assert lib.mate_selftest_wait_timeout(0, None) == _lib.MATE_ERR_ARG
+    assert lib.mate_selftest_wait_timeout(65537, None) == _lib.MATE_ERR_ARG
     # backward scan: fp32 blocks only, every pointer required, workspace checked
     nbw = lib.mate_ssd_backward_workspace_bytes(cp, 256)
     assert nbw > 0
@@ -147,8 +150,8 @@ def test_noalloc_scan_rejects_problems_beyond_its_scratch(lib):
 
 
 def test_kernel_names_are_distinct(lib):
-    names = [lib.mate_kernel_name(k).decode() for k in range(20)]
-    assert len(set(names)) == 20 and "unknown" not in names, names
+    names = [lib.mate_kernel_name(k).decode() for k in range(21)]
+    assert len(set(names)) == 21 and "unknown" not in names, names
     assert lib.mate_kernel_name(99).decode() == "unknown"
     assert lib.mate_trace_start(-1) == _lib.MATE_ERR_ARG
 
