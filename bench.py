@@ -100,14 +100,29 @@ class ClockSampler:
 
 
 def measured_peaks():
-    """(HBM GB/s, bf16 TFLOP/s sustained, source).  Kernels are timed inside the long timed region, so the
-    sustained GEMM figure is the denominator."""
+    """{hbm, burst, sustained, source}: HBM GB/s and bf16 TFLOP/s (a burst of one GEMM timed alone, and a
+    seconds-long loop under the power cap) from MEASURED_PEAKS.json, else the fallback figures."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return p["hbm_gbs"], p["bf16_tflops_sustained"], "measured (bf16 sustained)"
+        return {"hbm": p["hbm_gbs"], "burst": p["bf16_tflops"], "sustained": p["bf16_tflops_sustained"],
+                "source": "measured"}
     except Exception:
-        return 6650.0, 1400.0, "fallback (bf16 sustained)"
+        return {"hbm": 6650.0, "burst": 1590.0, "sustained": 1400.0, "source": "fallback"}
+
+
+def tensor_peak(peaks, region_s, clocks):
+    """The bf16 denominator for kernels timed in this run: the sustained figure only when the timed region
+    is long enough for the power cap to pull the clock down (at least a second, median SM clock below its
+    maximum); otherwise the burst figure."""
+    sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    at_max = sm is not None and smax is not None and sm >= 0.97 * smax
+    if region_s < 1.0 or at_max or sm is None:
+        why = "timed region under 1 s" if region_s < 1.0 else ("median SM clock at its maximum" if at_max else
+                                                               "no clock record")
+        return peaks["burst"], f"{peaks['source']} bf16 burst ({why})"
+    return peaks["sustained"], f"{peaks['source']} bf16 sustained (timed region {region_s:.1f} s, median SM " \
+                               f"clock {sm:.0f} of {smax:.0f} MHz)"
 
 
 # DRAM bytes per launch measured with ncu (dram__bytes_read.sum + dram__bytes_write.sum), scaled to the
@@ -136,18 +151,64 @@ def measured_traffic(kernel, workload):
     return m["bytes"]
 
 
-def kernel_work(cfg):
-    """Algorithmic work per launch of the kernels the roofline can name: (bound, amount, unit)."""
-    nin = cfg.nh * cfg.P + 2 * cfg.N + cfg.nh
+def kernel_work(cfg, per_dir=False):
+    """Algorithmic work per launch of each library kernel at this workload: {kernel: (flops or None, bytes)}.
+    FLOPs count a multiply-add as 2 and only the products the method needs (each causal half once, the
+    carried-state product C H^T once).  Bytes count each tensor once per kernel that must read or write it
+    (inputs, outputs and the scan's stored intermediates: Gram matrix, chunk states, carried states, decay
+    tables), nothing for re-reads."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    B, n, R, d, nh, P, N, Q = cfg.B, cfg.n, cfg.R, cfg.d, cfg.nh, cfg.P, cfg.N, cfg.Q
+    nin = nh * P + 2 * N + nh
     NI = nin + 3 * cfg.th * cfg.tp
-    KO = cfg.nh * cfg.P + cfg.th * cfg.tp
-    rows = cfg.B * cfg.n
+    KO = nh * P + cfg.th * cfg.tp
+    rows, rrows = B * n, B * R
     win = cfg.wt * cfg.wh * cfg.ww
+    nVc, nRc = B * -(-n // Q), B * -(-R // Q)
+    ldd = 2 * nh
+    PN = P * N
+    tbl = 2176 * 4 * 2        # decay tables per (video chunk, head): two 128-row tiles
     return {
-        "in_projection": ("tensor", 2.0 * rows * cfg.d * NI, "TFLOP/s"),
-        "out_projection": ("tensor", 2.0 * rows * KO * cfg.d, "TFLOP/s"),
-        "tesa": ("tensor", 4.0 * rows * cfg.th * win * cfg.tp, "TFLOP/s"),
+        "in_projection": (2.0 * rows * d * NI, rows * d * es + rows * NI * es + rows * nh * 4 + NI * d * es),
+        "in_projection_review": (2.0 * rrows * d * nin, rrows * d * es + rrows * nin * es + rrows * nh * 4),
+        "out_projection": (2.0 * rows * KO * d, rows * KO * es + rows * d * es + d * KO * es),
+        "tesa": (4.0 * rows * cfg.th * win * cfg.tp, rows * 3 * cfg.th * cfg.tp * es + rows * cfg.th * cfg.tp * es),
+        "review_pool": (None, rows * d * es + rrows * d * es),
+        "ssd_gram": (2.0 * nVc * Q * Q * N, rows * 2 * N * es + nVc * Q * Q * 2 + nVc * Q * 4),
+        "ssd_state": (2.0 * (2 * nVc + (2 if per_dir else 1) * nRc) * nh * N * P * Q,
+                      (rows + rrows) * (nh * P + N) * es + (rows + rrows) * ldd * 4 +
+                      (2 * nVc + (2 if per_dir else 1) * nRc) * nh * PN * 4 + nVc * nh * tbl + nVc * Q * 4),
+        "ssd_carry": (None, (2 * nVc + (2 if per_dir else 1) * nRc) * nh * PN * 4 + 2 * nVc * nh * 2 * PN * 2),
+        "ssd_output": (nVc * nh * (2.0 * Q * Q * P + 2.0 * Q * N * 2 * P),
+                       rows * (nh * P + N) * es + nVc * Q * Q * 2 + nVc * Q * 4 + 2 * nVc * nh * 2 * PN * 2 +
+                       nVc * nh * tbl + rows * nh * P * es),
+        "y_to_grid": (None, 2.0 * rows * nh * P * es),
+        "conv_silu": (None, 2.0 * (rows + rrows) * (nh * P + 2 * N) * es),
+        "gate_rmsnorm": (None, 3.0 * rows * nh * P * es),
+        "pack_weights": (None, 2.0 * (NI * d + d * KO) * es),
+        # the DiT block around the mixer
+        "ln_modulate": (None, 2.0 * rows * d * es),
+        "mlp_up": (2.0 * rows * d * 4 * d, rows * d * es + rows * 4 * d * es + 4 * d * d * es),
+        "mlp_down": (2.0 * rows * 4 * d * d, rows * 4 * d * es + 2 * rows * d * es + 4 * d * d * es),
     }
+
+
+def roofline_table(per, work, hbm_peak, tf_peak):
+    """Per traced kernel: launches, ms per launch, and achieved TFLOP/s and GB/s against the peaks."""
+    out = {}
+    for k, (cnt, tot) in sorted(per.items(), key=lambda kv: -kv[1][1]):
+        ms = tot / cnt
+        row = {"launches": cnt, "ms_per_launch": ms}
+        if k in work:
+            fl, by = work[k]
+            if fl is not None:
+                row["tflops"] = fl / (ms * 1e-3) / 1e12
+                row["tensor_frac"] = row["tflops"] / tf_peak
+            row["algorithmic_bytes"] = by
+            row["gbs"] = by / (ms * 1e-3) / 1e9
+            row["hbm_frac"] = row["gbs"] / hbm_peak
+        out[k] = row
+    return out
 
 
 def extras_weights(cfg, seed):
@@ -165,12 +226,13 @@ def time_block_variant(M, torch, cfg, wv, X, out, stream, steps):
     """ms per block of a MateBlock built from weights wv (3 warm-up forwards, `steps` timed ones cycling
     the layers) and per-kernel [launches, total ms] from the library trace."""
     blk = M.MateBlock(cfg, M.weights_to_device(wv, cfg))
-    for s in range(3):
+    nl = 0
+    for s in range(4):
         blk.forward(X, s, out)
-    nl = M.MateBlock.last_launch_count()
+        nl = max(nl, M.MateBlock.last_launch_count())
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    trace = M.KernelTrace(nl * steps).start()
+    trace = M.KernelTrace(nl * steps + 16).start()
     e0.record(stream)
     for s in range(steps):
         blk.forward(X, s % 4, out)
@@ -220,6 +282,101 @@ def measure_extras(M, torch, cfg, w, X, out, stream, base_ms, hbm_peak, steps=20
             gbs = b / (kms * 1e-3) / 1e9
             res[k] = {"ms_per_launch": kms, "algorithmic_bytes": b, "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
     return res
+
+
+def timing_weights(cfg, seed):
+    """Block weights with the workload's initialisation (linear weights N(0, 1/fan_in) rounded to bf16,
+    A_log U[0, 1], D N(0, 1), dt_bias 0) from their own seeded stream, without drawing a latent grid."""
+    rng = np.random.default_rng(seed)
+    lin = lambda o, i: mi.round_to_bf16((rng.standard_normal((o, i)) / np.sqrt(i)).astype(np.float32))
+    return dict(W_in=lin(cfg.d_in_proj, cfg.d), dt_bias=np.zeros(cfg.nh, np.float32),
+                A_log=rng.uniform(0.0, 1.0, cfg.nh).astype(np.float32), D=rng.standard_normal(cfg.nh).astype(np.float32),
+                W_out=lin(cfg.d, cfg.d_inner), W_qkv=lin(3 * cfg.d_attn, cfg.d), W_o=lin(cfg.d, cfg.d_attn))
+
+
+def measure_scaling(M, torch, stream, headline, headline_name, headline_ms, steps=12):
+    """ms per block of every bf16 workload (steps cycling the four layers; seeded Gaussian latents drawn on
+    the device, weights from the workload's seeded generator), the headline workload's own number reused,
+    and the per-token time of the three d = 1024 clips against the smallest one."""
+    out = {}
+    for name in ("bf16_16x32x32", "bf16_64x32x32", "bf16_256x32x32", "bf16_2x64x48x48_d2048"):
+        cfg = mi.CONFIGS[name]
+        if name == headline_name:
+            ms = headline_ms
+        else:
+            blk = M.MateBlock(cfg, M.weights_to_device(timing_weights(cfg, cfg.seed), cfg))
+            g = torch.Generator(device="cuda").manual_seed(cfg.seed)
+            X = torch.randn((cfg.B, cfg.T, cfg.H, cfg.W, cfg.d), generator=g, device="cuda").to(torch.bfloat16)
+            o = torch.empty_like(X)
+            for s in range(4):
+                blk.forward(X, s, o)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for s in range(steps):
+                blk.forward(X, s % 4, o)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / steps
+            del blk, X, o
+        tokens = cfg.B * cfg.n
+        out[name] = {"tokens": tokens, "ms_per_block": ms, "ns_per_token": ms * 1e6 / tokens}
+    clips = ("bf16_16x32x32", "bf16_64x32x32", "bf16_256x32x32")   # the same block width, 16 to 256 frames
+    base = out[clips[0]]["ns_per_token"]
+    for name in clips[1:]:
+        out[name]["per_token_vs_16x32x32"] = out[name]["ns_per_token"] / base
+    # linear in the token count: ms = fixed + slope * tokens (least squares over the three clips); the fit's
+    # largest relative residual says how far the measured times are from a straight line
+    nt = np.array([out[k]["tokens"] for k in clips], np.float64)
+    t = np.array([out[k]["ms_per_block"] for k in clips], np.float64)
+    slope, fixed = np.polyfit(nt, t, 1)
+    resid = float(np.max(np.abs(fixed + slope * nt - t) / t))
+    out["affine_fit"] = {"fixed_ms": float(fixed), "ns_per_token": float(slope * 1e6), "max_rel_residual": resid}
+    out["linear_within_15pct"] = resid <= 0.15
+    return out
+
+
+def measure_dit(M, torch, cfg, w, X, stream, hbm_peak, tf_peak, steps=12, dc=256):
+    """The DiT block around the mixer (adaLN modulation, layer norms, the mixer behind a gated residual, the
+    gated GELU MLP of width 4 d) at the headline workload, timed after the headline region: ms per block,
+    algorithmic TFLOP/s and the per-kernel fractions.  Weights: W_ada N(0, 1/dc), W1 N(0, 1/d), W2
+    N(0, 1/(4 d)), biases N(0, 0.1^2), c N(0, 1), seeded."""
+    rng = np.random.default_rng(777)
+    d = cfg.d
+    bf = lambda a: mi.round_to_bf16(a.astype(np.float32))
+    dw = dict(W_ada=bf(rng.standard_normal((6 * d, dc)) / np.sqrt(dc)), b_ada=(0.1 * rng.standard_normal(6 * d)),
+              W1=bf(rng.standard_normal((4 * d, d)) / np.sqrt(d)), b1=0.1 * rng.standard_normal(4 * d),
+              W2=bf(rng.standard_normal((d, 4 * d)) / np.sqrt(4 * d)), b2=0.1 * rng.standard_normal(d))
+    c = torch.as_tensor(rng.standard_normal((cfg.B, dc)).astype(np.float32)).cuda()
+    blk = M.DitBlock(cfg, M.weights_to_device(w, cfg), M.dit_weights_to_device(dw, cfg), dc)
+    out = torch.empty_like(X)
+    nl = 0
+    for s in range(4):
+        blk.forward(X, c, s, out)
+        nl = max(nl, M.MateBlock.last_launch_count())
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    trace = M.KernelTrace(nl * steps + 16).start()
+    e0.record(stream)
+    for s in range(steps):
+        blk.forward(X, c, s % 4, out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    trace.stop()
+    per = {}
+    for name, kms in trace.read():
+        a = per.setdefault(name, [0, 0.0])
+        a[0] += 1
+        a[1] += kms
+    ms = e0.elapsed_time(e1) / steps
+    rows = cfg.B * cfg.n
+    flops = sum(flops_per_block(cfg).values()) + 16.0 * rows * d * d
+    table = roofline_table(per, kernel_work(cfg), hbm_peak, tf_peak)
+    del blk
+    return {"ms_per_block": ms, "tokens_per_s": rows / (ms * 1e-3), "tflops": flops / (ms * 1e-3) / 1e12,
+            "steps": steps, "conditioning_width": dc,
+            "kernels": {k: table[k] for k in ("mlp_up", "mlp_down", "ln_modulate", "ada_modulation", "out_projection")
+                        if k in table}}
 
 
 def oracle_sample_cfg(cfg, frames):
@@ -300,6 +457,7 @@ def main():
     ap.add_argument("--oracle-frames", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the full-Mamba2-block side measurement")
+    ap.add_argument("--no-scaling", action="store_true", help="skip the per-workload ms/block side measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -330,9 +488,10 @@ def main():
         if world > 1:
             dist.barrier()
 
-    for s in range(args.warmup):
+    launches_per_step = 0
+    for s in range(max(args.warmup, 4)):   # every layer at least once: the trace is sized by the largest
         blk.forward(X, s % 4, out)
-    launches_per_step = M.MateBlock.last_launch_count()
+        launches_per_step = max(launches_per_step, M.MateBlock.last_launch_count())
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -341,7 +500,7 @@ def main():
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    trace = M.KernelTrace(launches_per_step * args.steps).start()   # events around every launch
+    trace = M.KernelTrace(launches_per_step * args.steps + 16).start()   # events around every launch
     e0.record(stream)
     for s in range(args.steps):
         blk.forward(X, s % 4, out)
@@ -364,26 +523,44 @@ def main():
     kernels = {k: {"launches": n, "ms_per_launch": t / n, "share": t / traced_ms}
                for k, (n, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
     work = kernel_work(cfg)
+    peaks = measured_peaks()
+    hbm_peak = peaks["hbm"]
+    tf_peak, tf_src = tensor_peak(peaks, ms * args.steps * 1e-3, clocks)
+    peak_src = tf_src
+    table = roofline_table(per, work, hbm_peak, tf_peak)
+    # the roofline names the kernel with the largest share of the traced time; a kernel with a FLOP model
+    # is measured against the tensor pipe, the others against HBM
     dom = max((k for k in per if k in work), key=lambda k: per[k][1])
-    bound, amount, runit = work[dom]
     dom_ms = per[dom][1] / per[dom][0]
-    hbm_peak, tf_peak, peak_src = measured_peaks()
-    achieved = amount / (dom_ms * 1e-3) / 1e12
+    dflops, dbytes = work[dom]
+    if dflops is not None:
+        bound, runit, achieved, dpeak = "tensor", "TFLOP/s", dflops / (dom_ms * 1e-3) / 1e12, tf_peak
+    else:
+        bound, runit, achieved, dpeak = "hbm", "GB/s", dbytes / (dom_ms * 1e-3) / 1e9, hbm_peak
+        peak_src = f"{peaks['source']} HBM copy bandwidth"
 
-    # end to end through mate_forward_host: pinned host X in, pinned host Out back, every step
+    # end to end through the host-buffer entry points: pinned host X in, pinned host Out back, every step;
+    # the headline uses the pipelined calls (each call's input copy overlaps the previous call's output
+    # copy), the one-call-at-a-time form is reported beside it
     xh = X.cpu().pin_memory()
     oh = torch.empty_like(xh).pin_memory()
-    for s in range(2):
-        blk.forward_host(xh, s, oh)
-    torch.cuda.synchronize()
-    barrier()
-    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h0.record(stream)
-    for s in range(args.e2e_steps):
-        blk.forward_host(xh, s % 4, oh)
-    h1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.e2e_steps, world, "cuda")
+
+    def e2e(pipelined):
+        for s in range(3):
+            blk.forward_host(xh, s, oh, pipelined=pipelined)
+        M.MateBlock.flush_host()
+        torch.cuda.synchronize()
+        barrier()
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        for s in range(args.e2e_steps):
+            blk.forward_host(xh, s % 4, oh, pipelined=pipelined)
+        M.MateBlock.flush_host()   # every step's output has reached the host before the end event
+        h1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(h0.elapsed_time(h1) / args.e2e_steps, world, "cuda")
+    e2e_ms = e2e(True)
+    e2e_serial_ms = e2e(False)
     nbytes = X.numel() * X.element_size()
 
     # scan locality of the workload's grid (outside the timed region): mean sequence distance of
@@ -403,8 +580,12 @@ def main():
 
     # side measurements, outside the headline region: the block with the rest of the Mamba2 block, and with
     # separate backward-scan parameters; a failure is reported in the line instead of ending the run
-    extras = per_direction = None
+    extras = per_direction = dit = None
     if not args.no_extras:
+        try:
+            dit = measure_dit(M, torch, cfg, w, X, stream, hbm_peak, tf_peak)
+        except Exception as e:  # noqa: BLE001
+            dit = {"error": f"{type(e).__name__}: {e}"}
         try:
             extras = measure_extras(M, torch, cfg, w, X, out, stream, ms, hbm_peak)
         except Exception as e:  # noqa: BLE001
@@ -413,6 +594,16 @@ def main():
             per_direction = measure_per_direction(M, torch, cfg, w, X, out, stream, ms)
         except Exception as e:  # noqa: BLE001
             per_direction = {"error": f"{type(e).__name__}: {e}"}
+
+    # linear scaling in token count: ms per block of every workload in the same run (outside the headline
+    # region), the 65,536-token clip over its four layers
+    scaling = None
+    if not args.no_scaling:
+        try:
+            scaling = measure_scaling(M, torch, stream, args.config, cfg.name, ms)
+            torch.cuda.empty_cache()
+        except Exception as e:  # noqa: BLE001
+            scaling = {"error": f"{type(e).__name__}: {e}"}
 
     tokens_per_step = cfg.B * cfg.n
     value = job_value(tokens_per_step, world, ms)
@@ -429,18 +620,25 @@ def main():
         "ms_per_block": ms,
         "block_tflops": total_flops / (ms * 1e-3) / 1e12,
         "block_frac_of_bf16_peak": total_flops / (ms * 1e-3) / 1e12 / tf_peak,
-        "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": tf_peak, "unit": runit,
-                     "frac": achieved / tf_peak, "traffic": measured_traffic(dom, args.config),
+        "scaling_mode": "weak",
+        "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": dpeak, "unit": runit,
+                     "frac": achieved / dpeak, "traffic": measured_traffic(dom, args.config),
                      "traffic_unit": "bytes per launch", "peak_source": peak_src,
+                     "algorithmic": dflops if dflops is not None else dbytes,
                      "kernel_ms": dom_ms, "launches_timed": per[dom][0],
                      "timing": "CUDA events around each launch inside the timed region (library trace)"},
         "kernels": kernels,
+        "kernel_roofline": {"peaks": {"tensor_tflops": tf_peak, "hbm_gbs": hbm_peak, "tensor_source": tf_src},
+                            "per_kernel": table},
+        "scaling": scaling,
         "e2e": {"value": job_value(tokens_per_step, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": nbytes,
-                "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms, "api": "mate_forward_host"},
+                "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms, "api": "mate_forward_host_pipelined",
+                "one_call_at_a_time_ms_per_step": e2e_serial_ms},
         "gpu_launches": len(records),
         "scan_locality": locality,
         "mamba_extras": extras,
         "per_direction_scan": per_direction,
+        "dit_block": dit,
         "clocks": clocks,
         "device_status": status,
     }

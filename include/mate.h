@@ -104,7 +104,24 @@ typedef struct {
   const float* conv_w;    /* [nh*P + 2N, 4] depthwise taps per channel of x | B | C, tap 3 on the current row */
   const float* conv_b;    /* [nh*P + 2N]  convolution bias                                           */
   const float* norm_w;    /* [nh*P]   gated RMSNorm weight                                           */
+  /* Optional: the buffer mate_pack_weights filled from these weights (same cfg, mamba_extras included).
+   * Given, mate_forward / mate_forward_host* read the packed projection matrices from it; null, they pack
+   * W_in, W_qkv, W_z, W_out and W_o into the workspace on every call. */
+  const void* packed;
 } mate_weights;
+
+/*
+ * The projections run as two GEMMs over packed weight matrices: [W_in; W_qkv (; W_z)] (the MA
+ * in-projection fused with TESA's qkv projection, the gate rows last) and [W_out | W_o] (the two
+ * out-projections side by side, so that the branch sum falls out of the K reduction).  mate_pack_weights
+ * writes both into `packed` (at least mate_packed_weights_bytes(cfg) bytes, 16-byte aligned) once; pass it
+ * as w->packed so that the block does not repack on every call.  Stream-ordered; MATE_ERR_ARG for a null
+ * or misaligned matrix (W_z required when cfg->mamba_extras = 1), MATE_ERR_WORKSPACE if packed_bytes is
+ * too small.  The pages have no counterpart: this is how the fused projections are laid out.
+ */
+MATE_API size_t mate_packed_weights_bytes(const mate_config* cfg);
+MATE_API mate_status mate_pack_weights(const mate_weights* w, const mate_config* cfg, void* packed,
+                                       size_t packed_bytes, mate_stream_t stream);
 
 /*
  * Self-test of the timeout report (no counterpart in the pages).  Launches one thread that waits on a
@@ -209,8 +226,8 @@ MATE_API mate_status ssd_scan_bidir_backward(const void* x, const void* Bm, cons
                                              const mate_config* cfg, void* ws, size_t ws_bytes,
                                              mate_stream_t stream);
 
-/* Size of the fixed device scratch buffer behind ssd_scan_bidir_noalloc: 32 MiB. */
-#define MATE_SSD_NOALLOC_SCRATCH_BYTES (32u << 20)
+/* Size of the fixed device scratch buffer behind ssd_scan_bidir_noalloc: 64 MiB. */
+#define MATE_SSD_NOALLOC_SCRATCH_BYTES (64u << 20)
 
 /*
  * ssd_scan_bidir for callers that must not allocate device memory.  The paper has no counterpart to
@@ -225,11 +242,14 @@ MATE_API mate_status ssd_scan_bidir_backward(const void* x, const void* Bm, cons
  * Every GPU on which the library's device code is loaded holds that array until the process exits.
  * A problem with mate_ssd_workspace_bytes(cfg, prefix_len) > MATE_SSD_NOALLOC_SCRATCH_BYTES is
  * rejected with MATE_ERR_TOO_LARGE before any device work (with the bf16 kernels, nh = 16, B = 1 and
- * 128 prefix rows, that admits up to about 7 000 video tokens).
+ * 128 prefix rows the scratch takes about 9.4 KiB per video token, which admits up to 26 chunks of 256
+ * video tokens, 6 656 tokens; the fp32 kernels need only the step sizes, 4 bytes per row and head).
  *
  * Set-up: the first call on a device (the device current at the call) looks up the array's device
  * address once, which can load the library's device code onto that device; make that first call
- * before any stream capture on the device.  Later calls on the device reuse the address.
+ * before any stream capture on the device.  Later calls on the device reuse the address as long as the
+ * device's CUDA context is the same one; after cudaDeviceReset the next call looks it up again (and is
+ * then again a first call).
  *
  * Sharing: all calls on one device use the same array, and it keeps what the last call left in it.
  * Each call writes every scratch byte it reads before reading it, so nothing needs clearing between
@@ -238,7 +258,8 @@ MATE_API mate_status ssd_scan_bidir_backward(const void* x, const void* Bm, cons
  * after the other and are safe.
  *
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine is called.  Errors as
- * ssd_scan_bidir, plus MATE_ERR_TOO_LARGE; MATE_ERR_CUDA if the address look-up fails.
+ * ssd_scan_bidir, plus MATE_ERR_TOO_LARGE (checked before the pointers); MATE_ERR_CUDA if the address
+ * look-up fails.
  */
 MATE_API mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const void* Cm, const float* dt,
                                             const float* dt_bias, const float* A_log, const float* D, int prefix_len,
@@ -295,18 +316,75 @@ MATE_API mate_status mate_forward(const void* X, const mate_weights* w, int laye
  * starts as soon as it has landed, and each chunk of Out leaves as soon as its out-projection is done.
  * The copies start after all earlier work on `stream`, and the call ends on `stream` only when the last
  * chunk has reached Out_host.  The host buffers must stay valid until the stream reaches the end of the
- * call.  ws: at least mate_workspace_bytes(cfg) + 2 * B*T*H*W*d*elem bytes.
+ * call.  ws: at least mate_forward_host_workspace_bytes(cfg) bytes.
  */
 MATE_API mate_status mate_forward_host(const void* X_host, const mate_weights* w, int layer_idx, void* Out_host,
                               const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream);
 
-/* Workspace bytes needed by mate_forward_host. */
+/*
+ * mate_forward_host for a sequence of calls on one workspace in which a call's host copies overlap the
+ * neighbouring calls' work: its input copy runs during the previous call's output copy (the two
+ * directions of the host link at the same time), and its output copy runs during the next call's block.
+ * Same arguments and result as mate_forward_host; calls alternate between two device input slots and two
+ * device output slots of the workspace.  Ordering:
+ *   - A call's input copy waits only until the call before the previous one (same slot) has read its
+ *     input, and for the output copies of the two previous calls whose Out_host overlaps X_host (so a
+ *     chain that feeds one call's output to the next call as input stays correct).  It does NOT wait for
+ *     other work enqueued on `stream` before the call: if device work on `stream` writes X_host (a
+ *     device-to-host copy), synchronise before the call.  The first call on a workspace, and a call after
+ *     calls on another workspace of the same device, start their copies after all earlier work on `stream`.
+ *   - When `stream` reaches the end of a call, the PREVIOUS pipelined call's Out_host is complete; this
+ *     call's Out_host is complete when `stream` reaches the end of the next pipelined call or of a
+ *     mate_forward_host_flush.  mate_forward_host (the one-at-a-time form) waits for all of them first.
+ * For bf16 blocks; fp32 blocks run as mate_forward_host.  The pages have no counterpart.
+ */
+MATE_API mate_status mate_forward_host_pipelined(const void* X_host, const mate_weights* w, int layer_idx,
+                                                 void* Out_host, const mate_config* cfg, void* ws, size_t ws_bytes,
+                                                 mate_stream_t stream);
+
+/* Makes `stream` wait for the output copies of every pipelined call on the current device that no stream
+ * waits for yet; once `stream` reaches this point, every such call's Out_host is complete. */
+MATE_API mate_status mate_forward_host_flush(mate_stream_t stream);
+
+/* Workspace bytes needed by mate_forward_host and mate_forward_host_pipelined: the block's workspace,
+ * two device input slots and two device output slots. */
 MATE_API size_t mate_forward_host_workspace_bytes(const mate_config* cfg);
 
 /*
+ * A DiT block with the MATE block as its token mixer ([ABS]: MATE replaces the self-attention of a DiT;
+ * [NEWS] method: the rest of the DiT stays as it is).  The pages do not describe that rest; this is the
+ * standard DiT block with adaLN-Zero conditioning:
+ *   [shift_a, scale_a, gate_a, shift_m, scale_m, gate_m] = silu(c_b) W_ada^T + b_ada   (sample b, 6 x d)
+ *   X1  = X  + gate_a * MATE(LN(X)  (1 + scale_a) + shift_a)          (MATE: mate_forward, layer_idx)
+ *   Out = X1 + gate_m * (W2 gelu_tanh(W1 (LN(X1) (1 + scale_m) + shift_m) + b1) + b2)
+ * LN: per token over d channels, no affine parameters, eps 1e-6; gelu_tanh(v) = v/2 (1 + tanh(sqrt(2/pi)
+ * (v + 0.044715 v^3))); no cross-attention (text enters through c).  The gated residuals are applied in the
+ * epilogues of the out-projection and of the MLP's second GEMM; the GELU in the first GEMM's epilogue.
+ *   X, Out [B, T, H, W, d] cfg->dtype (may not alias); c [B, dc] float; d <= 2048.
+ *   dw: W_ada [6d, dc], W1 [4d, d], W2 [d, 4d] in cfg->dtype; b_ada [6d], b1 [4d], b2 [d] float.
+ *   mw: the mixer's weights as for mate_forward (mw->packed may hold mate_pack_weights' buffer).
+ * ws: at least mate_dit_workspace_bytes(cfg) bytes.  MATE_ERR_UNSUPPORTED for d > 2048.
+ */
+typedef struct {
+  const void* W_ada;   /* [6d, dc] */
+  const float* b_ada;  /* [6d] */
+  const void* W1;      /* [4d, d] */
+  const float* b1;     /* [4d] */
+  const void* W2;      /* [d, 4d] */
+  const float* b2;     /* [d] */
+} mate_dit_weights;
+
+MATE_API size_t mate_dit_workspace_bytes(const mate_config* cfg);
+MATE_API mate_status mate_dit_block_forward(const void* X, const float* c, int dc, const mate_dit_weights* dw,
+                                            const mate_weights* mw, int layer_idx, void* Out, const mate_config* cfg,
+                                            void* ws, size_t ws_bytes, mate_stream_t stream);
+
+/*
  * Reads and clears the device status word that kernels set when a bounded wait runs out.  Synchronises
- * `stream` first.  *flags receives the raw bits (1 = wait timed out); returns MATE_ERR_TIMEOUT if any
- * bit was set, MATE_OK otherwise.
+ * `stream` first, then takes the word with one atomic exchange on the device (a flag that a kernel on
+ * another stream sets meanwhile is reported now or by the next call, never dropped), and synchronises
+ * `stream` again.  *flags receives the raw bits (1 = wait timed out); returns MATE_ERR_TIMEOUT if any bit
+ * was set, MATE_OK otherwise.
  */
 MATE_API mate_status mate_device_status(mate_stream_t stream, unsigned int* flags);
 
@@ -344,7 +422,11 @@ typedef enum {
   MATE_K_CONV_SILU = 17,       /* causal depthwise convolution + SiLU on x | B | C (mamba_extras) */
   MATE_K_GATE_NORM = 18,       /* y silu(z) and gated RMSNorm (mamba_extras) */
   MATE_K_SSD_BACKWARD = 19,    /* ssd_scan_bidir_backward (fp32) */
-  MATE_K_SELFTEST = 20         /* mate_selftest_wait_timeout */
+  MATE_K_SELFTEST = 20,        /* mate_selftest_wait_timeout */
+  MATE_K_ADA_MODULATION = 21,  /* DiT block: modulation vectors silu(c) W_ada^T + b_ada */
+  MATE_K_LN_MODULATE = 22,     /* DiT block: layer norm + scale and shift */
+  MATE_K_MLP_UP = 23,          /* DiT block: gelu(h W1^T + b1) */
+  MATE_K_MLP_DOWN = 24         /* DiT block: X1 + gate_m (Z W2^T + b2) */
 } mate_kernel;
 
 typedef struct {

@@ -7,7 +7,7 @@ LIB_PATH = os.path.join(_HERE, "libmate.so")
 
 (MATE_OK, MATE_ERR_ARG, MATE_ERR_SHAPE, MATE_ERR_WORKSPACE, MATE_ERR_CUDA, MATE_ERR_TIMEOUT, MATE_ERR_UNSUPPORTED,
  MATE_ERR_TOO_LARGE) = range(8)
-MATE_SSD_NOALLOC_SCRATCH_BYTES = 32 << 20
+MATE_SSD_NOALLOC_SCRATCH_BYTES = 64 << 20
 MATE_BF16, MATE_F32 = 0, 1
 
 # every symbol include/mate.h declares
@@ -17,7 +17,9 @@ EXPORTS = (
     "mate_forward_host_workspace_bytes", "mate_device_status", "mate_last_launch_count", "mate_project_bf16",
     "ssd_scan_bidir_noalloc", "mate_trace_start", "mate_trace_stop", "mate_trace_read", "mate_kernel_name",
     "mate_scan_locality", "ssd_scan_bidir_pd", "mate_ssd_pd_workspace_bytes", "ssd_scan_bidir_backward",
-    "mate_ssd_backward_workspace_bytes", "mate_selftest_wait_timeout",
+    "mate_ssd_backward_workspace_bytes", "mate_selftest_wait_timeout", "mate_forward_host_pipelined",
+    "mate_packed_weights_bytes", "mate_pack_weights", "mate_dit_workspace_bytes", "mate_dit_block_forward",
+    "mate_forward_host_flush",
 )
 
 _CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp", "wt", "wh", "ww", "st", "sh", "sw")
@@ -32,7 +34,12 @@ class CWeights(ctypes.Structure):
                 ("D", ctypes.c_void_p), ("W_out", ctypes.c_void_p), ("W_qkv", ctypes.c_void_p),
                 ("W_o", ctypes.c_void_p), ("dt_bias_b", ctypes.c_void_p), ("A_log_b", ctypes.c_void_p),
                 ("D_b", ctypes.c_void_p), ("W_z", ctypes.c_void_p), ("conv_w", ctypes.c_void_p),
-                ("conv_b", ctypes.c_void_p), ("norm_w", ctypes.c_void_p)]
+                ("conv_b", ctypes.c_void_p), ("norm_w", ctypes.c_void_p), ("packed", ctypes.c_void_p)]
+
+
+class CDitWeights(ctypes.Structure):
+    _fields_ = [("W_ada", ctypes.c_void_p), ("b_ada", ctypes.c_void_p), ("W1", ctypes.c_void_p),
+                ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
 
 
 class CTraceRecord(ctypes.Structure):
@@ -81,6 +88,12 @@ def load():
         "tesa_forward": (ci, [vp, vp, ci, cfgp, vp]),
         "mate_forward": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
         "mate_forward_host": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
+        "mate_forward_host_pipelined": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
+        "mate_packed_weights_bytes": (sz, [cfgp]),
+        "mate_forward_host_flush": (ci, [vp]),
+        "mate_pack_weights": (ci, [wp, cfgp, vp, sz, vp]),
+        "mate_dit_workspace_bytes": (sz, [cfgp]),
+        "mate_dit_block_forward": (ci, [vp, vp, ci, ctypes.POINTER(CDitWeights), wp, ci, vp, cfgp, vp, sz, vp]),
         "mate_forward_host_workspace_bytes": (sz, [cfgp]),
         "mate_device_status": (ci, [vp, ctypes.POINTER(ctypes.c_uint)]),
         "mate_last_launch_count": (ci, []),

@@ -9,6 +9,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,6 +23,10 @@ enum : unsigned { MATE_DEV_TIMEOUT = 1u, MATE_DEV_BAD_ARG = 2u };
 __device__ unsigned int g_dev_status = 0;
 
 __device__ __forceinline__ void flag_status(unsigned f) { atomicOr(&g_dev_status, f); }
+
+// mate_device_status's one-step read-and-clear: the word's bits move to g_dev_status_taken.
+__device__ unsigned int g_dev_status_taken = 0;
+__global__ void status_take_kernel() { g_dev_status_taken = atomicExch(&g_dev_status, 0u); }
 
 // ---------------------------------------------------------------------------------------------------
 // Rotary Major Scan index maps.  Order o lists the grid axes fastest-varying first:
@@ -60,6 +65,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
   return __bfloat1622float2(v);
+}
+
+// Two fp32 values to an fp16 pair (round to nearest; magnitudes beyond the fp16 range saturate to
+// +-65504 instead of becoming infinite).
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
+  __half2 v = *reinterpret_cast<__half2*>(&u);
+  return __half22float2(v);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -340,6 +358,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
          | (static_cast<uint32_t>(b_mn_major) << 16)  // B major
          | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+// The same for fp16 x fp16 -> fp32 (format code 0 for both operands).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4) | (static_cast<uint32_t>(a_mn_major) << 15) | (static_cast<uint32_t>(b_mn_major) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Byte offset of element (row, col) inside a K-major 128B-swizzled tile whose 64-column K blocks are

@@ -12,11 +12,39 @@
 //   warps 2..5  epilogue: tcgen05.ld the finished accumulator, convert, store; the other accumulator
 //               is being filled meanwhile.
 // Optional epilogue side output: columns [dt_col0, dt_col0 + dt_cols) also produce
-// delta = softplus(acc + dt_bias) in fp32 (the Mamba2 step size).
+// delta = softplus(acc + dt_bias) in fp32 (the Mamba2 step size).  Optional epilogue transforms
+// (GemmEpilogue) serve the DiT block around MATE: bias + GELU for the MLP's first layer, bias and a gated
+// residual for the MLP's second layer and for the token mixer's output.
 #pragma once
 #include "common.cuh"
 
 namespace mate {
+
+// Transforms of a projection's accumulator before it is stored, applied in this order:
+//   v = acc + bias[col]                               (bias: [N] fp32; null: none)
+//   v = gelu_tanh(v)                                  (act == 1)
+//   v = resid[row][col] + gate[row / gate_rows][col] v (resid: the residual stream, the output's element
+//                                                      type; gate [M / gate_rows][ld_gate] fp32, null: 1)
+struct GemmEpilogue {
+  const float* bias = nullptr;
+  int act = 0;
+  const void* resid = nullptr;
+  long long ld_resid = 0;
+  const float* gate = nullptr;
+  int ld_gate = 0;
+  int gate_rows = 1;
+};
+
+// GELU in its tanh form, v/2 (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))); `fast` takes tanh from the
+// special-function unit (relative error about 2^-11, below a bf16 rounding), otherwise from tanhf.
+template <bool fast>
+__device__ __forceinline__ float gelu_tanh_f(float v) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
+  float t;
+  if (fast) asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(u));
+  else t = tanhf(u);
+  return 0.5f * v * (1.f + t);
+}
 
 struct GemmParams {
   int M, N, K;
@@ -31,6 +59,7 @@ struct GemmParams {
   int dt_col0, dt_cols;
   const float* dt_bias;
   const float* dt_bias2;   // optional: a second side output softplus(acc + dt_bias2) at column offset dt_cols
+  GemmEpilogue ep;
 };
 
 constexpr int kGemmBM = 128;
@@ -147,6 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else {
     // epilogue warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1 of this CTA's 128 rows
     const int quad = warp & 3;
+    const bool has_ep = p.ep.bias != nullptr || p.ep.act != 0 || p.ep.resid != nullptr;
     int it = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
       const int mb = tile / p.num_n_tiles, nb = tile % p.num_n_tiles;
@@ -164,21 +194,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tmem_wait_ld();
         const int col0 = nb * p.bn + c0;
         if (!row_ok || col0 >= col_end) continue;
-        if (col0 + 32 <= col_end) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        const bool full32 = col0 + 32 <= col_end;
+        if (has_ep) {
+          const GemmEpilogue& e = p.ep;
+          if (e.bias != nullptr) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (full32 || col0 + j < col_end) v[j] += __ldg(e.bias + col0 + j);
+          }
+          if (e.act == 1) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_f<true>(v[j]);
+          }
+          if (e.resid != nullptr) {
+            const __nv_bfloat16* rr = static_cast<const __nv_bfloat16*>(e.resid) + row * e.ld_resid + col0;
+            const float* g = e.gate != nullptr ? e.gate + static_cast<long long>(row / e.gate_rows) * e.ld_gate + col0
+                                               : nullptr;
+            if (full32) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 x4 = __ldg(reinterpret_cast<const uint4*>(rr) + q);
+                const uint32_t* xw = reinterpret_cast<const uint32_t*>(&x4);
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                  const float2 xf = unpack_bf16x2(xw[e2]);
+                  const int j = q * 8 + 2 * e2;
+                  v[j] = xf.x + (g != nullptr ? __ldg(g + j) : 1.f) * v[j];
+                  v[j + 1] = xf.y + (g != nullptr ? __ldg(g + j + 1) : 1.f) * v[j + 1];
+                }
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < col_end) v[j] = __bfloat162float(rr[j]) + (g != nullptr ? __ldg(g + j) : 1.f) * v[j];
+            }
+          }
+        }
+        if (full32) {
           uint4* dst = reinterpret_cast<uint4*>(crow + col0);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int q = 0; q < 4; ++q) {
             uint4 pk;
-            pk.x = pack_bf16x2(__uint_as_float(r[v * 8 + 0]), __uint_as_float(r[v * 8 + 1]));
-            pk.y = pack_bf16x2(__uint_as_float(r[v * 8 + 2]), __uint_as_float(r[v * 8 + 3]));
-            pk.z = pack_bf16x2(__uint_as_float(r[v * 8 + 4]), __uint_as_float(r[v * 8 + 5]));
-            pk.w = pack_bf16x2(__uint_as_float(r[v * 8 + 6]), __uint_as_float(r[v * 8 + 7]));
-            dst[v] = pk;
+            pk.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+            pk.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+            pk.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+            pk.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+            dst[q] = pk;
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (col0 + j < col_end) crow[col0 + j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+            if (col0 + j < col_end) crow[col0 + j] = __float2bfloat16_rn(v[j]);
         }
         if (p.delta != nullptr && col0 < p.dt_col0 + p.dt_cols && col0 + 32 > p.dt_col0) {
 #pragma unroll

@@ -21,6 +21,7 @@
 #include "locality.cuh"
 #include "mamba_extras.cuh"
 #include "ssd_backward.cuh"
+#include "dit.cuh"
 
 using namespace mate;
 
@@ -113,15 +114,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D bf16 matrix [rows, cols] with row stride ld (elements); box = box_rows x 64 columns, 128B swizzle.
-bool make_tmap(CUtensorMap* m, const void* ptr, long long rows, long long cols, long long ld, int box_rows) {
+// 2D matrix of 2-byte elements [rows, cols] with row stride ld (elements); box = box_rows x 64 columns,
+// 128B swizzle.  The copy does not convert; the type only names the element (bf16 unless fp16 is given).
+bool make_tmap(CUtensorMap* m, const void* ptr, long long rows, long long cols, long long ld, int box_rows,
+               CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+  return fn(m, type, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -174,9 +177,10 @@ struct Carver {
 };
 
 struct SsdScratch {
-  __nv_bfloat16 *Gm, *Sf, *Sb, *Hf, *Hb;
+  __half* Gm;
+  float *Sf, *Sb, *Srb;      // fp32 chunk states
+  __nv_bfloat16 *Hf, *Hb;    // carried states as bf16 hi | lo pairs
   float *gl, *glb, *Gd, *tbl;
-  __nv_bfloat16* Srb;
   int* crow;
 };
 
@@ -187,14 +191,14 @@ SsdScratch carve_ssd(Carver& cv, int B, long long n, int R, int nh, bool per_dir
   SsdScratch s;
   const int nRc = ceil_div(R, kSsdQ), nVc = ceil_div(n, kSsdQ);
   const size_t PN = (size_t)kSsdP * kSsdN;
-  s.Gm = cv.take<__nv_bfloat16>((size_t)B * nVc * kSsdQ * kSsdQ);
-  s.Sf = cv.take<__nv_bfloat16>((size_t)B * (nRc + nVc) * nh * PN);
-  s.Sb = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
-  s.Hf = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
-  s.Hb = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * PN);
+  s.Gm = cv.take<__half>((size_t)B * nVc * kSsdQ * kSsdQ);
+  s.Sf = cv.take<float>((size_t)B * (nRc + nVc) * nh * PN);
+  s.Sb = cv.take<float>((size_t)B * nVc * nh * PN);
+  s.Hf = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * 2 * PN);
+  s.Hb = cv.take<__nv_bfloat16>((size_t)B * nVc * nh * 2 * PN);
   s.gl = cv.take<float>((size_t)B * (nRc + nVc) * nh);
   s.glb = per_dir ? cv.take<float>((size_t)B * (nRc + nVc) * nh) : nullptr;
-  s.Srb = per_dir ? cv.take<__nv_bfloat16>((size_t)B * nRc * nh * PN) : nullptr;
+  s.Srb = per_dir ? cv.take<float>((size_t)B * nRc * nh * PN) : nullptr;
   s.Gd = cv.take<float>((size_t)B * nVc * kSsdQ);
   s.tbl = cv.take<float>((size_t)B * nVc * nh * 2 * kOutTbl);
   s.crow = cv.take<int>((size_t)B * nVc * kSsdQ);
@@ -260,7 +264,7 @@ int choose_bn(int N) { return N >= 256 ? 256 : ((N + 15) / 16) * 16; }
 
 mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const void* Bw, int ldb, int N, void* C,
                       int ldc, float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias,
-                      cudaStream_t st, const float* dt_bias2 = nullptr) {
+                      cudaStream_t st, const float* dt_bias2 = nullptr, const GemmEpilogue* ep = nullptr) {
   if (M <= 0) return MATE_OK;
   if (K % kGemmBK) return MATE_ERR_UNSUPPORTED;
   GemmParams p;
@@ -277,6 +281,7 @@ mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const
   p.dt_cols = dt_cols;
   p.dt_bias = dt_bias;
   p.dt_bias2 = dt_bias2;
+  if (ep != nullptr) p.ep = *ep;
   // 256-row tiles computed by 2-CTA clusters (tcgen05 cta_group::2)
   p.num_tiles = ceil_div(M, 256) * p.num_n_tiles;
   const uint32_t psb = gemm_pair_stage_bytes(p.bn);
@@ -294,12 +299,13 @@ mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const
 
 mate_status gemm_f32(int kid, const float* A, int lda, long long M, int K, const float* Bw, int ldb, int N, float* C,
                      int ldc, float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias,
-                     cudaStream_t st, const float* dt_bias2 = nullptr) {
+                     cudaStream_t st, const float* dt_bias2 = nullptr, const GemmEpilogue* ep = nullptr) {
   if (M <= 0) return MATE_OK;
   dim3 grid(ceil_div(N, 64), ceil_div(M, 64));
+  const GemmEpilogue e = ep != nullptr ? *ep : GemmEpilogue{};
   trace_begin(kid, st);
   gemm_f32_kernel<<<grid, 256, 0, st>>>(A, lda, Bw, ldb, C, ldc, static_cast<int>(M), N, K, delta, ld_delta, dt_col0,
-                                        dt_cols, dt_bias, dt_bias2);
+                                        dt_cols, dt_bias, dt_bias2, e);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }
@@ -402,11 +408,11 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   SsdOutMaps mp;
   const long long vrows = (long long)c->B * rows.v_bstride;
   mp.rows = static_cast<int>(vrows);
-  const long long srows = (long long)c->B * p.nVc * c->nh * kSsdN;
+  const long long srows = (long long)c->B * p.nVc * c->nh * 2 * kSsdN;   // hi | lo rows of every state
   if (!make_tmap(&mp.x, rows.xv, vrows, (long long)c->nh * c->P, rows.ldxv, 1) ||
       !make_tmap(&mp.c, rows.cv, vrows, c->N, rows.ldcv, 1) || !make_tmap(&mp.hf, sc.Hf, srows, kSsdP, kSsdP, 128) ||
       !make_tmap(&mp.hb, sc.Hb, srows, kSsdP, kSsdP, 128) ||
-      !make_tmap(&mp.g, sc.Gm, (long long)c->B * p.nVc * kSsdQ, kSsdQ, kSsdQ, 128))
+      !make_tmap(&mp.g, sc.Gm, (long long)c->B * p.nVc * kSsdQ, kSsdQ, kSsdQ, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MATE_ERR_CUDA;
   const int out_groups = c->B * p.nVc * 2;
   trace_begin(MATE_K_SSD_OUTPUT, st);
@@ -463,12 +469,19 @@ mate_status run_tesa(const mate_config* c, const void* qkv, int ldq, int qcol, i
 // Host input and output of mate_forward_host, moved in row chunks on two copy streams so that the
 // host-to-device copy overlaps the in-projection of the chunks already landed and the device-to-host copy
 // overlaps the out-projection of the later chunks.  One set per device; the mutex keeps one call's
-// sequence of event records and waits together.
+// sequence of event records and waits together.  Pipelined calls alternate between two device input
+// slots; per slot the ring remembers the workspace and Out_host range of the last call that used it, the
+// event after which that call no longer reads its input slot, and the event of its last output copy.
 constexpr int kIoChunks = 4;
 struct HostIo {
   std::mutex mu;
   cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t start = nullptr, done = nullptr, in_ready[kIoChunks] = {}, out_ready[kIoChunks] = {};
+  cudaEvent_t start = nullptr, in_ready[kIoChunks] = {}, out_ready[kIoChunks] = {};
+  cudaEvent_t done[2] = {}, x_free[2] = {};
+  const void* slot_ws[2] = {};
+  uintptr_t out_lo[2] = {}, out_hi[2] = {};
+  bool pending[2] = {};   // a pipelined call's output copy that no stream has been made to wait for yet
+  long long calls = 0;
   bool ready = false, failed = false;
 };
 HostIo g_io[kMaxDevices];
@@ -484,8 +497,10 @@ HostIo* host_io() {
   if (!io.ready && !io.failed) {
     bool ok = cudaStreamCreateWithFlags(&io.h2d, cudaStreamNonBlocking) == cudaSuccess &&
               cudaStreamCreateWithFlags(&io.d2h, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaEventCreateWithFlags(&io.start, cudaEventDisableTiming) == cudaSuccess &&
-              cudaEventCreateWithFlags(&io.done, cudaEventDisableTiming) == cudaSuccess;
+              cudaEventCreateWithFlags(&io.start, cudaEventDisableTiming) == cudaSuccess;
+    for (int k = 0; ok && k < 2; ++k)
+      ok = cudaEventCreateWithFlags(&io.done[k], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&io.x_free[k], cudaEventDisableTiming) == cudaSuccess;
     for (int k = 0; ok && k < kIoChunks; ++k)
       ok = cudaEventCreateWithFlags(&io.in_ready[k], cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&io.out_ready[k], cudaEventDisableTiming) == cudaSuccess;
@@ -564,6 +579,7 @@ struct IoPlan {
   char* out_host;
   long long rows, chunk_rows;   // chunk c covers rows [c * chunk_rows, min(rows, (c + 1) * chunk_rows))
   size_t row_bytes;
+  cudaEvent_t x_free;           // recorded on the call's stream once the device input is no longer read
 };
 
 bool cuda_ok(cudaError_t e) {
@@ -572,8 +588,34 @@ bool cuda_ok(cudaError_t e) {
   return false;
 }
 
+// Byte offset of the packed out-projection [W_out | W_o] inside a mate_pack_weights buffer.
+size_t packed_out_offset(const mate_config* c) {
+  const ForwardPlan p = plan_forward(c, nullptr);
+  return ((size_t)p.NI * c->d * elem_size(c) + 255) & ~size_t(255);
+}
+
+size_t packed_bytes(const mate_config* c) {
+  const ForwardPlan p = plan_forward(c, nullptr);
+  return packed_out_offset(c) + (size_t)c->d * p.KO * elem_size(c);
+}
+
+// [W_in; W_qkv (; W_z)] into Wi (NI x d) and [W_out | W_o] into Wo (d x KO).
+mate_status pack_weights(const mate_weights* w, const mate_config* c, void* Wi, void* Wo, cudaStream_t st) {
+  const ForwardPlan pl = plan_forward(c, nullptr);
+  const size_t es = elem_size(c);
+  const int dI = c->nh * c->P;
+  MATE_TRY(copy_block(w->W_in, Wi, pl.NIn, c->d, c->d, 0, 0, es, st));
+  MATE_TRY(copy_block(w->W_qkv, Wi, 3 * c->th * c->tp, c->d, c->d, pl.NIn, 0, es, st));
+  if (c->mamba_extras) MATE_TRY(copy_block(w->W_z, Wi, dI, c->d, c->d, pl.zc0, 0, es, st));
+  MATE_TRY(copy_block(w->W_out, Wo, c->d, dI, pl.KO, 0, 0, es, st));
+  MATE_TRY(copy_block(w->W_o, Wo, c->d, c->th * c->tp, pl.KO, 0, dI, es, st));
+  return MATE_OK;
+}
+
+// out_ep: optional epilogue of the out-projection (the DiT block's gated residual around the mixer).
 mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, void* Out, const mate_config* c,
-                         void* ws, size_t ws_bytes, cudaStream_t st, const IoPlan* iop = nullptr) {
+                         void* ws, size_t ws_bytes, cudaStream_t st, const IoPlan* iop = nullptr,
+                         const GemmEpilogue* out_ep = nullptr) {
   MATE_TRY(check_config(c));
   if (X == nullptr || w == nullptr || Out == nullptr || ws == nullptr || layer_idx < 0) return MATE_ERR_ARG;
   if (w->W_in == nullptr || w->dt_bias == nullptr || w->A_log == nullptr || w->D == nullptr || w->W_out == nullptr ||
@@ -604,12 +646,15 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   const int ldd = per_dir ? 2 * c->nh : c->nh;                     // delta rows: forward | backward
   const float* dtb2 = per_dir ? w->dt_bias_b : nullptr;
 
-  // packed weights: Wi = [W_in; W_qkv] (NI x d), Wo = [W_out | W_o] (d x KO)
-  MATE_TRY(copy_block(w->W_in, pl.Wi, NIn, c->d, c->d, 0, 0, es, st));
-  MATE_TRY(copy_block(w->W_qkv, pl.Wi, 3 * c->th * c->tp, c->d, c->d, NIn, 0, es, st));
-  if (extras) MATE_TRY(copy_block(w->W_z, pl.Wi, dI, c->d, c->d, pl.zc0, 0, es, st));
-  MATE_TRY(copy_block(w->W_out, pl.Wo, c->d, dI, KO, 0, 0, es, st));
-  MATE_TRY(copy_block(w->W_o, pl.Wo, c->d, c->th * c->tp, KO, 0, dI, es, st));
+  // packed weights: Wi = [W_in; W_qkv (; W_z)] (NI x d), Wo = [W_out | W_o] (d x KO), from the caller's
+  // mate_pack_weights buffer when given, else packed into the workspace on every call
+  if (w->packed != nullptr) {
+    if (!aligned16(w->packed)) return MATE_ERR_ARG;
+    pl.Wi = const_cast<void*>(w->packed);
+    pl.Wo = static_cast<char*>(pl.Wi) + packed_out_offset(c);
+  } else {
+    MATE_TRY(pack_weights(w, c, pl.Wi, pl.Wo, st));
+  }
   // review tokens, then the projections of the video rows (grid order) and of the review rows
   if (c->dtype == MATE_BF16 && iop != nullptr) {
     // host input: project each row chunk as soon as it has landed; the review pool needs all of X
@@ -622,6 +667,7 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
                          c->nh, w->dt_bias, st, dtb2));
     }
     MATE_TRY(pool(X, pl.Rv, c, order, st));
+    if (!cuda_ok(cudaEventRecord(iop->x_free, st))) return MATE_ERR_CUDA;
     MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
   } else if (c->dtype == MATE_BF16) {
     MATE_TRY(pool(X, pl.Rv, c, order, st));
@@ -717,10 +763,11 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
         return MATE_ERR_CUDA;
     }
   } else if (c->dtype == MATE_BF16)
-    MATE_TRY(gemm_bf16(MATE_K_OUT_PROJ, pl.YO, KO, Mv, KO, pl.Wo, KO, c->d, Out, c->d, nullptr, 0, 0, 0, nullptr, st));
+    MATE_TRY(gemm_bf16(MATE_K_OUT_PROJ, pl.YO, KO, Mv, KO, pl.Wo, KO, c->d, Out, c->d, nullptr, 0, 0, 0, nullptr, st,
+                       nullptr, out_ep));
   else
     MATE_TRY(gemm_f32(MATE_K_OUT_PROJ, static_cast<const float*>(pl.YO), KO, Mv, KO, static_cast<const float*>(pl.Wo), KO, c->d,
-                      static_cast<float*>(Out), c->d, nullptr, 0, 0, 0, nullptr, st));
+                      static_cast<float*>(Out), c->d, nullptr, 0, 0, 0, nullptr, st, nullptr, out_ep));
   return MATE_OK;
 }
 
@@ -762,7 +809,8 @@ size_t mate_ssd_pd_workspace_bytes(const mate_config* cfg, int prefix_len) {
 size_t mate_forward_host_workspace_bytes(const mate_config* cfg) {
   if (check_config(cfg) != MATE_OK) return 0;
   const size_t xb = (size_t)cfg->B * cfg->T * cfg->H * cfg->W * cfg->d * elem_size(cfg);
-  return mate_workspace_bytes(cfg) + 2 * ((xb + 255) & ~size_t(255));
+  // the block's workspace, two device input slots and two device output slots (pipelined calls alternate)
+  return mate_workspace_bytes(cfg) + 4 * ((xb + 255) & ~size_t(255));
 }
 
 mate_status rms_permute(const void* X, void* Xp, int order, const mate_config* cfg, mate_stream_t stream) {
@@ -912,13 +960,35 @@ mate_status ssd_scan_bidir_backward(const void* x, const void* Bm, const void* C
 }
 
 // Fixed scratch behind ssd_scan_bidir_noalloc.  In host code this name is only a stand-in for the
-// device symbol; its device address comes from cudaGetSymbolAddress, once per device.
+// device symbol; its device address comes from cudaGetSymbolAddress, once per device and CUDA context.
 static __device__ __align__(256) unsigned char g_ssd_noalloc_scratch[MATE_SSD_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 constexpr int kNoallocMaxDevices = 128;
 std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kNoallocMaxDevices];  // device address of the scratch, by device ordinal
+// Device address of the scratch by device ordinal, with the CUDA context it was looked up in: the array
+// lives in the library's device code loaded into that context, so after cudaDeviceReset (a new context)
+// the address is looked up again.
+struct NoallocAddr {
+  CUcontext ctx;
+  void* addr;
+};
+NoallocAddr g_noalloc_addr[kNoallocMaxDevices];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
 }  // namespace
 
 mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const void* Cm, const float* dt,
@@ -928,6 +998,9 @@ mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const void* Cm
   if (prefix_len < 0) return MATE_ERR_ARG;
   if (ssd_ws_bytes(cfg, prefix_len, false, nullptr, nullptr, nullptr) > MATE_SSD_NOALLOC_SCRATCH_BYTES)
     return MATE_ERR_TOO_LARGE;
+  if (x == nullptr || Bm == nullptr || Cm == nullptr || dt == nullptr || dt_bias == nullptr || A_log == nullptr ||
+      D == nullptr || y == nullptr)
+    return MATE_ERR_ARG;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) {
     cudaGetLastError();
@@ -936,15 +1009,20 @@ mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const void* Cm
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_addr[dev] == nullptr) {
+    // cudaGetSymbolAddress also makes the context current and loads the device code if needed, so the
+    // context is read after it on the first call
+    const CUcontext ctx = current_context();
+    NoallocAddr& na = g_noalloc_addr[dev];
+    if (na.addr == nullptr || ctx == nullptr || na.ctx != ctx) {
       void* addr = nullptr;
       if (cudaGetSymbolAddress(&addr, g_ssd_noalloc_scratch) != cudaSuccess || addr == nullptr) {
         cudaGetLastError();
         return MATE_ERR_CUDA;
       }
-      g_noalloc_addr[dev] = addr;
+      na.addr = addr;
+      na.ctx = current_context();
     }
-    scratch = g_noalloc_addr[dev];
+    scratch = na.addr;
   }
   return ssd_scan_bidir(x, Bm, Cm, dt, dt_bias, A_log, D, prefix_len, y, cfg, scratch, MATE_SSD_NOALLOC_SCRATCH_BYTES,
                         stream);
@@ -998,25 +1076,40 @@ mate_status mate_forward(const void* X, const mate_weights* w, int layer_idx, vo
   return forward_impl(X, w, layer_idx, Out, cfg, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
-mate_status mate_forward_host(const void* X_host, const mate_weights* w, int layer_idx, void* Out_host,
-                              const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream) {
+}  // extern "C"
+
+namespace {
+bool ranges_overlap(uintptr_t a0, uintptr_t a1, uintptr_t b0, uintptr_t b1) { return a0 < b1 && b0 < a1; }
+
+mate_status forward_host_impl(const void* X_host, const mate_weights* w, int layer_idx, void* Out_host,
+                              const mate_config* cfg, void* ws, size_t ws_bytes, cudaStream_t st, bool pipelined) {
   MATE_TRY(check_config(cfg));
   if (X_host == nullptr || Out_host == nullptr || ws == nullptr) return MATE_ERR_ARG;
   if (ws_bytes < mate_forward_host_workspace_bytes(cfg)) return MATE_ERR_WORKSPACE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t fw = mate_workspace_bytes(cfg);
   const size_t xb = (size_t)cfg->B * cfg->T * cfg->H * cfg->W * cfg->d * elem_size(cfg);
-  char* xdev = static_cast<char*>(ws) + ((fw + 255) & ~size_t(255));
-  char* odev = xdev + ((xb + 255) & ~size_t(255));
+  const size_t xb_al = (xb + 255) & ~size_t(255);
+  char* xslot0 = static_cast<char*>(ws) + ((fw + 255) & ~size_t(255));
   t_launches = 0;
   HostIo* io = cfg->dtype == MATE_BF16 ? host_io() : nullptr;
   if (io == nullptr) {   // one copy each way on `stream`
-    if (cudaMemcpyAsync(xdev, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MATE_ERR_CUDA;
-    MATE_TRY(forward_impl(xdev, w, layer_idx, odev, cfg, ws, fw, st));
+    char* odev = xslot0 + 2 * xb_al;
+    if (cudaMemcpyAsync(xslot0, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MATE_ERR_CUDA;
+    MATE_TRY(forward_impl(xslot0, w, layer_idx, odev, cfg, ws, fw, st));
     if (cudaMemcpyAsync(Out_host, odev, xb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MATE_ERR_CUDA;
     return MATE_OK;
   }
   std::lock_guard<std::mutex> lock(io->mu);
+  const int slot = pipelined ? static_cast<int>(io->calls & 1) : 0;
+  char* xdev = xslot0 + slot * xb_al;
+  char* odev = xslot0 + (2 + slot) * xb_al;
+  if (!pipelined) {   // no earlier pipelined output copy may still be running when this call starts
+    for (int j = 0; j < 2; ++j)
+      if (io->pending[j]) {
+        if (!cuda_ok(cudaStreamWaitEvent(st, io->done[j], 0))) return MATE_ERR_CUDA;
+        io->pending[j] = false;
+      }
+  }
   IoPlan iop;
   iop.io = io;
   iop.x_host = static_cast<const char*>(X_host);
@@ -1024,10 +1117,23 @@ mate_status mate_forward_host(const void* X_host, const mate_weights* w, int lay
   iop.rows = (long long)cfg->B * cfg->T * cfg->H * cfg->W;
   iop.row_bytes = (size_t)cfg->d * elem_size(cfg);
   iop.chunk_rows = ((iop.rows + kIoChunks - 1) / kIoChunks + 255) / 256 * 256;
-  // both copy streams start after all earlier work on `stream` (the workspace may still be in use)
-  if (!cuda_ok(cudaEventRecord(io->start, st)) || !cuda_ok(cudaStreamWaitEvent(io->h2d, io->start, 0)) ||
-      !cuda_ok(cudaStreamWaitEvent(io->d2h, io->start, 0)))
-    return MATE_ERR_CUDA;
+  iop.x_free = io->x_free[slot];
+  const uintptr_t x0 = reinterpret_cast<uintptr_t>(X_host), o0 = reinterpret_cast<uintptr_t>(Out_host);
+  if (!pipelined || io->slot_ws[slot] != ws) {
+    // the copies start after all earlier work on `stream` (the workspace may still be in use)
+    if (!cuda_ok(cudaEventRecord(io->start, st)) || !cuda_ok(cudaStreamWaitEvent(io->h2d, io->start, 0)) ||
+        !cuda_ok(cudaStreamWaitEvent(io->d2h, io->start, 0)))
+      return MATE_ERR_CUDA;
+  } else {
+    // the input copy waits only until the call that last used this input slot has read it, and for the
+    // output copies of earlier calls whose Out_host overlaps X_host; everything else of the previous call
+    // (its output copies included) may still run
+    if (!cuda_ok(cudaStreamWaitEvent(io->h2d, io->x_free[slot], 0))) return MATE_ERR_CUDA;
+    for (int j = 0; j < 2; ++j)
+      if (ranges_overlap(x0, x0 + xb, io->out_lo[j], io->out_hi[j]) &&
+          !cuda_ok(cudaStreamWaitEvent(io->h2d, io->done[j], 0)))
+        return MATE_ERR_CUDA;
+  }
   for (int k = 0; k < kIoChunks; ++k) {
     const long long r0 = k * iop.chunk_rows, r1 = std::min(iop.rows, r0 + iop.chunk_rows);
     if (r1 > r0 && !cuda_ok(cudaMemcpyAsync(xdev + r0 * iop.row_bytes, iop.x_host + r0 * iop.row_bytes,
@@ -1036,18 +1142,209 @@ mate_status mate_forward_host(const void* X_host, const mate_weights* w, int lay
     if (!cuda_ok(cudaEventRecord(io->in_ready[k], io->h2d))) return MATE_ERR_CUDA;
   }
   MATE_TRY(forward_impl(xdev, w, layer_idx, odev, cfg, ws, fw, st, &iop));
-  // the call ends on `stream` only when the last chunk has reached the host
-  if (!cuda_ok(cudaEventRecord(io->done, io->d2h)) || !cuda_ok(cudaStreamWaitEvent(st, io->done, 0)))
+  if (!cuda_ok(cudaEventRecord(io->done[slot], io->d2h))) return MATE_ERR_CUDA;
+  if (!pipelined) {
+    // the call ends on `stream` only when the last chunk has reached the host
+    if (!cuda_ok(cudaStreamWaitEvent(st, io->done[slot], 0))) return MATE_ERR_CUDA;
+  } else {
+    // this call's output copy runs on beside the next call's work; the stream waits here for the previous
+    // call's output copy (whose device output slot the next call overwrites)
+    const int prev = slot ^ 1;
+    if (io->pending[prev]) {
+      if (!cuda_ok(cudaStreamWaitEvent(st, io->done[prev], 0))) return MATE_ERR_CUDA;
+      io->pending[prev] = false;
+    }
+    io->pending[slot] = true;
+  }
+  io->slot_ws[slot] = ws;
+  io->out_lo[slot] = o0;
+  io->out_hi[slot] = o0 + xb;
+  ++io->calls;
+  return MATE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+mate_status mate_forward_host(const void* X_host, const mate_weights* w, int layer_idx, void* Out_host,
+                              const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream) {
+  return forward_host_impl(X_host, w, layer_idx, Out_host, cfg, ws, ws_bytes,
+                           reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+mate_status mate_forward_host_pipelined(const void* X_host, const mate_weights* w, int layer_idx, void* Out_host,
+                                        const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream) {
+  return forward_host_impl(X_host, w, layer_idx, Out_host, cfg, ws, ws_bytes,
+                           reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+mate_status mate_forward_host_flush(mate_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
     return MATE_ERR_CUDA;
+  }
+  HostIo& io = g_io[dev];
+  std::lock_guard<std::mutex> lock(io.mu);
+  if (!io.ready) return MATE_OK;
+  for (int j = 0; j < 2; ++j)
+    if (io.pending[j]) {
+      if (!cuda_ok(cudaStreamWaitEvent(st, io.done[j], 0))) return MATE_ERR_CUDA;
+      io.pending[j] = false;
+    }
+  return MATE_OK;
+}
+
+size_t mate_packed_weights_bytes(const mate_config* cfg) {
+  if (check_config(cfg) != MATE_OK) return 0;
+  return packed_bytes(cfg);
+}
+
+mate_status mate_pack_weights(const mate_weights* w, const mate_config* cfg, void* packed, size_t packed_bytes_,
+                              mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (w == nullptr || packed == nullptr || !aligned16(packed) || w->W_in == nullptr || w->W_out == nullptr ||
+      w->W_qkv == nullptr || w->W_o == nullptr || !aligned16(w->W_in) || !aligned16(w->W_out) ||
+      !aligned16(w->W_qkv) || !aligned16(w->W_o))
+    return MATE_ERR_ARG;
+  if (cfg->mamba_extras && (w->W_z == nullptr || !aligned16(w->W_z))) return MATE_ERR_ARG;
+  if (packed_bytes_ < packed_bytes(cfg)) return MATE_ERR_WORKSPACE;
+  t_launches = 0;
+  return pack_weights(w, cfg, packed, static_cast<char*>(packed) + packed_out_offset(cfg),
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+struct DitPlan {
+  float* mod;   // [B][6][d] modulation
+  void *h, *X1, *Z;
+  void* mate_ws;
+  size_t mate_bytes, bytes;
+};
+
+DitPlan plan_dit(const mate_config* c, void* ws) {
+  DitPlan p;
+  Carver cv{static_cast<char*>(ws)};
+  const size_t es = elem_size(c);
+  const size_t rows = (size_t)c->B * c->T * c->H * c->W;
+  p.mod = cv.take<float>((size_t)c->B * 6 * c->d);
+  p.h = cv.take<char>(rows * c->d * es);
+  p.X1 = cv.take<char>(rows * c->d * es);
+  p.Z = cv.take<char>(rows * 4 * c->d * es);
+  p.mate_bytes = plan_forward(c, nullptr).bytes;
+  p.mate_ws = cv.take<char>(p.mate_bytes);
+  p.bytes = cv.off + 256;
+  return p;
+}
+
+mate_status ln_modulate(const mate_config* c, const void* x, void* h, const float* shift, const float* scale,
+                        cudaStream_t st) {
+  const long long n = (long long)c->T * c->H * c->W, rows = (long long)c->B * n;
+  const int blocks = static_cast<int>((rows + 7) / 8);
+  trace_begin(MATE_K_LN_MODULATE, st);
+  if (c->dtype == MATE_BF16)
+    ln_modulate_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                                  static_cast<__nv_bfloat16*>(h), rows, c->d, n, shift,
+                                                                  scale);
+  else
+    ln_modulate_kernel<float, 4><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), static_cast<float*>(h), rows,
+                                                          c->d, n, shift, scale);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t mate_dit_workspace_bytes(const mate_config* cfg) {
+  if (check_config(cfg) != MATE_OK || cfg->d > 2048) return 0;
+  return plan_dit(cfg, nullptr).bytes;
+}
+
+mate_status mate_dit_block_forward(const void* X, const float* c, int dc, const mate_dit_weights* dw,
+                                   const mate_weights* mw, int layer_idx, void* Out, const mate_config* cfg, void* ws,
+                                   size_t ws_bytes, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (cfg->d > 2048) return MATE_ERR_UNSUPPORTED;
+  if (X == nullptr || c == nullptr || dc <= 0 || dw == nullptr || mw == nullptr || Out == nullptr || ws == nullptr ||
+      layer_idx < 0 || dw->W_ada == nullptr || dw->b_ada == nullptr || dw->W1 == nullptr || dw->b1 == nullptr ||
+      dw->W2 == nullptr || dw->b2 == nullptr)
+    return MATE_ERR_ARG;
+  if (!aligned16(X) || !aligned16(Out) || !aligned16(ws) || !aligned16(dw->W1) || !aligned16(dw->W2) ||
+      !aligned16(dw->b1) || !aligned16(dw->b2))
+    return MATE_ERR_ARG;
+  if (X == Out) return MATE_ERR_ARG;
+  DitPlan pl = plan_dit(cfg, nullptr);
+  if (ws_bytes < pl.bytes) return MATE_ERR_WORKSPACE;
+  pl = plan_dit(cfg, ws);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  const int d = cfg->d;
+  const long long n = (long long)cfg->T * cfg->H * cfg->W, rows = (long long)cfg->B * n;
+  // modulation vectors of every sample
+  {
+    const long long warps = (long long)cfg->B * 6 * d;
+    trace_begin(MATE_K_ADA_MODULATION, st);
+    if (cfg->dtype == MATE_BF16)
+      ada_modulation_kernel<__nv_bfloat16><<<static_cast<int>((warps + 7) / 8), 256, 0, st>>>(
+          c, dc, static_cast<const __nv_bfloat16*>(dw->W_ada), dw->b_ada, pl.mod, 6 * d, cfg->B);
+    else
+      ada_modulation_kernel<float><<<static_cast<int>((warps + 7) / 8), 256, 0, st>>>(
+          c, dc, static_cast<const float*>(dw->W_ada), dw->b_ada, pl.mod, 6 * d, cfg->B);
+    MATE_LAUNCH_CHECK();
+  }
+  const float *shift_a = pl.mod, *scale_a = pl.mod + d, *gate_a = pl.mod + 2 * d;
+  const float *shift_m = pl.mod + 3 * d, *scale_m = pl.mod + 4 * d, *gate_m = pl.mod + 5 * d;
+  // X1 = X + gate_a * MATE(LN(X) (1 + scale_a) + shift_a): the gated residual in the out-projection's epilogue
+  MATE_TRY(ln_modulate(cfg, X, pl.h, shift_a, scale_a, st));
+  GemmEpilogue mix_ep;
+  mix_ep.resid = X;
+  mix_ep.ld_resid = d;
+  mix_ep.gate = gate_a;
+  mix_ep.ld_gate = 6 * d;
+  mix_ep.gate_rows = static_cast<int>(n);
+  MATE_TRY(forward_impl(pl.h, mw, layer_idx, pl.X1, cfg, pl.mate_ws, pl.mate_bytes, st, nullptr, &mix_ep));
+  // Out = X1 + gate_m * MLP(LN(X1) (1 + scale_m) + shift_m)
+  MATE_TRY(ln_modulate(cfg, pl.X1, pl.h, shift_m, scale_m, st));
+  GemmEpilogue up_ep;
+  up_ep.bias = dw->b1;
+  up_ep.act = 1;
+  GemmEpilogue down_ep;
+  down_ep.bias = dw->b2;
+  down_ep.resid = pl.X1;
+  down_ep.ld_resid = d;
+  down_ep.gate = gate_m;
+  down_ep.ld_gate = 6 * d;
+  down_ep.gate_rows = static_cast<int>(n);
+  if (cfg->dtype == MATE_BF16) {
+    MATE_TRY(gemm_bf16(MATE_K_MLP_UP, pl.h, d, rows, d, dw->W1, d, 4 * d, pl.Z, 4 * d, nullptr, 0, 0, 0, nullptr, st,
+                       nullptr, &up_ep));
+    MATE_TRY(gemm_bf16(MATE_K_MLP_DOWN, pl.Z, 4 * d, rows, 4 * d, dw->W2, 4 * d, d, Out, d, nullptr, 0, 0, 0, nullptr,
+                       st, nullptr, &down_ep));
+  } else {
+    MATE_TRY(gemm_f32(MATE_K_MLP_UP, static_cast<const float*>(pl.h), d, rows, d, static_cast<const float*>(dw->W1), d,
+                      4 * d, static_cast<float*>(pl.Z), 4 * d, nullptr, 0, 0, 0, nullptr, st, nullptr, &up_ep));
+    MATE_TRY(gemm_f32(MATE_K_MLP_DOWN, static_cast<const float*>(pl.Z), 4 * d, rows, 4 * d,
+                      static_cast<const float*>(dw->W2), 4 * d, d, static_cast<float*>(Out), d, nullptr, 0, 0, 0,
+                      nullptr, st, nullptr, &down_ep));
+  }
   return MATE_OK;
 }
 
 mate_status mate_device_status(mate_stream_t stream, unsigned int* flags) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return MATE_ERR_CUDA;
-  unsigned int v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(v)) != cudaSuccess) return MATE_ERR_CUDA;
-  if (cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(zero)) != cudaSuccess) return MATE_ERR_CUDA;
+  // read and clear in one atomic exchange on the device, so that a flag set meanwhile by a kernel on
+  // another stream is either returned now or kept for the next call, never lost
+  status_take_kernel<<<1, 1, 0, st>>>();
+  unsigned int v = 0;
+  if (!cuda_ok(cudaGetLastError()) ||
+      !cuda_ok(cudaMemcpyFromSymbolAsync(&v, g_dev_status_taken, sizeof(v), 0, cudaMemcpyDeviceToHost, st)) ||
+      !cuda_ok(cudaStreamSynchronize(st)))
+    return MATE_ERR_CUDA;
   if (flags) *flags = v;
   return v ? MATE_ERR_TIMEOUT : MATE_OK;
 }
@@ -1131,6 +1428,10 @@ const char* mate_kernel_name(int kernel) {
     case MATE_K_GATE_NORM: return "gate_rmsnorm";
     case MATE_K_SSD_BACKWARD: return "ssd_backward_f32";
     case MATE_K_SELFTEST: return "selftest_wait_timeout";
+    case MATE_K_ADA_MODULATION: return "ada_modulation";
+    case MATE_K_LN_MODULATE: return "ln_modulate";
+    case MATE_K_MLP_UP: return "mlp_up";
+    case MATE_K_MLP_DOWN: return "mlp_down";
   }
   return "unknown";
 }

@@ -5,6 +5,7 @@
 //   * small helpers (weight packing, softplus of raw step sizes).
 #pragma once
 #include "common.cuh"
+#include "gemm_bf16.cuh"
 
 namespace mate {
 
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
                                                        int ldb, float* __restrict__ C, int ldc, int M, int N, int K,
                                                        float* __restrict__ delta, int ld_delta, int dt_col0,
                                                        int dt_cols, const float* __restrict__ dt_bias,
-                                                       const float* __restrict__ dt_bias2) {
+                                                       const float* __restrict__ dt_bias2, const GemmEpilogue ep) {
   __shared__ float As[16][65];
   __shared__ float Bs[16][65];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -168,7 +169,13 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
     for (int c = 0; c < 4; ++c) {
       const int col = n0 + tx * 4 + c;
       if (col >= N) continue;
-      C[(long long)r * ldc + col] = acc[a][c];
+      float v = acc[a][c];
+      if (ep.bias != nullptr) v += ep.bias[col];
+      if (ep.act == 1) v = gelu_tanh_f<false>(v);
+      if (ep.resid != nullptr)
+        v = static_cast<const float*>(ep.resid)[(long long)r * ep.ld_resid + col] +
+            (ep.gate != nullptr ? ep.gate[(long long)(r / ep.gate_rows) * ep.ld_gate + col] : 1.f) * v;
+      C[(long long)r * ldc + col] = v;
       if (delta != nullptr && col >= dt_col0 && col < dt_col0 + dt_cols) {
         const float v = acc[a][c] + dt_bias[col - dt_col0];
         delta[(long long)r * ld_delta + col - dt_col0] = v > 20.f ? v : log1pf(expf(v));

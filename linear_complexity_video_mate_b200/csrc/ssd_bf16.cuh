@@ -25,6 +25,13 @@
 //                      Sb = sum_j exp(s'_j) delta_j x_j B_j^T, and s_last per (chunk, head)  [tcgen05]
 //   ssd_carry_kernel   sequential carry over chunks: H_in(next) = exp(s_last) H_in + S     [CUDA cores]
 //   ssd_output_kernel  y for one (video chunk, head): M x + row-scaled C Hf^T, C Hb^T      [tcgen05]
+//
+// Precision.  States, decays and accumulations are fp32.  The chunk states S are stored in fp32; the
+// carried states H, an operand of the C H^T product, are stored as a bf16 pair hi + lo (hi = bf16(H),
+// lo = bf16(H - hi)) and multiplied as two accumulating products, which keeps about 16 bits of H.  G and
+// the state products' operands (the decay-weighted x and B) are fp16 (11 bits), so M = G delta dec is
+// rounded once, to the bf16 MMA operand, from an fp16 G that is already 8 times finer than bf16.  fp16
+// conversions saturate at +-65504 (|C_i . B_j| and |delta_j x_j| stay far below that for these blocks).
 // Rows are gathered through the scan-order map (the permutation is done by addressing) and y is
 // stored back at grid-order rows.
 #pragma once
@@ -54,13 +61,13 @@ struct SsdBf16Params {
   int B, nh, nRc, nVc;
   const float* A_log;
   const float* Dp;
-  __nv_bfloat16* Gm;  // [B][nVc][Q][Q]  C B^T of each video chunk (off-diagonal use)
+  __half* Gm;         // [B][nVc][Q][Q]  C B^T of each video chunk in fp16 (off-diagonal use)
   float* Gd;          // [B][nVc][Q]     its diagonal C_i . B_i in fp32
-  __nv_bfloat16* Sf;  // [B][nRc + nVc][nh][N][P]   (states are stored transposed: n-major, p fastest)
-  __nv_bfloat16* Sb;  // [B][nVc][nh][N][P]
+  float* Sf;          // [B][nRc + nVc][nh][N][P]   (states are stored transposed: n-major, p fastest)
+  float* Sb;          // [B][nVc][nh][N][P]
   float* gl;          // [B][nRc + nVc][nh]  s_last of each chunk
-  __nv_bfloat16* Hf;  // [B][nVc][nh][N][P]  state entering video chunk v, forward traversal
-  __nv_bfloat16* Hb;  // [B][nVc][nh][N][P]  state entering video chunk v, backward traversal
+  __nv_bfloat16* Hf;  // [B][nVc][nh][2][N][P]  state entering video chunk v, forward traversal, as hi | lo
+  __nv_bfloat16* Hb;  // [B][nVc][nh][2][N][P]  state entering video chunk v, backward traversal, as hi | lo
   int* crow;          // [B][nVc][Q]     source row of each video-chunk row (-1 past the end)
   float* tbl;         // [B][nVc][nh][2][kOutTbl]  decay tables of each 128-row tile (layout below)
   // Optional separate parameters of the backward scan (null: shared with the forward scan).  With them,
@@ -70,7 +77,7 @@ struct SsdBf16Params {
   const float* A_log_b;
   const float* Dp_b;
   float* glb;           // [B][nRc + nVc][nh]
-  __nv_bfloat16* Srb;   // [B][nRc][nh][N][P]
+  float* Srb;           // [B][nRc][nh][N][P]
   __nv_bfloat16* y;   // row b*y_bstride + map(q), column h*P
   int ldy;
   long long y_bstride;
@@ -221,11 +228,12 @@ __global__ void __launch_bounds__(128, 1) ssd_gram_kernel(const SsdBf16Params p)
     }
     mma_commit(bar);
   }
-  mbar_wait(bar, 0);
+  // a wait that ran out (flagged in the status word) skips the read-out; the CTA still frees its TMEM
+  const bool ok = !__syncthreads_or(!mbar_wait(bar, 0));
   tc_fence_after();
   const int i = t * 128 + warp * 32 + lane;
-  __nv_bfloat16* grow = p.Gm + ((static_cast<long long>(b) * p.nVc + v) * kSsdQ + i) * kSsdQ;
-  for (int c0 = 0; c0 < 256; c0 += 32) {
+  __half* grow = p.Gm + ((static_cast<long long>(b) * p.nVc + v) * kSsdQ + i) * kSsdQ;
+  for (int c0 = 0; c0 < 256 && ok; c0 += 32) {
     uint32_t r[32];
     tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, r);
     tmem_wait_ld();
@@ -240,10 +248,10 @@ __global__ void __launch_bounds__(128, 1) ssd_gram_kernel(const SsdBf16Params p)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint4 pk;
-      pk.x = pack_bf16x2(__uint_as_float(r[q * 8 + 0]), __uint_as_float(r[q * 8 + 1]));
-      pk.y = pack_bf16x2(__uint_as_float(r[q * 8 + 2]), __uint_as_float(r[q * 8 + 3]));
-      pk.z = pack_bf16x2(__uint_as_float(r[q * 8 + 4]), __uint_as_float(r[q * 8 + 5]));
-      pk.w = pack_bf16x2(__uint_as_float(r[q * 8 + 6]), __uint_as_float(r[q * 8 + 7]));
+      pk.x = pack_f16x2_sat(__uint_as_float(r[q * 8 + 0]), __uint_as_float(r[q * 8 + 1]));
+      pk.y = pack_f16x2_sat(__uint_as_float(r[q * 8 + 2]), __uint_as_float(r[q * 8 + 3]));
+      pk.z = pack_f16x2_sat(__uint_as_float(r[q * 8 + 4]), __uint_as_float(r[q * 8 + 5]));
+      pk.w = pack_f16x2_sat(__uint_as_float(r[q * 8 + 6]), __uint_as_float(r[q * 8 + 7]));
       dst[q] = pk;
     }
   }
@@ -258,7 +266,8 @@ __global__ void __launch_bounds__(128, 1) ssd_gram_kernel(const SsdBf16Params p)
 // ---------------------------------------------------------------------------------------------------
 // Chunk-local end states.  grid (nRc + nVc, B, nh / heads_per_cta), 256 threads (thread j = token j).
 // D[n][p] = sum_j B[j][n] * (w_j x[j][p]): A operand = the B tile read MN-major, B operand = the
-// weighted x tile (MN-major), M = N_state = 128, N = P = 64, K = Q = 256.
+// weighted x tile (MN-major), M = N_state = 128, N = P = 64, K = Q = 256; both operands fp16 (the B
+// rows are converted once per chunk, the weighted x per head), states written in fp32.
 // ---------------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p, int heads_per_cta) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -287,12 +296,29 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
   if (warp == 0) tmem_alloc(slot, 128);
   fill_chunk_rows(p.s, b, c, p.nRc, srow);
   __syncthreads();
-  for (int it = threadIdx.x; it < 256 * 16; it += 256) {
-    const int r = it >> 4, ch = it & 15;
-    const long long rw = srow[r];
-    load_row128_kmajor(sB, r, cb.b + (rw < 0 ? 0 : rw) * cb.ldb, rw >= 0, 32768, ch);
+  {
+    // the chunk's B rows, bf16 -> fp16, into the K-major swizzled tile (zeros past a partial chunk's end)
+    uint4 bv[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int it = threadIdx.x + u * 256;
+      const long long rw = srow[it >> 4];
+      bv[u] = rw >= 0 ? __ldg(reinterpret_cast<const uint4*>(cb.b + rw * cb.ldb) + (it & 15)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int it = threadIdx.x + u * 256;
+      const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bv[u]);
+      uint4 o;
+      uint32_t* po = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack_bf16x2(bw[e]);
+        po[e] = pack_f16x2_sat(f.x, f.y);
+      }
+      *reinterpret_cast<uint4*>(sB + sw128_kmajor_offset(it >> 4, (it & 15) * 8, 32768)) = o;
+    }
   }
-  cp_async_commit();
   const long long myrw = srow[j];
   tc_fence_after();
   const uint32_t tmem = *slot;
@@ -383,19 +409,18 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 f = unpack_bf16x2(xw[e]);
-        pf[e] = pack_bf16x2(f.x * wf, f.y * wf);
-        pb[e] = pack_bf16x2(f.x * wb, f.y * wb);
+        pf[e] = pack_f16x2_sat(f.x * wf, f.y * wf);
+        pb[e] = pack_f16x2_sat(f.x * wb, f.y * wb);
       }
       const uint32_t off = sw128_mnmajor_offset(r, ch * 8, 32768);
       *reinterpret_cast<uint4*>(sXf + off) = of;
       *reinterpret_cast<uint4*>(sXb + off) = ob;
     }
-    if (hh == 0) cp_async_wait<0>();
     fence_proxy_async();
     __syncthreads();
     if (threadIdx.x == 0) {
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
+      const uint32_t idesc = idesc_f16_f32(128, 64, 1, 1);
       const uint32_t ab = smem_u32(sB), xf = smem_u32(sXf), xb = smem_u32(sXb);
 #pragma unroll 4
       for (int k = 0; k < 16; ++k) {
@@ -410,37 +435,36 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
       dl_next = myrw >= 0 ? cb.d[myrw * cb.ldd + h + 1] : 0.f;
       dlb_next = per_dir ? (myrw >= 0 ? cb.d[myrw * cb.ldd + p.s.db_off + h + 1] : 0.f) : dl_next;
     }
-    mbar_wait(bar, phase);
+    const bool ok = mbar_wait(bar, phase);
     phase ^= 1;
+    // a wait that ran out (flagged in the status word) ends the walk for the whole CTA: no read-out, no
+    // further heads; the CTA still frees its TMEM
+    if (__syncthreads_or(!ok)) break;
     tc_fence_after();
     const int dir = warp >> 2, quad = warp & 3;
     const int nidx = quad * 32 + lane;
     if (dir == 0 || video || per_dir) {
-      __nv_bfloat16* dst = dir == 0
+      float* dst = dir == 0
           ? p.Sf + ((static_cast<long long>(b) * nC + c) * p.nh + h) * (kSsdP * kSsdN)
           : (video ? p.Sb + ((static_cast<long long>(b) * p.nVc + (c - p.nRc)) * p.nh + h) * (kSsdP * kSsdN)
                    : p.Srb + ((static_cast<long long>(b) * p.nRc + c) * p.nh + h) * (kSsdP * kSsdN));
-      // lane = state row n: its 64 p values are one contiguous 128-byte row of the [N][P] state
+      // lane = state row n: its 64 p values are one contiguous 256-byte row of the [N][P] fp32 state
       for (int pc = 0; pc < 2; ++pc) {
         uint32_t r[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + dir * 64 + pc * 32, r);
         tmem_wait_ld();
-        uint4* d4 = reinterpret_cast<uint4*>(dst + nidx * kSsdP + pc * 32);
+        float4* d4 = reinterpret_cast<float4*>(dst + nidx * kSsdP + pc * 32);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 pk;
-          pk.x = pack_bf16x2(__uint_as_float(r[q * 8 + 0]), __uint_as_float(r[q * 8 + 1]));
-          pk.y = pack_bf16x2(__uint_as_float(r[q * 8 + 2]), __uint_as_float(r[q * 8 + 3]));
-          pk.z = pack_bf16x2(__uint_as_float(r[q * 8 + 4]), __uint_as_float(r[q * 8 + 5]));
-          pk.w = pack_bf16x2(__uint_as_float(r[q * 8 + 6]), __uint_as_float(r[q * 8 + 7]));
-          d4[q] = pk;
-        }
+        for (int q = 0; q < 8; ++q)
+          d4[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                              __uint_as_float(r[4 * q + 3]));
       }
     }
     if (threadIdx.x == 0) p.gl[(static_cast<long long>(b) * nC + c) * p.nh + h] = s_last;
     tc_fence_before();
     __syncthreads();
   }
+  __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 128);
@@ -450,7 +474,8 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
 // ---------------------------------------------------------------------------------------------------
 // Sequential carry across chunks.  grid (P*N/8/128, nh, 2*B), 128 threads; thread = 8 state elements.
 // Review chunks are visited first (same order in both directions); then the video chunks ascending
-// (forward) or descending (backward).  Writes the state entering each video chunk.
+// (forward) or descending (backward).  Reads the fp32 chunk states and writes the state entering each
+// video chunk as the bf16 pair hi | lo (hi = bf16(H), lo = bf16(H - hi)).
 // ---------------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
   const int e8 = blockIdx.x * blockDim.x + threadIdx.x;  // vector of 8 elements
@@ -462,34 +487,40 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
   float H[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) H[e] = 0.f;
-  auto step = [&](float glv, uint4 sv) {
+  auto step = [&](float glv, float4 s0, float4 s1) {
     const float g = __expf(glv);
-    const uint32_t* u = reinterpret_cast<const uint32_t*>(&sv);
+    H[0] = fmaf(g, H[0], s0.x); H[1] = fmaf(g, H[1], s0.y); H[2] = fmaf(g, H[2], s0.z); H[3] = fmaf(g, H[3], s0.w);
+    H[4] = fmaf(g, H[4], s1.x); H[5] = fmaf(g, H[5], s1.y); H[6] = fmaf(g, H[6], s1.z); H[7] = fmaf(g, H[7], s1.w);
+  };
+  auto store = [&](__nv_bfloat16* base) {   // base: the [2][N][P] hi | lo pair of one (chunk, head)
+    uint4 hi, lo;
+    uint32_t* uh = reinterpret_cast<uint32_t*>(&hi);
+    uint32_t* ul = reinterpret_cast<uint32_t*>(&lo);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 f = unpack_bf16x2(u[e]);
-      H[2 * e] = fmaf(g, H[2 * e], f.x);
-      H[2 * e + 1] = fmaf(g, H[2 * e + 1], f.y);
+      uh[e] = pack_bf16x2(H[2 * e], H[2 * e + 1]);
+      const float2 r = unpack_bf16x2(uh[e]);
+      ul[e] = pack_bf16x2(H[2 * e] - r.x, H[2 * e + 1] - r.y);
     }
+    *reinterpret_cast<uint4*>(base + e8 * 8) = hi;
+    *reinterpret_cast<uint4*>(base + PN + e8 * 8) = lo;
   };
-  auto store = [&](__nv_bfloat16* base) {
-    uint4 o;
-    uint32_t* u = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(H[2 * e], H[2 * e + 1]);
-    *reinterpret_cast<uint4*>(base + e8 * 8) = o;
+  auto load = [&](const float* S, float4& s0, float4& s1) {
+    s0 = __ldg(reinterpret_cast<const float4*>(S) + 2 * e8);
+    s1 = __ldg(reinterpret_cast<const float4*>(S) + 2 * e8 + 1);
   };
   const bool bwd_own = dir == 1 && p.A_log_b != nullptr;   // backward scan with its own parameters
   const float* gld = bwd_own ? p.glb : p.gl;
   for (int c = 0; c < p.nRc; ++c) {
     const long long ci = (static_cast<long long>(b) * nC + c) * p.nh + h;
-    const __nv_bfloat16* S = bwd_own ? p.Srb + ((static_cast<long long>(b) * p.nRc + c) * p.nh + h) * PN
-                                     : p.Sf + ci * PN;
-    step(gld[ci], __ldg(reinterpret_cast<const uint4*>(S) + e8));
+    const float* S = bwd_own ? p.Srb + ((static_cast<long long>(b) * p.nRc + c) * p.nh + h) * PN : p.Sf + ci * PN;
+    float4 s0, s1;
+    load(S, s0, s1);
+    step(gld[ci], s0, s1);
   }
-  constexpr int U = 16;   // chunks in flight per thread (4: 0.30 ms, 8: 0.27 ms, 16: 0.22 ms at 1024 chunks)
+  constexpr int U = 8;   // chunks in flight per thread (256 bytes of fp32 state)
   for (int k0 = 0; k0 < p.nVc; k0 += U) {
-    uint4 sv[U];
+    float4 sv[U][2];
     float gv[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -499,7 +530,7 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
         const long long ci = (static_cast<long long>(b) * nC + p.nRc + v) * p.nh + h;
         const long long vi = (static_cast<long long>(b) * p.nVc + v) * p.nh + h;
         gv[u] = gld[ci];
-        sv[u] = __ldg(reinterpret_cast<const uint4*>((dir == 0 ? p.Sf + ci * PN : p.Sb + vi * PN)) + e8);
+        load(dir == 0 ? p.Sf + ci * PN : p.Sb + vi * PN, sv[u][0], sv[u][1]);
       }
     }
 #pragma unroll
@@ -508,8 +539,8 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
       if (k < p.nVc) {
         const int v = dir == 0 ? k : p.nVc - 1 - k;
         const long long vi = (static_cast<long long>(b) * p.nVc + v) * p.nh + h;
-        store((dir == 0 ? p.Hf : p.Hb) + vi * PN);
-        step(gv[u], sv[u]);
+        store((dir == 0 ? p.Hf : p.Hb) + vi * 2 * PN);
+        step(gv[u], sv[u][0], sv[u][1]);
       }
     }
   }
@@ -522,15 +553,16 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 // they are loaded once per group and stay in shared memory.
 //
 //   warp 0       per item: the head's decay tables (one bulk copy) and x rows (all 256 of the chunk,
-//                MN-major, TMA four-row gathers) into one of two x buffers; the head's incoming states
-//                [Hf | Hb] (MN-major, 2D TMA) into the H buffer once the previous item's C H^T product
-//                is done.
-//   warp 1       per group: the tile's C rows (K-major, four-row gathers).
+//                MN-major, TMA four-row gathers) into one of two x buffers.
+//   warp 1       per group: the tile's C rows (K-major, four-row gathers); per item: the head's incoming
+//                states [Hf | Hb] (MN-major, 2D TMA), first their hi parts, then, once the hi product is
+//                done, their lo parts into the same buffer.
 //   warp 2       per group: the tile's rows of G (2D TMA) into four 64-column slots, each refilled once
 //                the last head of the previous group has read it.
 //   warp 3       MMA issue (lane 0 only; an issuing thread stalls while the tensor pipe is busy, so it has
-//                no other work): Yd = M x per K half of M (A from TMEM) and, after the first half,
-//                [Yf | Yb] = C [Hf | Hb]^T as one N = 128 product, into one of two TMEM accumulator sets.
+//                no other work): Yd = M x per K half of M (A from TMEM) and, after each half,
+//                [Yf | Yb] (+)= C [Hf | Hb]^T as one N = 128 product (hi parts, then lo parts), into one of
+//                two TMEM accumulator sets.
 //   warps 4..11  transform (two warps per TMEM lane quadrant, alternating 8-column chunks): form
 //                M_ij = G_ij delta_j dec(i, j) (diagonal excluded) from the G slots and store M straight
 //                into TMEM as the A operand of the MMA (two bf16 per 32-bit column), in two K halves.
@@ -556,7 +588,7 @@ constexpr uint32_t kOutTblBytes = kOutTbl * 4;         // 8704
 constexpr uint32_t kOutXBuf = 41984;                    // x tile (32 KB) + the head's tables, two of them
 constexpr uint32_t kOutOffTbl = 32768;
 constexpr uint32_t kOutOffC = 2 * kOutXBuf;             // C rows of the tile: 2 K blocks of 16 KB
-constexpr uint32_t kOutOffH = kOutOffC + 32768;         // [Hf | Hb]: 2 MN blocks of [N = 128][P = 64]
+constexpr uint32_t kOutOffH = kOutOffC + 32768;         // [Hf | Hb] hi or lo: 2 MN blocks of [N = 128][P = 64]
 constexpr uint32_t kOutOffG = kOutOffH + 32768;         // 4 slots of [128 rows][64 cols] K-major
 constexpr uint32_t kOutOffBar = kOutOffG + 4 * 16384;
 constexpr uint32_t kOutSmem = kOutOffBar + 256;
@@ -564,8 +596,8 @@ static_assert(kOutOffTbl + kOutTblBytes <= kOutXBuf, "tables overflow the x buff
 static_assert(kOutXBuf % 1024 == 0 && kOutOffC % 1024 == 0 && kOutOffG % 1024 == 0, "1024-byte operand tiles");
 
 // Tensor maps of the output kernel: x and C rows of the video arrays (one-row boxes of 64 columns, for
-// four-row gathers), the carried states ([N rows][P] per chunk and head, 64 x 128 boxes) and G
-// ([chunk rows][Q] bf16, 64 x 128 boxes).
+// four-row gathers), the carried states ([2][N rows][P] hi | lo per chunk and head, 64 x 128 boxes) and G
+// ([chunk rows][Q] fp16, 64 x 128 boxes).
 struct SsdOutMaps {
   CUtensorMap x, c, hf, hb, g;
   int rows;   // row extent of the x / C maps; gathers of invalid rows use this (out of range -> zeros)
@@ -578,8 +610,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOutOffBar);
   uint64_t* x_full = bars;         // [2] x + table bytes
   uint64_t* x_empty = bars + 2;    // [2] last Yd MMA commit + 4 epilogue warps
-  uint64_t* h_full = bars + 4;     // Hf + Hb bytes
-  uint64_t* h_empty = bars + 5;    // Yf / Yb MMA commit
+  uint64_t* h_full = bars + 4;     // Hf + Hb bytes (hi parts, then lo parts: two phases per item)
+  uint64_t* h_empty = bars + 5;    // Yf / Yb MMA commit (one per part)
   uint64_t* c_full = bars + 6;     // C bytes (per group)
   uint64_t* c_empty = bars + 7;    // last head's Yf / Yb MMA commit
   uint64_t* g_full = bars + 8;     // [4] one G slot's bytes (per group)
@@ -666,26 +698,19 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           for (int e = 0; e < 4; ++e) id[e] = rows[4 * u + e] < 0 ? mp.rows : rows[4 * u + e];
           tma_gather4(&mp.x, &x_full[buf], XB + (2 * lane + u) * 512, h * kSsdP, id[0], id[1], id[2], id[3]);
         }
-        if (!wait_all(h_empty, (k & 1) ^ 1)) { ok = false; break; }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(h_full, 32768);
-          const int hrow = static_cast<int>((cidx * nh + h) * kSsdN);
-          tma_load_2d(&mp.hf, h_full, smem + kOutOffH, 0, hrow);
-          tma_load_2d(&mp.hb, h_full, smem + kOutOffH + 16384, 0, hrow);
-        }
-        __syncwarp();
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) rows[e] = rows_next[e];
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------------------ C rows, per group
-    int kg = 0;
-    for (int g = blockIdx.x; g < ngroups; g += gridDim.x, ++kg) {
+    // ------------------------------------------------------------------------------ C rows per group, H per item
+    int kg = 0, k = 0;
+    bool ok = true;
+    for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x, ++kg) {
       int b, v, t;
       decode(g, b, v, t);
-      const int4 r4 = reinterpret_cast<const int4*>(p.crow + (static_cast<long long>(b) * p.nVc + v) * kSsdQ +
-                                                    t * 128)[lane];
+      const long long cidx = static_cast<long long>(b) * p.nVc + v;
+      const int4 r4 = reinterpret_cast<const int4*>(p.crow + cidx * kSsdQ + t * 128)[lane];
       const int id[4] = {r4.x < 0 ? mp.rows : r4.x, r4.y < 0 ? mp.rows : r4.y, r4.z < 0 ? mp.rows : r4.z,
                          r4.w < 0 ? mp.rows : r4.w};
       if (!wait_all(c_empty, (kg & 1) ^ 1)) break;
@@ -694,6 +719,18 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb)
         tma_gather4(&mp.c, c_full, smem + kOutOffC + kb * 16384 + lane * 512, kb * 64, id[0], id[1], id[2], id[3]);
+      for (int h = 0; h < nh && ok; ++h, ++k) {
+        for (int part = 0; part < 2; ++part) {   // hi parts, then lo parts, through the one H buffer
+          if (!wait_all(h_empty, part ^ 1)) { ok = false; break; }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(h_full, 32768);
+            const int hrow = static_cast<int>(((cidx * nh + h) * 2 + part) * kSsdN);
+            tma_load_2d(&mp.hf, h_full, smem + kOutOffH, 0, hrow);
+            tma_load_2d(&mp.hb, h_full, smem + kOutOffH + 16384, 0, hrow);
+          }
+          __syncwarp();
+        }
+      }
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------------------------ G rows, per group
@@ -734,15 +771,14 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           for (int q = 0; q < 8; ++q)   // Yd = M x, first K half (M in TMEM, 8 columns per 16 elements)
             mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, q > 0);
           mma_commit(&m_empty[0]);
-          ok = mbar_wait(h_full, k & 1) && (h > 0 || mbar_wait(c_full, kg & 1));
+          ok = mbar_wait(h_full, 0) && (h > 0 || mbar_wait(c_full, kg & 1));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int q = 0; q < 8; ++q)   // [Yf | Yb] = C [Hf | Hb]^T, K = N_state = 128
+          for (int q = 0; q < 8; ++q)   // [Yf | Yb] = C [Hf | Hb]_hi^T, K = N_state = 128
             mma_bf16_ss(ybase + 64, desc_sw128(cbase + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
                         desc_sw128(hbase + q * 2048, 16384, 1024), idesc_h, q > 0);
           mma_commit(h_empty);
-          if (h == nh - 1) mma_commit(c_empty);
           ok = mbar_wait(&m_full[1], k & 1);
           if (!ok) break;
           tc_fence_after();
@@ -750,8 +786,17 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           for (int q = 8; q < 16; ++q)   // Yd, second K half
             mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, true);
           mma_commit(&m_empty[1]);
-          mma_commit(&y_full[acc]);
           mma_commit(&x_empty[buf]);
+          ok = mbar_wait(h_full, 1);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int q = 0; q < 8; ++q)   // [Yf | Yb] += C [Hf | Hb]_lo^T
+            mma_bf16_ss(ybase + 64, desc_sw128(cbase + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
+                        desc_sw128(hbase + q * 2048, 16384, 1024), idesc_h, true);
+          mma_commit(h_empty);
+          if (h == nh - 1) mma_commit(c_empty);
+          mma_commit(&y_full[acc]);
         }
       }
     }
@@ -796,10 +841,10 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
               const float4 wa = *reinterpret_cast<const float4*>(w + qq * 16);
               const float4 wc = *reinterpret_cast<const float4*>(w + qq * 16 + 4);
               // the same products as g * (u * w) elementwise, two per instruction
-              const float2 m0 = mul_f32x2(unpack_bf16x2(gc.x), mul_f32x2(uu, make_float2(wa.x, wa.y)));
-              const float2 m1 = mul_f32x2(unpack_bf16x2(gc.y), mul_f32x2(uu, make_float2(wa.z, wa.w)));
-              const float2 m2 = mul_f32x2(unpack_bf16x2(gc.z), mul_f32x2(uu, make_float2(wc.x, wc.y)));
-              const float2 m3 = mul_f32x2(unpack_bf16x2(gc.w), mul_f32x2(uu, make_float2(wc.z, wc.w)));
+              const float2 m0 = mul_f32x2(unpack_f16x2(gc.x), mul_f32x2(uu, make_float2(wa.x, wa.y)));
+              const float2 m1 = mul_f32x2(unpack_f16x2(gc.y), mul_f32x2(uu, make_float2(wa.z, wa.w)));
+              const float2 m2 = mul_f32x2(unpack_f16x2(gc.z), mul_f32x2(uu, make_float2(wc.x, wc.y)));
+              const float2 m3 = mul_f32x2(unpack_f16x2(gc.w), mul_f32x2(uu, make_float2(wc.z, wc.w)));
               tmem_st4(tcol + qq * 8, pack_bf16x2(m0.x, m0.y), pack_bf16x2(m1.x, m1.y), pack_bf16x2(m2.x, m2.y),
                        pack_bf16x2(m3.x, m3.y));
             }
@@ -830,7 +875,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
               uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const float2 gm = mul_f32x2(unpack_bf16x2(gu[e]), make_float2(m[2 * e], m[2 * e + 1]));
+                const float2 gm = mul_f32x2(unpack_f16x2(gu[e]), make_float2(m[2 * e], m[2 * e + 1]));
                 pk[e] = pack_bf16x2(gm.x, gm.y);
               }
               tmem_st4(tcol + qq * 8, pk[0], pk[1], pk[2], pk[3]);

@@ -13,7 +13,7 @@ import torch
 
 from . import _lib
 
-__all__ = ["MateBlock", "rms_permute", "rms_unpermute", "review_pool", "ssd_scan_bidir", "ssd_scan_bidir_pd",
+__all__ = ["MateBlock", "DitBlock", "dit_weights_to_device", "rms_permute", "rms_unpermute", "review_pool", "ssd_scan_bidir", "ssd_scan_bidir_pd",
            "ssd_scan_bidir_noalloc", "ssd_scan_bidir_backward", "tesa_forward", "project_bf16", "device_status",
            "torch_dtype", "weights_to_device", "scan_locality", "KernelTrace"]
 
@@ -53,9 +53,11 @@ def weights_to_device(w: Dict, cfg, device="cuda") -> Dict[str, torch.Tensor]:
 class MateBlock:
     """One MATE block (MA + TE branches) with its weights resident on the GPU and a reusable workspace.
     Weights W_z, conv_w, conv_b and norm_w, given together, make the MA branch's core a full Mamba2 block
-    (causal convolution + SiLU on x | B | C, SiLU(z) gate, gated RMSNorm)."""
+    (causal convolution + SiLU on x | B | C, SiLU(z) gate, gated RMSNorm).  The projection matrices are
+    packed once here (mate_pack_weights); pack=False makes every forward pack them again instead."""
 
-    def __init__(self, cfg, weights: Dict[str, torch.Tensor], device="cuda"):
+    def __init__(self, cfg, weights: Dict[str, torch.Tensor], device="cuda", pack: bool = True,
+                 workspace: bool = True):
         lib = _lib.load()
         self.cfg = cfg
         ext = [k for k in ("W_z", "conv_w", "conv_b", "norm_w") if k in weights]
@@ -88,8 +90,15 @@ class MateBlock:
         self.cw = _lib.CWeights(*(weights[k].data_ptr() if k in weights else None for k in
                                   ("W_in", "dt_bias", "A_log", "D", "W_out", "W_qkv", "W_o", "dt_bias_b", "A_log_b",
                                    "D_b", "W_z", "conv_w", "conv_b", "norm_w")))
+        self.packed = None
+        if pack:
+            nb = lib.mate_packed_weights_bytes(ctypes.byref(self.ccfg))
+            self.packed = torch.empty(nb, dtype=torch.uint8, device=self.device)
+            _lib.check(lib.mate_pack_weights(ctypes.byref(self.cw), ctypes.byref(self.ccfg), _p(self.packed), nb,
+                                             _s(None)), "mate_pack_weights")
+            self.cw.packed = self.packed.data_ptr()
         self.ws_bytes = lib.mate_workspace_bytes(ctypes.byref(self.ccfg))
-        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        self.ws = torch.empty(self.ws_bytes if workspace else 0, dtype=torch.uint8, device=self.device)
         self.ws_host = None
         self.numel = cfg.B * cfg.T * cfg.H * cfg.W * cfg.d
 
@@ -106,8 +115,10 @@ class MateBlock:
         return out
 
     def forward_host(self, X_host: torch.Tensor, layer_idx: int, out_host: torch.Tensor,
-                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-        """mate_forward_host: host (page-locked) input and output, copies inside the call."""
+                     stream: Optional[torch.cuda.Stream] = None, pipelined: bool = False) -> torch.Tensor:
+        """mate_forward_host: host (page-locked) input and output, copies inside the call.  pipelined: the copies
+        overlap the neighbouring calls' work (mate_forward_host_pipelined); out_host is then complete once the
+        stream reaches the end of the next pipelined call or of flush_host()."""
         lib = _lib.load()
         if self.ws_host is None:
             nb = lib.mate_forward_host_workspace_bytes(ctypes.byref(self.ccfg))
@@ -115,14 +126,69 @@ class MateBlock:
         for t, nm in ((X_host, "X_host"), (out_host, "out_host")):
             if t.is_cuda or t.dtype != self.dtype or t.numel() != self.numel or not t.is_contiguous():
                 raise ValueError(f"{nm}: expected a contiguous host {self.dtype} tensor with {self.numel} elements")
-        st = lib.mate_forward_host(_p(X_host), ctypes.byref(self.cw), int(layer_idx), _p(out_host),
-                                   ctypes.byref(self.ccfg), _p(self.ws_host), self.ws_host.numel(), _s(stream))
-        _lib.check(st, "mate_forward_host")
+        fn = lib.mate_forward_host_pipelined if pipelined else lib.mate_forward_host
+        st = fn(_p(X_host), ctypes.byref(self.cw), int(layer_idx), _p(out_host), ctypes.byref(self.ccfg),
+                _p(self.ws_host), self.ws_host.numel(), _s(stream))
+        _lib.check(st, "mate_forward_host_pipelined" if pipelined else "mate_forward_host")
         return out_host
+
+    @staticmethod
+    def flush_host(stream: Optional[torch.cuda.Stream] = None):
+        """mate_forward_host_flush: the stream waits for every pipelined call's output copy."""
+        _lib.check(_lib.load().mate_forward_host_flush(_s(stream)), "mate_forward_host_flush")
 
     @staticmethod
     def last_launch_count() -> int:
         return _lib.load().mate_last_launch_count()
+
+
+def dit_weights_to_device(w: Dict, cfg, device="cuda") -> Dict[str, torch.Tensor]:
+    """Host DiT-block weights (W_ada [6d, dc], W1 [4d, d], W2 [d, 4d], b_ada, b1, b2) -> device tensors in the
+    library's dtypes (matrices in the block's dtype, biases fp32)."""
+    dt = torch_dtype(cfg)
+    out = {k: torch.as_tensor(w[k]).to(device=device, dtype=dt).contiguous() for k in ("W_ada", "W1", "W2")}
+    out.update({k: torch.as_tensor(w[k]).to(device=device, dtype=torch.float32).contiguous()
+                for k in ("b_ada", "b1", "b2")})
+    return out
+
+
+class DitBlock:
+    """A DiT block with the MATE block as its token mixer (mate_dit_block_forward): adaLN-Zero modulation
+    from a per-sample conditioning vector c [B, dc], the mixer behind a gated residual, and a gated GELU MLP
+    of width 4 d."""
+
+    def __init__(self, cfg, mate_weights: Dict[str, torch.Tensor], dit_weights: Dict[str, torch.Tensor], dc: int,
+                 device="cuda"):
+        lib = _lib.load()
+        self.cfg, self.dc = cfg, int(dc)
+        self.mix = MateBlock(cfg, mate_weights, device, workspace=False)
+        d = cfg.d
+        dt = torch_dtype(cfg)
+        _need(dit_weights["W_ada"], dt, 6 * d * self.dc, "W_ada")
+        _need(dit_weights["W1"], dt, 4 * d * d, "W1")
+        _need(dit_weights["W2"], dt, 4 * d * d, "W2")
+        _need(dit_weights["b_ada"], torch.float32, 6 * d, "b_ada")
+        _need(dit_weights["b1"], torch.float32, 4 * d, "b1")
+        _need(dit_weights["b2"], torch.float32, d, "b2")
+        self.w = dit_weights
+        self.cw = _lib.CDitWeights(*(dit_weights[k].data_ptr() for k in ("W_ada", "b_ada", "W1", "b1", "W2", "b2")))
+        self.ws_bytes = lib.mate_dit_workspace_bytes(ctypes.byref(self.mix.ccfg))
+        if self.ws_bytes == 0:
+            raise ValueError("mate_dit_workspace_bytes: configuration not supported by the DiT block")
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+
+    def forward(self, X: torch.Tensor, c: torch.Tensor, layer_idx: int, out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        _need(X, self.mix.dtype, self.mix.numel, "X")
+        _need(c, torch.float32, self.cfg.B * self.dc, "c")
+        if out is None:
+            out = torch.empty_like(X)
+        _need(out, self.mix.dtype, self.mix.numel, "out")
+        st = _lib.load().mate_dit_block_forward(_p(X), _p(c), self.dc, ctypes.byref(self.cw),
+                                                ctypes.byref(self.mix.cw), int(layer_idx), _p(out),
+                                                ctypes.byref(self.mix.ccfg), _p(self.ws), self.ws_bytes, _s(stream))
+        _lib.check(st, "mate_dit_block_forward")
+        return out
 
 
 def _cfg(cfg):

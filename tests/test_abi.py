@@ -1,6 +1,7 @@
 """The C ABI library: it builds, loads without a GPU, exports every symbol include/mate.h declares, and
 validates arguments on the host before touching the device."""
 import ctypes
+import dataclasses
 import os
 import re
 
@@ -147,6 +148,22 @@ def test_noalloc_scan_rejects_problems_beyond_its_scratch(lib):
     assert lib.mate_ssd_workspace_bytes(ctypes.byref(c), cfg.R) > _lib.MATE_SSD_NOALLOC_SCRATCH_BYTES
     st = lib.ssd_scan_bidir_noalloc(16, 16, 16, 16, 16, 16, 16, cfg.R, 16, ctypes.byref(c), None)
     assert st == _lib.MATE_ERR_TOO_LARGE, _lib.status_str(st)
+
+
+def test_noalloc_scan_limit_follows_the_workspace_size(lib):
+    """Shapes on either side of the scratch size: those whose workspace fits are accepted up to the pointer
+    check (a null x gives MATE_ERR_ARG, before any device work), the others get MATE_ERR_TOO_LARGE."""
+    base = mi.TEST_CONFIGS["bf16_small_8x16x16"]
+    seen = set()
+    for T in (44, 48, 52, 56, 60):
+        cfg = dataclasses.replace(base, T=T, H=8, W=16, R=64)
+        c = _lib.make_config(cfg)
+        assert lib.mate_check_config(ctypes.byref(c)) == _lib.MATE_OK
+        fits = lib.mate_ssd_workspace_bytes(ctypes.byref(c), cfg.R) <= _lib.MATE_SSD_NOALLOC_SCRATCH_BYTES
+        seen.add(fits)
+        st = lib.ssd_scan_bidir_noalloc(None, 16, 16, 16, 16, 16, 16, cfg.R, 16, ctypes.byref(c), None)
+        assert st == (_lib.MATE_ERR_ARG if fits else _lib.MATE_ERR_TOO_LARGE), (T, _lib.status_str(st))
+    assert seen == {True, False}
 
 
 def test_kernel_names_are_distinct(lib):

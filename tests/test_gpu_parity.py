@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 from helpers import assert_close, assert_close_elementwise, oracle_cached, requires_gpu
-from bf16_floor import bf16_storage_forward, elementwise_err, rms_normalised_max_err, ssd_bf16_storage_emulation
+from bf16_floor import bf16_storage_forward, elementwise_err, rms_normalised_max_err, round_bf16
 import mate_inputs as mi
 from edge_configs import all_test_configs
 from oracle import mate_oracle as O
@@ -122,8 +122,7 @@ def test_ssd_scan_bidir(name, long_memory):
                          dev(A_log, torch.float32), dev(D, torch.float32), cfg.R, cfg)
     got = host(y).reshape(cfg.B, cfg.n, cfg.nh, cfg.P)
     ref = oracle_cached(f"ssd-{name}-{long_memory}", lambda: _ssd_oracle(cfg, *args))
-    assert_close_elementwise(got, ref, cfg.dtype, f"ssd {name} long={long_memory}",
-                             _ssd_floor(cfg, args, ref, f"ssd-{name}-{long_memory}"))
+    assert_close_elementwise(got, ref, cfg.dtype, f"ssd {name} long={long_memory}", _ssd_floor(cfg, ref))
 
 
 @pytest.mark.parametrize("regime", ["fast_decay", "no_decay"])
@@ -154,28 +153,15 @@ def test_ssd_scan_extreme_decays(name, regime):
         want = diag[..., None] * x.astype(np.float64)[:, cfg.R:].reshape(cfg.B, cfg.n, cfg.nh, cfg.P)
         # (the cached oracle result is stored in float32: relative 1e-6 is far below any dropped term)
         assert np.abs(ref - want).max() <= 1e-6 * max(1.0, np.abs(want).max())
-    assert_close_elementwise(got, ref, cfg.dtype, f"ssd {name} {regime}", _ssd_floor(cfg, args, ref, key))
+    assert_close_elementwise(got, ref, cfg.dtype, f"ssd {name} {regime}", _ssd_floor(cfg, ref))
 
 
-def _ssd_floor(cfg, args, ref, key, heads=None, rows=None):
-    """Element-wise error of the bf16-storage emulation of the chunked scan (0 for fp32 blocks), on the
-    video rows `rows` (all rows when None) that ref holds."""
+def _ssd_floor(cfg, ref):
+    """Storage floor of the scan entry point (0 for fp32 blocks): its inputs are bf16 already, so its only
+    stored bf16 tensor is the output y; the element-wise error of bf16(ref) against ref."""
     if cfg.dtype != "bf16":
         return 0.0
-    x, Bm, Cm, dt, dt_bias, A_log, D = args
-    heads = list(range(cfg.nh)) if heads is None else heads
-
-    def emu():
-        outs = []
-        for b in range(cfg.B):
-            delta = O.softplus(dt[b].astype(np.float64) + dt_bias.astype(np.float64))[:, heads]
-            A = -np.exp(A_log.astype(np.float64))[heads]
-            xs = x[b].reshape(-1, cfg.nh, cfg.P)[:, heads]
-            outs.append(ssd_bf16_storage_emulation(xs, Bm[b], Cm[b], delta, A, D.astype(np.float64)[heads], cfg.R,
-                                                   cfg.Q))
-        emu_out = np.stack(outs)
-        return np.array([elementwise_err(emu_out if rows is None else emu_out[:, rows], ref)])
-    return float(oracle_cached(f"floor-{key}", emu)[0])
+    return elementwise_err(round_bf16(ref), ref)
 
 
 # ------------------------------------------------------------------ TESA
@@ -213,9 +199,10 @@ def _block(cfg, variant):
     return mi.make_inputs(cfg, **kw)
 
 
-def _check_block(cfg, w, layer, variant, out):
-    """Compare the GPU block output with the oracle on all rows (small blocks) or on a fixed sample of
-    1024 rows (large blocks, whose oracle output is cached only on those rows)."""
+def block_reference(cfg, w, layer, variant):
+    """(rows, oracle output on those rows, bf16 storage floor on them) of a block case: all rows of a small
+    block, or a fixed sample of 1024 rows of a large one (whose oracle output is cached only on those
+    rows)."""
     rows = _sample_rows(cfg)
     key = f"{cfg.name}-{layer}-{variant}" + ("" if len(rows) == cfg.B * cfg.n else f"-rows{len(rows)}")
     holder = {}
@@ -230,6 +217,12 @@ def _check_block(cfg, w, layer, variant, out):
     if cfg.dtype == "bf16":
         floor = float(oracle_cached(f"floor-{key}", lambda: np.array([rms_normalised_max_err(
             bf16_storage_forward(w["X"], w, cfg, layer).reshape(cfg.B * cfg.n, cfg.d)[rows], ref)]))[0])
+    return rows, ref, floor
+
+
+def _check_block(cfg, w, layer, variant, out):
+    """Compare the GPU block output with the oracle (see block_reference)."""
+    rows, ref, floor = block_reference(cfg, w, layer, variant)
     got = np.asarray(out).reshape(cfg.B * cfg.n, cfg.d)[rows]
     assert_close(got, ref, cfg.dtype, f"mate {cfg.name} layer {layer} {variant}", floor)
 
@@ -277,6 +270,51 @@ def test_mate_forward_host_matches_device_path(name, layer):
     assert torch.equal(oh, ref.cpu())
 
 
+def test_packed_weights_match_per_call_packing():
+    """Weights packed once (mate_pack_weights, the default of MateBlock) and packed again inside every call
+    give the same bits."""
+    cfg = all_test_configs()["bf16_b2_20x16x16_d512"]
+    w = _block(cfg, "default")
+    wd = M.weights_to_device(w, cfg)
+    Xd = dev(w["X"], torch.bfloat16)
+    for layer in (1, 2):
+        a = M.MateBlock(cfg, wd).forward(Xd, layer)
+        b = M.MateBlock(cfg, wd, pack=False).forward(Xd, layer)
+        assert torch.equal(a, b), layer
+
+
+def test_pipelined_host_calls_match_device_path():
+    """Pipelined host calls (each input copy overlapping the previous call's output copy, inputs in
+    alternating device slots): a chain whose every output is the next call's input (the output copy must
+    land before the next input copy reads it), then calls that reuse one input buffer; all bit-equal to
+    the device-buffer path."""
+    cfg = all_test_configs()["bf16_small_8x16x16"]
+    w = dict(_block(cfg, "default"))
+    # the MA branch's output grows with the cube of its input, so a chain through it overflows in a few
+    # steps; the chain runs the attention branch alone, which is linear in its input
+    w["W_out"] = np.zeros_like(w["W_out"])
+    blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
+    X0 = dev(w["X"], torch.bfloat16)
+    dchain = [X0]
+    for layer in range(3):
+        dchain.append(blk.forward(dchain[-1], layer).clone())
+    hchain = [X0.cpu().pin_memory()] + [torch.empty_like(X0, device="cpu").pin_memory() for _ in range(3)]
+    for layer in range(3):
+        blk.forward_host(hchain[layer], layer, hchain[layer + 1], pipelined=True)
+    M.MateBlock.flush_host()
+    torch.cuda.synchronize()
+    for layer in range(3):
+        assert torch.equal(hchain[layer + 1], dchain[layer + 1].cpu()), f"chain step {layer}"
+    outs = [torch.empty_like(hchain[0]).pin_memory() for _ in range(4)]
+    for layer in range(4):
+        blk.forward_host(hchain[0], layer, outs[layer], pipelined=True)
+    M.MateBlock.flush_host()
+    torch.cuda.synchronize()
+    for layer in range(4):
+        assert torch.equal(outs[layer], blk.forward(X0, layer).cpu()), f"shared input, layer {layer}"
+    assert M.device_status() == 0
+
+
 def test_repeated_calls_are_deterministic():
     cfg = mi.TEST_CONFIGS["bf16_ragged_12x16x24"]
     w = _block(cfg, "long")
@@ -290,15 +328,26 @@ def test_repeated_calls_are_deterministic():
 
 # ------------------------------------------------------------------ full-size workloads
 
-@pytest.mark.parametrize("name,layer", [("bf16_256x32x32", 1), ("bf16_64x32x32", 2), ("bf16_64x32x32", 3),
-                                        ("bf16_2x64x48x48_d2048", 1)])
-def test_mate_forward_full_size(name, layer):
+# The workloads at full size: all four layers of the 65,536-token clip (every scan order, both shift
+# phases), and at the 262,144-token and the batch-2 d = 2048 workloads a spatial-order layer and the two
+# time-fastest orders (whose scan output goes through the scan-order buffer), plus the long-memory block.
+FULL_SIZE_CASES = [("bf16_64x32x32", 0, "default"), ("bf16_64x32x32", 1, "default"),
+                   ("bf16_64x32x32", 2, "default"), ("bf16_64x32x32", 3, "default"),
+                   ("bf16_256x32x32", 1, "default"), ("bf16_256x32x32", 2, "default"),
+                   ("bf16_256x32x32", 3, "default"), ("bf16_256x32x32", 0, "long"),
+                   ("bf16_2x64x48x48_d2048", 1, "default"), ("bf16_2x64x48x48_d2048", 2, "default"),
+                   ("bf16_2x64x48x48_d2048", 3, "default")]
+
+
+@pytest.mark.parametrize("name,layer,variant", FULL_SIZE_CASES)
+def test_mate_forward_full_size(name, layer, variant):
     """The block at its full workload sizes, in the launch configuration the benchmark times."""
     cfg = mi.CONFIGS[name]
-    w = mi.make_inputs(cfg)
+    w = _block(cfg, variant)
     blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
     out = host(blk.forward(dev(w["X"], torch.bfloat16), layer))
-    _check_block(cfg, w, layer, "default", out)
+    del blk
+    _check_block(cfg, w, layer, variant, out)
 
 
 def test_ssd_full_size_sampled_head():
@@ -312,7 +361,7 @@ def test_ssd_full_size_sampled_head():
     got = host(y).reshape(cfg.B, cfg.n, cfg.nh, cfg.P)[:, rows][:, :, [5]]
     key = "ssd-full-bf16_256x32x32-h5-every16"
     ref = oracle_cached(key, lambda: _ssd_oracle(cfg, *args, heads=[5])[:, rows])
-    assert_close_elementwise(got, ref, "bf16", "ssd full size head 5", _ssd_floor(cfg, args, ref, key, [5], rows))
+    assert_close_elementwise(got, ref, "bf16", "ssd full size head 5", _ssd_floor(cfg, ref))
 
 
 # ------------------------------------------------------------------ scan locality

@@ -69,24 +69,13 @@ def video_rows(cfg, stride=16):
 
 def scan_reference(name, long_memory):
     """(inputs, backward parameters, sampled rows, oracle y on those rows, bf16 storage floor) of the
-    per-direction scan case.  The floor is the larger of the two shared-parameter emulations (each
-    direction's decays alone), each measured against its own shared-parameter oracle on the same rows."""
-    from test_gpu_parity import _ssd_oracle
+    per-direction scan case.  The floor is that of the stored bf16 output on the same rows."""
     cfg = all_test_configs()[name]
     args, bwd = _scan_args(cfg, long_memory)
     rows = video_rows(cfg)
     key = f"pd-ssd-{name}-{long_memory}-every16"
     ref = oracle_cached(key, lambda: _pd_oracle(cfg, *args, *bwd)[:, rows], PD_SRC)
-    floor = 0.0
-    if cfg.dtype == "bf16":
-        x, Bm, Cm, dt, dt_bias, A_log, D = args
-        for tag, params in (("f", (dt_bias, A_log, D)), ("b", bwd)):
-            a2 = (x, Bm, Cm, dt) + tuple(params)
-            k2 = f"pd-ssd-{name}-{long_memory}-every16-shared{tag}"
-            # only the scalar floor is kept on disk
-            fl = lambda a2=a2, k2=k2: np.array([_ssd_floor(cfg, a2, _ssd_oracle(cfg, *a2)[:, rows], k2, rows=rows)])
-            floor = max(floor, float(oracle_cached(f"pd-floor-{k2}", fl, PD_SRC)[0]))
-    return args, bwd, rows, ref, floor
+    return args, bwd, rows, ref, _ssd_floor(cfg, ref)
 
 
 @pytest.mark.parametrize("long_memory", [False, True])
