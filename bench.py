@@ -336,18 +336,26 @@ def measure_scaling(M, torch, stream, headline, headline_name, headline_ms, step
     return out
 
 
-def measure_dit(M, torch, cfg, w, X, stream, hbm_peak, tf_peak, steps=12, dc=256):
-    """The DiT block around the mixer (adaLN modulation, layer norms, the mixer behind a gated residual, the
-    gated GELU MLP of width 4 d) at the headline workload, timed after the headline region: ms per block,
-    algorithmic TFLOP/s and the per-kernel fractions.  Weights: W_ada N(0, 1/dc), W1 N(0, 1/d), W2
-    N(0, 1/(4 d)), biases N(0, 0.1^2), c N(0, 1), seeded."""
-    rng = np.random.default_rng(777)
+def dit_weights(cfg, dc, seed):
+    """Seeded DiT-block weights and conditioning: W_ada N(0, 1/dc), W1 N(0, 1/d), W2 N(0, 1/(4 d)) rounded to
+    bf16, biases N(0, 0.1^2), c N(0, 1)."""
+    rng = np.random.default_rng(seed)
     d = cfg.d
     bf = lambda a: mi.round_to_bf16(a.astype(np.float32))
     dw = dict(W_ada=bf(rng.standard_normal((6 * d, dc)) / np.sqrt(dc)), b_ada=(0.1 * rng.standard_normal(6 * d)),
               W1=bf(rng.standard_normal((4 * d, d)) / np.sqrt(d)), b1=0.1 * rng.standard_normal(4 * d),
               W2=bf(rng.standard_normal((d, 4 * d)) / np.sqrt(4 * d)), b2=0.1 * rng.standard_normal(d))
-    c = torch.as_tensor(rng.standard_normal((cfg.B, dc)).astype(np.float32)).cuda()
+    return dw, rng.standard_normal((cfg.B, dc)).astype(np.float32)
+
+
+def measure_dit(M, torch, cfg, w, X, stream, hbm_peak, tf_peak, steps=12, dc=256):
+    """The DiT block around the mixer (adaLN modulation, layer norms, the mixer behind a gated residual, the
+    gated GELU MLP of width 4 d) at the headline workload, timed after the headline region: ms per block,
+    algorithmic TFLOP/s and the per-kernel fractions.  Weights: W_ada N(0, 1/dc), W1 N(0, 1/d), W2
+    N(0, 1/(4 d)), biases N(0, 0.1^2), c N(0, 1), seeded."""
+    d = cfg.d
+    dw, c = dit_weights(cfg, dc, 777)
+    c = torch.as_tensor(c).cuda()
     blk = M.DitBlock(cfg, M.weights_to_device(w, cfg), M.dit_weights_to_device(dw, cfg), dc)
     out = torch.empty_like(X)
     nl = 0
@@ -377,6 +385,56 @@ def measure_dit(M, torch, cfg, w, X, stream, hbm_peak, tf_peak, steps=12, dc=256
             "steps": steps, "conditioning_width": dc,
             "kernels": {k: table[k] for k in ("mlp_up", "mlp_down", "ln_modulate", "ada_modulation", "out_projection")
                         if k in table}}
+
+
+def measure_permute(M, torch, cfg, X, stream, hbm_peak, steps=10):
+    """The standalone Rotary Major Scan permute and unpermute (rms_permute / rms_unpermute, every order),
+    timed after the headline region against the HBM roofline: each reads and writes the whole grid once."""
+    Xp = torch.empty((cfg.B, cfg.n, cfg.d), dtype=X.dtype, device=X.device)
+    Xb = torch.empty_like(X)
+    for o in range(4):
+        M.rms_permute(X, o, cfg, Xp)
+        M.rms_unpermute(Xp, o, cfg, Xb)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(steps):
+        M.rms_permute(X, s % 4, cfg, Xp)
+        M.rms_unpermute(Xp, s % 4, cfg, Xb)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (2 * steps)
+    nbytes = 2.0 * X.numel() * X.element_size()
+    ok = bool(torch.equal(Xb, X))
+    del Xp, Xb
+    return {"ms_per_call": ms, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm_peak, "round_trip_exact": ok}
+
+
+def profile_run(M, torch, cfg, w, X, out):
+    """Every kernel of the path a few times, untimed, for an ncu capture to select launches from: the
+    block over the four layers, the block with the Mamba2 extras, the DiT block, and the standalone
+    permute and unpermute."""
+    blk = M.MateBlock(cfg, M.weights_to_device(w, cfg))
+    for s in range(4):
+        blk.forward(X, s, out)
+    del blk
+    we = dict(w)
+    we.update(extras_weights(cfg, 4242))
+    blk = M.MateBlock(cfg, M.weights_to_device(we, cfg))
+    for s in range(2):
+        blk.forward(X, s, out)
+    del blk
+    dw, c = dit_weights(cfg, 256, 777)
+    blk = M.DitBlock(cfg, M.weights_to_device(w, cfg), M.dit_weights_to_device(dw, cfg), 256)
+    blk.forward(X, torch.as_tensor(c).cuda(), 1, out)
+    del blk
+    Xp = torch.empty((cfg.B, cfg.n, cfg.d), dtype=X.dtype, device=X.device)
+    for o in range(2):
+        M.rms_permute(X, o, cfg, Xp)
+        M.rms_unpermute(Xp, o, cfg, out)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_run": cfg.name, "status": M.device_status()}), flush=True)
 
 
 def oracle_sample_cfg(cfg, frames):
@@ -458,6 +516,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the full-Mamba2-block side measurement")
     ap.add_argument("--no-scaling", action="store_true", help="skip the per-workload ms/block side measurement")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="run every kernel of the path a few times without timing (for an ncu capture) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -483,6 +543,9 @@ def main():
     X = torch.as_tensor(w["X"]).to(device="cuda", dtype=torch.bfloat16)
     out = torch.empty_like(X)
     stream = torch.cuda.current_stream()
+    if args.profile_run:
+        profile_run(M, torch, cfg, w, X, out)
+        return 0
 
     def barrier():
         if world > 1:
@@ -580,7 +643,11 @@ def main():
 
     # side measurements, outside the headline region: the block with the rest of the Mamba2 block, and with
     # separate backward-scan parameters; a failure is reported in the line instead of ending the run
-    extras = per_direction = dit = None
+    extras = per_direction = dit = permute = None
+    try:
+        permute = measure_permute(M, torch, cfg, X, stream, hbm_peak)
+    except Exception as e:  # noqa: BLE001
+        permute = {"error": f"{type(e).__name__}: {e}"}
     if not args.no_extras:
         try:
             dit = measure_dit(M, torch, cfg, w, X, stream, hbm_peak, tf_peak)
@@ -639,6 +706,7 @@ def main():
         "mamba_extras": extras,
         "per_direction_scan": per_direction,
         "dit_block": dit,
+        "rms_permute": permute,
         "clocks": clocks,
         "device_status": status,
     }

@@ -275,6 +275,22 @@ MATE_API mate_status ssd_scan_bidir_noalloc(const void* x, const void* Bm, const
 MATE_API mate_status tesa_forward(const void* qkv, void* O, int shifted, const mate_config* cfg, mate_stream_t stream);
 
 /*
+ * Backward pass of tesa_forward (training; the pages give only the forward computation, and its gradient
+ * follows by the chain rule).  Given the forward's input qkv, its output O and the output gradient dO
+ * (all [B, T, H, W, .] as for tesa_forward, heads in the same column order), writes dqkv [B, T, H, W,
+ * 3*th*tp] (dq | dk | dv in the column layout of qkv).  Per window and head, with P the forward's masked
+ * softmax of q k^T / sqrt(tp):
+ *     dv = P^T dO,   dP = dO v^T,   dS = P (dP - rowsum(dO * O)),   dq = dS k / sqrt(tp),   dk = dS^T q / sqrt(tp).
+ * Every token belongs to exactly one window per layer, so each row of dqkv is written once.  bf16 blocks
+ * only (MATE_ERR_UNSUPPORTED otherwise); tensor-core products with bf16 operands (P and dS rounded to bf16)
+ * and fp32 softmax statistics.  ws: at least mate_tesa_backward_workspace_bytes(cfg) bytes (per window,
+ * head and query: the softmax normaliser and rowsum(dO * O), written by the first kernel, read by the second).
+ */
+MATE_API size_t mate_tesa_backward_workspace_bytes(const mate_config* cfg);
+MATE_API mate_status tesa_backward(const void* qkv, const void* O, const void* dO, void* dqkv, int shifted,
+                                   const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream);
+
+/*
  * Scan locality ([NEWS] method, Rotary Major Scan paragraphs; [FEAT] 功能特色 / RMS: the alternating
  * orders bring the average distance, after the scan, between originally adjacent tokens down to the level
  * of Zigzag and Hilbert scans).  Over all pairs of tokens of a T x H x W grid that differ by one step along
@@ -426,7 +442,9 @@ typedef enum {
   MATE_K_ADA_MODULATION = 21,  /* DiT block: modulation vectors silu(c) W_ada^T + b_ada */
   MATE_K_LN_MODULATE = 22,     /* DiT block: layer norm + scale and shift */
   MATE_K_MLP_UP = 23,          /* DiT block: gelu(h W1^T + b1) */
-  MATE_K_MLP_DOWN = 24         /* DiT block: X1 + gate_m (Z W2^T + b2) */
+  MATE_K_MLP_DOWN = 24,        /* DiT block: X1 + gate_m (Z W2^T + b2) */
+  MATE_K_TESA_BWD_DQ = 25,     /* tesa_backward: row statistics, delta and dQ */
+  MATE_K_TESA_BWD_DKDV = 26    /* tesa_backward: dK and dV */
 } mate_kernel;
 
 typedef struct {

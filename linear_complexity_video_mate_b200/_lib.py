@@ -19,7 +19,7 @@ EXPORTS = (
     "mate_scan_locality", "ssd_scan_bidir_pd", "mate_ssd_pd_workspace_bytes", "ssd_scan_bidir_backward",
     "mate_ssd_backward_workspace_bytes", "mate_selftest_wait_timeout", "mate_forward_host_pipelined",
     "mate_packed_weights_bytes", "mate_pack_weights", "mate_dit_workspace_bytes", "mate_dit_block_forward",
-    "mate_forward_host_flush",
+    "mate_forward_host_flush", "mate_tesa_backward_workspace_bytes", "tesa_backward",
 )
 
 _CONFIG_FIELDS = ("B", "T", "H", "W", "d", "nh", "P", "N", "Q", "R", "th", "tp", "wt", "wh", "ww", "st", "sh", "sw")
@@ -91,6 +91,8 @@ def load():
         "mate_forward_host_pipelined": (ci, [vp, wp, ci, vp, cfgp, vp, sz, vp]),
         "mate_packed_weights_bytes": (sz, [cfgp]),
         "mate_forward_host_flush": (ci, [vp]),
+        "mate_tesa_backward_workspace_bytes": (sz, [cfgp]),
+        "tesa_backward": (ci, [vp, vp, vp, vp, ci, cfgp, vp, sz, vp]),
         "mate_pack_weights": (ci, [wp, cfgp, vp, sz, vp]),
         "mate_dit_workspace_bytes": (sz, [cfgp]),
         "mate_dit_block_forward": (ci, [vp, vp, ci, ctypes.POINTER(CDitWeights), wp, ci, vp, cfgp, vp, sz, vp]),

@@ -92,10 +92,20 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const T* __restrict__ 
   for (int q = 0; q < kMaxVec; ++q) {
     const int c0 = (q * 32 + lane) * V;
     if (c0 < d) {
+      // shift and scale of these V channels: V / 4 sixteen-byte loads each (the modulation rows are
+      // 16-byte aligned: 6 d floats per sample, d a multiple of 8)
+      float scv[V], shv[V];
+#pragma unroll
+      for (int i = 0; i < V; i += 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(sc + c0 + i));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(sh + c0 + i));
+        scv[i] = a.x; scv[i + 1] = a.y; scv[i + 2] = a.z; scv[i + 3] = a.w;
+        shv[i] = b.x; shv[i + 1] = b.y; shv[i + 2] = b.z; shv[i + 3] = b.w;
+      }
       uint4 u;
       T* e = reinterpret_cast<T*>(&u);
 #pragma unroll
-      for (int i = 0; i < V; ++i) e[i] = static_cast<T>((v[q][i] - mean) * rstd * (1.f + sc[c0 + i]) + sh[c0 + i]);
+      for (int i = 0; i < V; ++i) e[i] = static_cast<T>(fmaf((v[q][i] - mean) * rstd, 1.f + scv[i], shv[i]));
       *reinterpret_cast<uint4*>(hr + c0) = u;
     }
   }

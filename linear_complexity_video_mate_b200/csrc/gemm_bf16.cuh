@@ -201,9 +201,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (has_ep) {
           const GemmEpilogue& e = p.ep;
           if (e.bias != nullptr) {
+            if (full32) {   // 32 consecutive columns: eight 16-byte loads (bias 16-byte aligned, col0 % 32 == 0)
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (full32 || col0 + j < col_end) v[j] += __ldg(e.bias + col0 + j);
+              for (int q = 0; q < 8; ++q) {
+                const float4 b4 = __ldg(reinterpret_cast<const float4*>(e.bias + col0) + q);
+                v[4 * q] += b4.x; v[4 * q + 1] += b4.y; v[4 * q + 2] += b4.z; v[4 * q + 3] += b4.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < col_end) v[j] += __ldg(e.bias + col0 + j);
+            }
           }
           if (e.act == 1) {
 #pragma unroll
@@ -218,12 +226,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               for (int q = 0; q < 4; ++q) {
                 const uint4 x4 = __ldg(reinterpret_cast<const uint4*>(rr) + q);
                 const uint32_t* xw = reinterpret_cast<const uint32_t*>(&x4);
+                float4 g0 = make_float4(1.f, 1.f, 1.f, 1.f), g1 = g0;
+                if (g != nullptr) {
+                  g0 = __ldg(reinterpret_cast<const float4*>(g) + 2 * q);
+                  g1 = __ldg(reinterpret_cast<const float4*>(g) + 2 * q + 1);
+                }
+                const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
                 for (int e2 = 0; e2 < 4; ++e2) {
                   const float2 xf = unpack_bf16x2(xw[e2]);
                   const int j = q * 8 + 2 * e2;
-                  v[j] = xf.x + (g != nullptr ? __ldg(g + j) : 1.f) * v[j];
-                  v[j + 1] = xf.y + (g != nullptr ? __ldg(g + j + 1) : 1.f) * v[j + 1];
+                  v[j] = fmaf(gg[2 * e2], v[j], xf.x);
+                  v[j + 1] = fmaf(gg[2 * e2 + 1], v[j + 1], xf.y);
                 }
               }
             } else {

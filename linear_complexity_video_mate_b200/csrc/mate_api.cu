@@ -22,6 +22,7 @@
 #include "mamba_extras.cuh"
 #include "ssd_backward.cuh"
 #include "dit.cuh"
+#include "tesa_backward.cuh"
 
 using namespace mate;
 
@@ -1259,6 +1260,66 @@ mate_status ln_modulate(const mate_config* c, const void* x, void* h, const floa
 
 extern "C" {
 
+size_t mate_tesa_backward_workspace_bytes(const mate_config* cfg) {
+  if (check_config(cfg) != MATE_OK) return 0;
+  const long long items = (long long)(cfg->T / cfg->wt) * (cfg->H / cfg->wh) * (cfg->W / cfg->ww) * cfg->B * cfg->th;
+  return (size_t)items * 256 * 2 * sizeof(float) + 256;
+}
+
+mate_status tesa_backward(const void* qkv, const void* O, const void* dO, void* dqkv, int shifted,
+                          const mate_config* cfg, void* ws, size_t ws_bytes, mate_stream_t stream) {
+  MATE_TRY(check_config(cfg));
+  if (cfg->dtype != MATE_BF16) return MATE_ERR_UNSUPPORTED;
+  if (qkv == nullptr || O == nullptr || dO == nullptr || dqkv == nullptr || ws == nullptr || !aligned16(qkv) ||
+      !aligned16(O) || !aligned16(dO) || !aligned16(dqkv) || !aligned16(ws))
+    return MATE_ERR_ARG;
+  if (ws_bytes < mate_tesa_backward_workspace_bytes(cfg)) return MATE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  const int a = cfg->th * cfg->tp;
+  const int sft = shifted ? 1 : 0;
+  TesaBwdParams p;
+  p.qkv = static_cast<const __nv_bfloat16*>(qkv);
+  p.ldq = 3 * a;
+  p.qcol = 0;
+  p.kcol = a;
+  p.vcol = 2 * a;
+  p.O = static_cast<const __nv_bfloat16*>(O);
+  p.dO = static_cast<const __nv_bfloat16*>(dO);
+  p.ldo = a;
+  p.ocol = 0;
+  p.dqkv = static_cast<__nv_bfloat16*>(dqkv);
+  p.ldg = 3 * a;
+  p.gq = 0;
+  p.gk = a;
+  p.gv = 2 * a;
+  p.stats = static_cast<float*>(ws);
+  p.B = cfg->B;
+  p.T = cfg->T;
+  p.H = cfg->H;
+  p.W = cfg->W;
+  p.th = cfg->th;
+  p.wt = cfg->wt;
+  p.wh = cfg->wh;
+  p.ww = cfg->ww;
+  p.st = sft ? cfg->st : 0;
+  p.sh = sft ? cfg->sh : 0;
+  p.sw = sft ? cfg->sw : 0;
+  p.shifted = sft;
+  p.scale = 1.f / std::sqrt(static_cast<float>(cfg->tp));
+  p.scale_log2 = 1.4426950408889634f * p.scale;
+  const int items = (cfg->T / cfg->wt) * (cfg->H / cfg->wh) * (cfg->W / cfg->ww) * cfg->B * cfg->th;
+  const size_t s1 = 1024 + kBdqSmem, s2 = 1024 + kBkvSmem;
+  if (!set_smem(tesa_bwd_dq_kernel, s1) || !set_smem(tesa_bwd_dkdv_kernel, s2)) return MATE_ERR_CUDA;
+  trace_begin(MATE_K_TESA_BWD_DQ, st);
+  tesa_bwd_dq_kernel<<<dim3(items, 2), kTesaBwdThreads, s1, st>>>(p);
+  MATE_LAUNCH_CHECK();
+  trace_begin(MATE_K_TESA_BWD_DKDV, st);
+  tesa_bwd_dkdv_kernel<<<dim3(items, 2), kTesaBwdThreads, s2, st>>>(p);
+  MATE_LAUNCH_CHECK();
+  return MATE_OK;
+}
+
 size_t mate_dit_workspace_bytes(const mate_config* cfg) {
   if (check_config(cfg) != MATE_OK || cfg->d > 2048) return 0;
   return plan_dit(cfg, nullptr).bytes;
@@ -1432,6 +1493,8 @@ const char* mate_kernel_name(int kernel) {
     case MATE_K_LN_MODULATE: return "ln_modulate";
     case MATE_K_MLP_UP: return "mlp_up";
     case MATE_K_MLP_DOWN: return "mlp_down";
+    case MATE_K_TESA_BWD_DQ: return "tesa_backward_dq";
+    case MATE_K_TESA_BWD_DKDV: return "tesa_backward_dkdv";
   }
   return "unknown";
 }

@@ -14,7 +14,7 @@ import torch
 from . import _lib
 
 __all__ = ["MateBlock", "DitBlock", "dit_weights_to_device", "rms_permute", "rms_unpermute", "review_pool", "ssd_scan_bidir", "ssd_scan_bidir_pd",
-           "ssd_scan_bidir_noalloc", "ssd_scan_bidir_backward", "tesa_forward", "project_bf16", "device_status",
+           "ssd_scan_bidir_noalloc", "ssd_scan_bidir_backward", "tesa_forward", "tesa_backward", "project_bf16", "device_status",
            "torch_dtype", "weights_to_device", "scan_locality", "KernelTrace"]
 
 
@@ -296,6 +296,27 @@ def tesa_forward(qkv: torch.Tensor, shifted: bool, cfg, out: Optional[torch.Tens
     c = _cfg(cfg)
     _lib.check(_lib.load().tesa_forward(_p(qkv), _p(out), int(bool(shifted)), ctypes.byref(c), _s(stream)),
                "tesa_forward")
+    return out
+
+
+def tesa_backward(qkv: torch.Tensor, O: torch.Tensor, dO: torch.Tensor, shifted: bool, cfg, out=None, ws=None,
+                  stream=None) -> torch.Tensor:
+    """Gradient of tesa_forward with respect to qkv [B, T, H, W, 3 th tp], given its output O and the output
+    gradient dO [B, T, H, W, th tp] (bf16 blocks)."""
+    lib = _lib.load()
+    c = _cfg(cfg)
+    a = cfg.th * cfg.tp
+    n = cfg.B * cfg.T * cfg.H * cfg.W
+    _need(qkv, torch.bfloat16, n * 3 * a, "qkv")
+    _need(O, torch.bfloat16, n * a, "O")
+    _need(dO, torch.bfloat16, n * a, "dO")
+    if out is None:
+        out = torch.empty_like(qkv)
+    nb = lib.mate_tesa_backward_workspace_bytes(ctypes.byref(c))
+    if ws is None or ws.numel() < nb:
+        ws = torch.empty(nb, dtype=torch.uint8, device=qkv.device)
+    _lib.check(lib.tesa_backward(_p(qkv), _p(O), _p(dO), _p(out), int(bool(shifted)), ctypes.byref(c), _p(ws),
+                                 ws.numel(), _s(stream)), "tesa_backward")
     return out
 
 
