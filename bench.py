@@ -411,6 +411,36 @@ def measure_permute(M, torch, cfg, X, stream, hbm_peak, steps=10):
             "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm_peak, "round_trip_exact": ok}
 
 
+def measure_tesa_backward(M, torch, cfg, stream, tf_peak, steps=10):
+    """TESA's backward pass (tesa_backward: dq | dk | dv from qkv, the forward output and its gradient) at
+    the headline workload, timed after the headline region on seeded Gaussian qkv and output gradient;
+    shifted and unshifted layers alternate.  Algorithmic work: five 256 x 256 x tp products per window and
+    head (dV, dP, dS K, dS^T Q and the recomputed scores)."""
+    g = torch.Generator(device="cuda").manual_seed(91)
+    a = cfg.th * cfg.tp
+    rows = cfg.B * cfg.n
+    qkv = torch.randn((rows, 3 * a), generator=g, device="cuda").to(torch.bfloat16)
+    dO = torch.randn((rows, a), generator=g, device="cuda").to(torch.bfloat16)
+    O = M.tesa_forward(qkv, False, cfg)
+    out = torch.empty_like(qkv)
+    for s in range(2):
+        M.tesa_backward(qkv, O, dO, s % 2 == 1, cfg, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(steps):
+        M.tesa_backward(qkv, O, dO, s % 2 == 1, cfg, out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    win = cfg.wt * cfg.wh * cfg.ww
+    flops = 5 * 2.0 * rows * cfg.th * win * cfg.tp
+    del qkv, dO, O, out
+    return {"ms_per_call": ms, "algorithmic_tflops": flops / 1e12, "tflops": flops / (ms * 1e-3) / 1e12,
+            "frac_of_bf16_peak": flops / (ms * 1e-3) / 1e12 / tf_peak, "steps": steps,
+            "forward_tesa_ms": None}
+
+
 def profile_run(M, torch, cfg, w, X, out):
     """Every kernel of the path a few times, untimed, for an ncu capture to select launches from: the
     block over the four layers, the block with the Mamba2 extras, the DiT block, and the standalone
@@ -429,6 +459,13 @@ def profile_run(M, torch, cfg, w, X, out):
     blk = M.DitBlock(cfg, M.weights_to_device(w, cfg), M.dit_weights_to_device(dw, cfg), 256)
     blk.forward(X, torch.as_tensor(c).cuda(), 1, out)
     del blk
+    g = torch.Generator(device="cuda").manual_seed(91)
+    a = cfg.th * cfg.tp
+    qkv = torch.randn((cfg.B * cfg.n, 3 * a), generator=g, device="cuda").to(torch.bfloat16)
+    dO = torch.randn((cfg.B * cfg.n, a), generator=g, device="cuda").to(torch.bfloat16)
+    O = M.tesa_forward(qkv, True, cfg)
+    M.tesa_backward(qkv, O, dO, True, cfg)
+    del qkv, dO, O
     Xp = torch.empty((cfg.B, cfg.n, cfg.d), dtype=X.dtype, device=X.device)
     for o in range(2):
         M.rms_permute(X, o, cfg, Xp)
@@ -643,12 +680,18 @@ def main():
 
     # side measurements, outside the headline region: the block with the rest of the Mamba2 block, and with
     # separate backward-scan parameters; a failure is reported in the line instead of ending the run
-    extras = per_direction = dit = permute = None
+    extras = per_direction = dit = permute = tesa_bwd = None
     try:
         permute = measure_permute(M, torch, cfg, X, stream, hbm_peak)
     except Exception as e:  # noqa: BLE001
         permute = {"error": f"{type(e).__name__}: {e}"}
     if not args.no_extras:
+        try:
+            tesa_bwd = measure_tesa_backward(M, torch, cfg, stream, tf_peak)
+            if "tesa" in per:
+                tesa_bwd["forward_tesa_ms"] = per["tesa"][1] / per["tesa"][0]
+        except Exception as e:  # noqa: BLE001
+            tesa_bwd = {"error": f"{type(e).__name__}: {e}"}
         try:
             dit = measure_dit(M, torch, cfg, w, X, stream, hbm_peak, tf_peak)
         except Exception as e:  # noqa: BLE001
@@ -707,6 +750,7 @@ def main():
         "per_direction_scan": per_direction,
         "dit_block": dit,
         "rms_permute": permute,
+        "tesa_backward": tesa_bwd,
         "clocks": clocks,
         "device_status": status,
     }

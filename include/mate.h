@@ -282,8 +282,8 @@ MATE_API mate_status tesa_forward(const void* qkv, void* O, int shifted, const m
  * softmax of q k^T / sqrt(tp):
  *     dv = P^T dO,   dP = dO v^T,   dS = P (dP - rowsum(dO * O)),   dq = dS k / sqrt(tp),   dk = dS^T q / sqrt(tp).
  * Every token belongs to exactly one window per layer, so each row of dqkv is written once.  bf16 blocks
- * only (MATE_ERR_UNSUPPORTED otherwise); tensor-core products with bf16 operands (P and dS rounded to bf16)
- * and fp32 softmax statistics.  ws: at least mate_tesa_backward_workspace_bytes(cfg) bytes (per window,
+ * only (MATE_ERR_UNSUPPORTED otherwise); tensor-core products on fp16 operands (q, k, v and dO converted
+ * exactly, P and dS rounded to fp16, values beyond the fp16 range saturating) and fp32 softmax statistics.  ws: at least mate_tesa_backward_workspace_bytes(cfg) bytes (per window,
  * head and query: the softmax normaliser and rowsum(dO * O), written by the first kernel, read by the second).
  */
 MATE_API size_t mate_tesa_backward_workspace_bytes(const mate_config* cfg);

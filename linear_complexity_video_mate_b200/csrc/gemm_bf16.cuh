@@ -9,8 +9,10 @@
 //   warp 0      TMA producer: A and B tiles (BK = 64, 128-byte swizzle) into an S-stage ring;
 //   warp 1      MMA issuer (leader CTA): 256 x BN x 16 tcgen05.mma.cta_group::2 into one of two TMEM
 //               accumulators;
-//   warps 2..5  epilogue: tcgen05.ld the finished accumulator, convert, store; the other accumulator
-//               is being filled meanwhile.
+//   warps 2..9  epilogue: tcgen05.ld the finished accumulator, convert, store; the other accumulator
+//               is being filled meanwhile.  Two warps per TMEM lane quadrant, one column half each, so
+//               that a tile's epilogue (bias, GELU, residual, 256 columns) keeps up with a short
+//               (K = 1024) main loop.
 // Optional epilogue side output: columns [dt_col0, dt_col0 + dt_cols) also produce
 // delta = softplus(acc + dt_bias) in fp32 (the Mamba2 step size).  Optional epilogue transforms
 // (GemmEpilogue) serve the DiT block around MATE: bias + GELU for the MLP's first layer, bias and a gated
@@ -60,11 +62,13 @@ struct GemmParams {
   const float* dt_bias;
   const float* dt_bias2;   // optional: a second side output softplus(acc + dt_bias2) at column offset dt_cols
   GemmEpilogue ep;
+  int f16_cols;      // columns [0, f16_cols) are stored as fp16 (saturating), the rest as bf16; a multiple of 32
 };
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmEpiWarps = 8;
+constexpr int kGemmThreads = (2 + kGemmEpiWarps) * 32;   // 320
 
 __host__ __device__ inline uint32_t gemm_stage_bytes(int bn) { return kGemmBM * 128 + bn * 128; }
 
@@ -107,7 +111,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each of the 2 CTAs
+      mbar_init(&tempty[a], 2 * kGemmEpiWarps);  // the epilogue warps of both CTAs
     }
     mbar_fence_init();
     prefetch_tensormap(&tmA);
@@ -174,8 +178,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // epilogue warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1 of this CTA's 128 rows
+    // epilogue warps 2..9 -> TMEM lane quadrants 2, 3, 0, 1, 2, 3, 0, 1 of this CTA's 128 rows; warps 2..5
+    // take the first 128 columns of a tile, warps 6..9 the rest
     const int quad = warp & 3;
+    const int chalf = (warp - 2) >> 2;
     const bool has_ep = p.ep.bias != nullptr || p.ep.act != 0 || p.ep.resid != nullptr;
     int it = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
@@ -188,7 +194,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const bool row_ok = row < p.M;
       __nv_bfloat16* crow = p.C + static_cast<size_t>(row) * p.ldc;
       const int col_end = min(p.N, nb * p.bn + p.bn);
-      for (int c0 = 0; c0 < col_end - nb * p.bn; c0 += 32) {
+      const int c_hi = min(col_end - nb * p.bn, chalf * 128 + 128);
+      for (int c0 = chalf * 128; c0 < c_hi; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256 + c0, r);
         tmem_wait_ld();
@@ -247,21 +254,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
+        const bool f16 = col0 < p.f16_cols;   // the 32-column slice lies wholly on one side
         if (full32) {
           uint4* dst = reinterpret_cast<uint4*>(crow + col0);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 pk;
-            pk.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-            pk.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-            pk.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-            pk.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+            if (f16) {
+              pk.x = pack_f16x2_sat(v[q * 8 + 0], v[q * 8 + 1]);
+              pk.y = pack_f16x2_sat(v[q * 8 + 2], v[q * 8 + 3]);
+              pk.z = pack_f16x2_sat(v[q * 8 + 4], v[q * 8 + 5]);
+              pk.w = pack_f16x2_sat(v[q * 8 + 6], v[q * 8 + 7]);
+            } else {
+              pk.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+              pk.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+              pk.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+              pk.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+            }
             dst[q] = pk;
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (col0 + j < col_end) crow[col0 + j] = __float2bfloat16_rn(v[j]);
+            if (col0 + j < col_end) {
+              if (f16) {
+                const uint32_t hh = pack_f16x2_sat(v[j], 0.f);
+                reinterpret_cast<uint16_t*>(crow)[col0 + j] = static_cast<uint16_t>(hh & 0xffffu);
+              } else {
+                crow[col0 + j] = __float2bfloat16_rn(v[j]);
+              }
+            }
         }
         if (p.delta != nullptr && col0 < p.dt_col0 + p.dt_cols && col0 + 32 > p.dt_col0) {
 #pragma unroll

@@ -116,6 +116,132 @@ __global__ void __launch_bounds__(256) conv_silu_kernel(SeqRows s, int C, const 
   }
 }
 
+// Causal depthwise convolution + SiLU as a tiled stencil: a CTA takes kCvTP consecutive sequence positions
+// x kCvTC channels of one sample, loads those rows plus the kConvK - 1 rows before them into shared memory
+// (every load of the tile in flight at once, rows gathered through the scan-order map), then computes the
+// outputs from shared memory.  Same result as conv_silu_kernel; needs 16-byte vectors (C % V == 0, aligned
+// rows).  Dynamic shared memory: (kCvTP + kConvK - 1) * kCvTC * sizeof(T_).
+constexpr int kCvTP = 64, kCvTC = 256;
+
+template <typename T_>
+__global__ void __launch_bounds__(256) conv_silu_tiled_kernel(SeqRows s, int C, const float* __restrict__ w,
+                                                              const float* __restrict__ bias, T_* __restrict__ out_v,
+                                                              T_* __restrict__ out_r, int ldo, int ntp, int ntc) {
+  extern __shared__ __align__(16) uint8_t cv_smem[];
+  T_* tile = reinterpret_cast<T_*>(cv_smem);   // [kCvTP + kConvK - 1][kCvTC]
+  constexpr int V = 16 / sizeof(T_);
+  constexpr int NV = kCvTC / V;                // vectors per tile row
+  const int L = s.R + s.n;
+  const int t = blockIdx.x;
+  const int ct = t % ntc, pt = (t / ntc) % ntp, b = t / (ntc * ntp);
+  const int pos0 = pt * kCvTP, ch0 = ct * kCvTC;
+  auto row_of = [&](int i, bool& pre) -> long long {
+    pre = i < s.R;
+    return pre ? s.rrow(b, i) : s.vrow(b, i - s.R);
+  };
+  constexpr int RW = kCvTP + kConvK - 1;
+#pragma unroll 4
+  for (int it = threadIdx.x; it < RW * NV; it += blockDim.x) {
+    const int r = it / NV, cv = it % NV;
+    const int i = pos0 - (kConvK - 1) + r, ch = ch0 + cv * V;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (i >= 0 && i < L && ch < C) {
+      bool pre;
+      const long long row = row_of(i, pre);
+      const T_* src = pre ? static_cast<const T_*>(s.xr) + row * s.ldxr : static_cast<const T_*>(s.xv) + row * s.ldxv;
+      v = __ldg(reinterpret_cast<const uint4*>(src + ch));
+    }
+    *reinterpret_cast<uint4*>(tile + r * kCvTC + cv * V) = v;
+  }
+  __syncthreads();
+  const int cv = threadIdx.x % NV, ch = ch0 + cv * V;
+  if (ch >= C) return;
+  float wt[V][kConvK], bs[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) {
+    const float4 q = __ldg(reinterpret_cast<const float4*>(w + (size_t)(ch + e) * kConvK));
+    wt[e][0] = q.x; wt[e][1] = q.y; wt[e][2] = q.z; wt[e][3] = q.w;
+    bs[e] = __ldg(bias + ch + e);
+  }
+  for (int p = threadIdx.x / NV; p < kCvTP; p += blockDim.x / NV) {
+    const int i = pos0 + p;
+    if (i >= L) break;
+    float o[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) o[e] = bs[e];
+#pragma unroll
+    for (int k = 0; k < kConvK; ++k) {   // tile row p + k holds position i - (kConvK - 1) + k
+      float f[V];
+      const uint4 u = *reinterpret_cast<const uint4*>(tile + (p + k) * kCvTC + cv * V);
+      const T_* e8 = reinterpret_cast<const T_*>(&u);
+#pragma unroll
+      for (int e = 0; e < V; ++e) f[e] = to_f32(e8[e]);
+#pragma unroll
+      for (int e = 0; e < V; ++e) o[e] = fmaf(wt[e][k], f[e], o[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < V; ++e) o[e] = silu_f(o[e]);
+    bool pre;
+    const long long row = row_of(i, pre);
+    store_vec<T_, V>((pre ? out_r : out_v) + row * ldo + ch, o);
+  }
+}
+
+// Gated RMSNorm in place with the row held in registers: one warp per row, each lane keeps its MAXQ
+// 16-byte vectors of y and z as loaded (all loads of the row in flight at once), sums (y silu(z))^2, then
+// writes y silu(z) / rms * norm_w from the registers.  C / V <= 32 * MAXQ.
+template <typename T_, int MAXQ>
+__global__ void __launch_bounds__(256) gate_rmsnorm_reg_kernel(T_* __restrict__ y, long long ldy,
+                                                               const T_* __restrict__ z, long long ldz,
+                                                               const float* __restrict__ norm_w, int C,
+                                                               long long rows) {
+  constexpr int V = 16 / sizeof(T_);
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  const int nvec = C / V;
+  for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    T_* yr = y + r * ldy;
+    const T_* zr = z + r * ldz;
+    uint4 yv[MAXQ], zv[MAXQ];
+#pragma unroll
+    for (int q = 0; q < MAXQ; ++q) {
+      const int v = lane + 32 * q;
+      if (v < nvec) {
+        yv[q] = __ldg(reinterpret_cast<const uint4*>(yr + v * V));
+        zv[q] = __ldg(reinterpret_cast<const uint4*>(zr + v * V));
+      }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int q = 0; q < MAXQ; ++q) {
+      if (lane + 32 * q < nvec) {
+        const T_* a = reinterpret_cast<const T_*>(&yv[q]);
+        const T_* c = reinterpret_cast<const T_*>(&zv[q]);
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          const float g = to_f32(a[e]) * silu_f(to_f32(c[e]));
+          ss = fmaf(g, g, ss);
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = rsqrtf(ss / static_cast<float>(C) + kNormEps);
+#pragma unroll
+    for (int q = 0; q < MAXQ; ++q) {
+      const int v = lane + 32 * q;
+      if (v < nvec) {
+        const T_* a = reinterpret_cast<const T_*>(&yv[q]);
+        const T_* c = reinterpret_cast<const T_*>(&zv[q]);
+        float o[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) o[e] = to_f32(a[e]) * silu_f(to_f32(c[e])) * inv * __ldg(norm_w + v * V + e);
+        store_vec<T_, V>(yr + v * V, o);
+      }
+    }
+  }
+}
+
 // Gated RMSNorm in place, one warp per row: g = y * silu(z) over the row's C channels (C a multiple of
 // V), y <- g * rsqrt(mean(g^2) + eps) * norm_w.  The second pass recomputes g from the row, which the
 // first pass left in L1.

@@ -265,7 +265,8 @@ int choose_bn(int N) { return N >= 256 ? 256 : ((N + 15) / 16) * 16; }
 
 mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const void* Bw, int ldb, int N, void* C,
                       int ldc, float* delta, int ld_delta, int dt_col0, int dt_cols, const float* dt_bias,
-                      cudaStream_t st, const float* dt_bias2 = nullptr, const GemmEpilogue* ep = nullptr) {
+                      cudaStream_t st, const float* dt_bias2 = nullptr, const GemmEpilogue* ep = nullptr,
+                      int f16_cols = 0) {
   if (M <= 0) return MATE_OK;
   if (K % kGemmBK) return MATE_ERR_UNSUPPORTED;
   GemmParams p;
@@ -283,6 +284,7 @@ mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const
   p.dt_bias = dt_bias;
   p.dt_bias2 = dt_bias2;
   if (ep != nullptr) p.ep = *ep;
+  p.f16_cols = f16_cols;
   // 256-row tiles computed by 2-CTA clusters (tcgen05 cta_group::2)
   p.num_tiles = ceil_div(M, 256) * p.num_n_tiles;
   const uint32_t psb = gemm_pair_stage_bytes(p.bn);
@@ -392,8 +394,10 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   const size_t smem_gram = 1024 + 98304 + 2048 + 64;
   const size_t smem_state = 1024 + 131072 + 2048 + 64 + 2048 + 64;
   const size_t smem_out = 1024 + kOutSmem;
-  if (!set_smem(ssd_gram_kernel, smem_gram) || !set_smem(ssd_state_kernel, smem_state) ||
-      !set_smem(ssd_output_kernel, smem_out))
+  const bool xf16 = rows.x_f16 != 0;
+  auto state_k = xf16 ? ssd_state_kernel<true> : ssd_state_kernel<false>;
+  auto out_k = xf16 ? ssd_output_kernel<true> : ssd_output_kernel<false>;
+  if (!set_smem(ssd_gram_kernel, smem_gram) || !set_smem(state_k, smem_state) || !set_smem(out_k, smem_out))
     return MATE_ERR_CUDA;
   trace_begin(MATE_K_SSD_GRAM, st);
   ssd_gram_kernel<<<dim3(p.nVc, c->B, 2), 128, smem_gram, st>>>(p);
@@ -401,7 +405,7 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   int hpc = 1;
   while (hpc < 16 && c->nh % (hpc * 2) == 0) hpc *= 2;   // heads per CTA (c3: 2: 0.72 ms, 4: 0.63, 8: 0.58, 16: 0.56)
   trace_begin(MATE_K_SSD_STATE, st);
-  ssd_state_kernel<<<dim3(p.nRc + p.nVc, c->B, c->nh / hpc), 256, smem_state, st>>>(p, hpc);
+  state_k<<<dim3(p.nRc + p.nVc, c->B, c->nh / hpc), 256, smem_state, st>>>(p, hpc);
   MATE_LAUNCH_CHECK();
   trace_begin(MATE_K_SSD_CARRY, st);
   ssd_carry_kernel<<<dim3(kSsdP * kSsdN / 8 / 128, c->nh, 2 * c->B), 128, 0, st>>>(p);
@@ -410,14 +414,15 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   const long long vrows = (long long)c->B * rows.v_bstride;
   mp.rows = static_cast<int>(vrows);
   const long long srows = (long long)c->B * p.nVc * c->nh * 2 * kSsdN;   // hi | lo rows of every state
-  if (!make_tmap(&mp.x, rows.xv, vrows, (long long)c->nh * c->P, rows.ldxv, 1) ||
+  if (!make_tmap(&mp.x, rows.xv, vrows, (long long)c->nh * c->P, rows.ldxv, 1,
+                 xf16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
       !make_tmap(&mp.c, rows.cv, vrows, c->N, rows.ldcv, 1) || !make_tmap(&mp.hf, sc.Hf, srows, kSsdP, kSsdP, 128) ||
       !make_tmap(&mp.hb, sc.Hb, srows, kSsdP, kSsdP, 128) ||
       !make_tmap(&mp.g, sc.Gm, (long long)c->B * p.nVc * kSsdQ, kSsdQ, kSsdQ, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MATE_ERR_CUDA;
   const int out_groups = c->B * p.nVc * 2;
   trace_begin(MATE_K_SSD_OUTPUT, st);
-  ssd_output_kernel<<<std::min(out_groups, device_sms()), kSsdOutThreads, smem_out, st>>>(p, mp);
+  out_k<<<std::min(out_groups, device_sms()), kSsdOutThreads, smem_out, st>>>(p, mp);
   MATE_LAUNCH_CHECK();
   return MATE_OK;
 }
@@ -530,7 +535,21 @@ mate_status run_conv(const mate_config* c, const SeqRows& rows, int Cx, const fl
   const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, (long long)device_sms() * 16));
   if (total == 0) return MATE_OK;
   trace_begin(MATE_K_CONV_SILU, st);
-  if (c->dtype == MATE_BF16) {
+  if (vec && (Cx * es) % 16 == 0) {
+    // tiled stencil: every row load of a tile in flight at once
+    const int ntp = ceil_div(L, kCvTP), ntc = ceil_div(Cx, kCvTC);
+    const long long tiles = (long long)c->B * ntp * ntc;
+    const size_t smem = (size_t)(kCvTP + kConvK - 1) * kCvTC * es;
+    if (c->dtype == MATE_BF16) {
+      if (!set_smem(conv_silu_tiled_kernel<__nv_bfloat16>, smem)) return MATE_ERR_CUDA;
+      conv_silu_tiled_kernel<__nv_bfloat16><<<static_cast<unsigned>(tiles), 256, smem, st>>>(
+          rows, Cx, w, bias, static_cast<__nv_bfloat16*>(out_v), static_cast<__nv_bfloat16*>(out_r), Cx, ntp, ntc);
+    } else {
+      if (!set_smem(conv_silu_tiled_kernel<float>, smem)) return MATE_ERR_CUDA;
+      conv_silu_tiled_kernel<float><<<static_cast<unsigned>(tiles), 256, smem, st>>>(
+          rows, Cx, w, bias, static_cast<float*>(out_v), static_cast<float*>(out_r), Cx, ntp, ntc);
+    }
+  } else if (c->dtype == MATE_BF16) {
     if (vec)
       conv_silu_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(rows, Cx, w, bias, static_cast<__nv_bfloat16*>(out_v),
                                                                 static_cast<__nv_bfloat16*>(out_r), Cx, nruns, c->B);
@@ -561,7 +580,12 @@ mate_status run_gate_norm(const mate_config* c, void* y, int ldy, const void* z,
   if (c->dtype == MATE_BF16) {
     auto* yy = static_cast<__nv_bfloat16*>(y);
     const auto* zz = static_cast<const __nv_bfloat16*>(z);
-    if (vec) gate_rmsnorm_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
+    // rows that fit the registers: each lane holds up to 4 (or 8) 16-byte vectors of y and of z
+    if (vec && C / 8 <= 32 * 4)
+      gate_rmsnorm_reg_kernel<__nv_bfloat16, 4><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
+    else if (vec && C / 8 <= 32 * 8)
+      gate_rmsnorm_reg_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
+    else if (vec) gate_rmsnorm_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
     else gate_rmsnorm_kernel<__nv_bfloat16, 1><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
   } else {
     auto* yy = static_cast<float*>(y);
@@ -645,6 +669,9 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   const int NIn = pl.NIn, NI = pl.NI, KO = pl.KO;
   const int dt0 = dI + 2 * c->N;
   const int ldd = per_dir ? 2 * c->nh : c->nh;                     // delta rows: forward | backward
+  // the scan's x columns of the projections are stored in fp16 (finer intra-chunk operand, packed fp16
+  // arithmetic in the scan output kernel), except on the full-Mamba2 path whose convolution reads bf16
+  const int xf16c = (c->dtype == MATE_BF16 && !extras) ? dI : 0;
   const float* dtb2 = per_dir ? w->dt_bias_b : nullptr;
 
   // packed weights: Wi = [W_in; W_qkv (; W_z)] (NI x d), Wo = [W_out | W_o] (d x KO), from the caller's
@@ -665,15 +692,18 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
       if (r1 <= r0) continue;
       MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, static_cast<const char*>(X) + r0 * c->d * es, c->d, r1 - r0, c->d, pl.Wi,
                          c->d, NI, static_cast<char*>(pl.Zv) + r0 * NI * es, NI, pl.Dv + r0 * ldd, ldd, dt0,
-                         c->nh, w->dt_bias, st, dtb2));
+                         c->nh, w->dt_bias, st, dtb2, nullptr, xf16c));
     }
     MATE_TRY(pool(X, pl.Rv, c, order, st));
     if (!cuda_ok(cudaEventRecord(iop->x_free, st))) return MATE_ERR_CUDA;
-    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, ldd, dt0,
+                       c->nh, w->dt_bias, st, dtb2, nullptr, xf16c));
   } else if (c->dtype == MATE_BF16) {
     MATE_TRY(pool(X, pl.Rv, c, order, st));
-    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, X, c->d, Mv, c->d, pl.Wi, c->d, NI, pl.Zv, NI, pl.Dv, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
-    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, ldd, dt0, c->nh, w->dt_bias, st, dtb2));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ, X, c->d, Mv, c->d, pl.Wi, c->d, NI, pl.Zv, NI, pl.Dv, ldd, dt0, c->nh,
+                       w->dt_bias, st, dtb2, nullptr, xf16c));
+    MATE_TRY(gemm_bf16(MATE_K_IN_PROJ_REVIEW, pl.Rv, c->d, Mr, c->d, pl.Wi, c->d, NIn, pl.Zr, NI, pl.Dr, ldd, dt0,
+                       c->nh, w->dt_bias, st, dtb2, nullptr, xf16c));
   } else {
     MATE_TRY(pool(X, pl.Rv, c, order, st));
     MATE_TRY(gemm_f32(MATE_K_IN_PROJ, static_cast<const float*>(X), c->d, Mv, c->d, static_cast<const float*>(pl.Wi), c->d, NI,
@@ -728,6 +758,7 @@ mate_status forward_impl(const void* X, const mate_weights* w, int layer_idx, vo
   // rows back to grid order afterwards (measured on the B200).
   const bool y_in_scan_order = c->dtype == MATE_BF16 && order >= 2;
   rows.y_order = y_in_scan_order ? -1 : order;
+  rows.x_f16 = xf16c > 0 ? 1 : 0;
   if (y_in_scan_order) {
     MATE_TRY(run_ssd(c, rows, w->A_log, w->D, pl.Ys, dI, n, pl.ssd, st, w->A_log_b, w->D_b));
     const int vec = static_cast<int>(dI * es / 16);

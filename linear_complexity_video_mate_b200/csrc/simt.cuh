@@ -202,6 +202,7 @@ struct SeqRows {
   int db_off;    // column offset of the backward direction's delta in the delta rows (0: shared delta)
   int order;     // scan order of the video input rows (row of scan position q: scan_to_raster(q)); -1: identity
   int y_order;   // scan order of the output rows (y of scan position q goes to row map(q)); -1: identity
+  int x_f16 = 0; // bf16 tensor-core scan: the x rows are fp16 (1) or bf16 (0); B and C rows are bf16
   __host__ __device__ __forceinline__ int map(int q) const {
     return y_order < 0 ? q : scan_to_raster(q, T, H, W, y_order);
   }

@@ -26,6 +26,12 @@
 //   ssd_carry_kernel   sequential carry over chunks: H_in(next) = exp(s_last) H_in + S     [CUDA cores]
 //   ssd_output_kernel  y for one (video chunk, head): M x + row-scaled C Hf^T, C Hb^T      [tcgen05]
 //
+// fp16 x.  When the x rows are fp16 (the block stores its projected x in fp16), the output kernel forms M
+// with packed fp16 multiplies from fp16 column-factor tables and runs M x as an fp16 MMA: fewer ALU
+// operations per element and an intra-chunk operand 8 times finer than bf16.  |M_ij| = |C_i . B_j| delta_j
+// dec(i, j) must then stay below 65504 (the products are not saturated).  With bf16 x (the standalone entry
+// points) M is formed in fp32 and rounded once to bf16.
+//
 // Precision.  States, decays and accumulations are fp32.  The chunk states S are stored in fp32; the
 // carried states H, an operand of the C H^T product, are stored as a bf16 pair hi + lo (hi = bf16(H),
 // lo = bf16(H - hi)) and multiplied as two accumulating products, which keeps about 16 bits of H.  G and
@@ -50,6 +56,7 @@ constexpr int kSsdN = 128;   // state size
 //   uf, ub   row factors exp(s_i - s_{64 ib - 1}), exp(s'_{64 ib + 64} - s'_i) of row block ib = i / 64
 //   si, sx   s_i log2(e), s'_i log2(e)               ef, eb  exp(s_i), exp(s_last - s'_i)
 //   dl       delta_i                                  wf, wb  [2][256] column factors of row blocks 2t, 2t + 1
+//                                                             (fp16, first half of the slot, for fp16 x)
 //   lf, lb   log2(delta_j) - s_j log2(e), log2(delta_j) + s'_j log2(e) for the tile's own columns
 // (s inclusive and s' = s - delta A exclusive cumulative sums of delta A over the chunk).
 constexpr int kTUf = 0, kTUb = 128, kTSi = 256, kTSx = 384, kTEf = 512, kTEb = 640, kTDl = 768, kTWf = 896,
@@ -269,6 +276,7 @@ __global__ void __launch_bounds__(128, 1) ssd_gram_kernel(const SsdBf16Params p)
 // weighted x tile (MN-major), M = N_state = 128, N = P = 64, K = Q = 256; both operands fp16 (the B
 // rows are converted once per chunk, the weighted x per head), states written in fp32.
 // ---------------------------------------------------------------------------------------------------
+template <bool XF16>
 __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p, int heads_per_cta) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -385,9 +393,17 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
       T[kTLb + r] = l2db + sx * kLog2e;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {   // column factors of row block q (stored with the tile holding it)
-        float* W = T0 + (q >> 1) * kOutTbl + (q & 1) * 256 + j;
-        W[kTWf] = (q > 0 && j < 64 * q) ? dl * __expf(bnd[q - 1] - s) : 0.f;
-        W[kTWb] = (q < 3 && j >= 64 * q + 64) ? dlb * __expf(sx - bnd[4 + q]) : 0.f;
+        const float wfv = (q > 0 && j < 64 * q) ? dl * __expf(bnd[q - 1] - s) : 0.f;
+        const float wbv = (q < 3 && j >= 64 * q + 64) ? dlb * __expf(sx - bnd[4 + q]) : 0.f;
+        if (XF16) {
+          float* Tq = T0 + (q >> 1) * kOutTbl;
+          reinterpret_cast<__half*>(Tq + kTWf)[(q & 1) * 256 + j] = __float2half_rn(wfv);
+          reinterpret_cast<__half*>(Tq + kTWb)[(q & 1) * 256 + j] = __float2half_rn(wbv);
+        } else {
+          float* W = T0 + (q >> 1) * kOutTbl + (q & 1) * 256 + j;
+          W[kTWf] = wfv;
+          W[kTWb] = wbv;
+        }
       }
     }
     if (threadIdx.x == 0 && per_dir) p.glb[(static_cast<long long>(b) * nC + c) * p.nh + h] = sb_last;
@@ -408,7 +424,7 @@ __global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p
       uint32_t* pb = reinterpret_cast<uint32_t*>(&ob);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 f = unpack_bf16x2(xw[e]);
+        const float2 f = XF16 ? unpack_f16x2(xw[e]) : unpack_bf16x2(xw[e]);
         pf[e] = pack_f16x2_sat(f.x * wf, f.y * wf);
         pb[e] = pack_f16x2_sat(f.x * wb, f.y * wb);
       }
@@ -603,6 +619,7 @@ struct SsdOutMaps {
   int rows;   // row extent of the x / C maps; gathers of invalid rows use this (out of range -> zeros)
 };
 
+template <bool XF16>
 __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const SsdBf16Params p,
                                                                         const __grid_constant__ SsdOutMaps mp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -754,7 +771,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
   } else if (warp == kOutMmaWarp) {
     // ------------------------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t idesc_d = idesc_bf16_f32(128, 64, 0, 1);    // Yd: N = P
+      // Yd: N = P, fp16 operands when x is fp16
+      const uint32_t idesc_d = XF16 ? idesc_f16_f32(128, 64, 0, 1) : idesc_bf16_f32(128, 64, 0, 1);
       const uint32_t idesc_h = idesc_bf16_f32(128, 128, 0, 1);   // [Yf | Yb]: N = 2 P, B = [Hf | Hb]
       const uint32_t cbase = smem_u32(smem + kOutOffC), hbase = smem_u32(smem + kOutOffH);
       int k = 0, kg = 0;
@@ -830,7 +848,20 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           if (h == 0 && !wait_all(&g_full[cb], kg & 1)) { ok = false; break; }
           const uint8_t* grow = smem + kOutOffG + cb * 16384 + r * 128;
           const uint32_t tcol = tm_row + cb * 32;
-          if (cb != ib) {
+          if (cb != ib && XF16) {
+            // M = (G w) u in packed fp16: two multiplies per element pair
+            const uint32_t uu = pack_f16x2_sat(cb < ib ? ufi : ubi, cb < ib ? ufi : ubi);
+            const __half* wh = reinterpret_cast<const __half*>(tb + (cb < ib ? kTWf : kTWb)) + (ib - 2 * t) * 256 +
+                               cb * 64 + half * 8;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const int ch = 2 * qq + half;
+              const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
+              const uint4 wv = *reinterpret_cast<const uint4*>(wh + qq * 16);
+              tmem_st4(tcol + qq * 8, mul_f16x2(mul_f16x2(gc.x, wv.x), uu), mul_f16x2(mul_f16x2(gc.y, wv.y), uu),
+                       mul_f16x2(mul_f16x2(gc.z, wv.z), uu), mul_f16x2(mul_f16x2(gc.w, wv.w), uu));
+            }
+          } else if (cb != ib) {
             const float u = cb < ib ? ufi : ubi;
             const float2 uu = make_float2(u, u);
             const float* w = (cb < ib ? wfr : wbr) + cb * 64 + half * 8;
@@ -875,8 +906,12 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
               uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const float2 gm = mul_f32x2(unpack_f16x2(gu[e]), make_float2(m[2 * e], m[2 * e + 1]));
-                pk[e] = pack_bf16x2(gm.x, gm.y);
+                if (XF16) {
+                  pk[e] = mul_f16x2(gu[e], pack_f16x2_sat(m[2 * e], m[2 * e + 1]));
+                } else {
+                  const float2 gm = mul_f32x2(unpack_f16x2(gu[e]), make_float2(m[2 * e], m[2 * e + 1]));
+                  pk[e] = pack_bf16x2(gm.x, gm.y);
+                }
               }
               tmem_st4(tcol + qq * 8, pk[0], pk[1], pk[2], pk[3]);
             }
@@ -938,7 +973,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
             uint32_t ou[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float2 xf = unpack_bf16x2(xw[pc * 8 + e]);
+              const float2 xf = XF16 ? unpack_f16x2(xw[pc * 8 + e]) : unpack_bf16x2(xw[pc * 8 + e]);
               const int k0 = 2 * e;
               const float y0 = __uint_as_float(yd[k0]) + ef * __uint_as_float(yf[k0]) +
                                eb * __uint_as_float(yb[k0]) + D2 * xf.x;

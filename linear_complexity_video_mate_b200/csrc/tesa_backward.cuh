@@ -12,6 +12,10 @@
 //   tesa_bwd_dkdv_kernel  key block kb: for the two query tiles in turn, S and dP against the block's 128
 //                         keys, P and dS from the stored statistics (bf16 into shared memory, read MN-major
 //                         as the A operand), and dV += P^T dO, dK += dS^T Q in TMEM columns [256, 512).
+// Precision: the products run on fp16 operands.  q, k, v and dO are bf16 in memory and convert to fp16
+// exactly on the way into shared memory; P and dS are rounded to fp16 (8 times finer than bf16: dQ and dK
+// sum dS terms that cancel, since every row of dS sums to zero, so their relative error is amplified).
+// Values beyond the fp16 range saturate at +-65504.
 // One thread issues the MMAs; all 8 warps do the elementwise work (two warps per TMEM lane quadrant, one
 // column half each).  Bounded waits as everywhere in the library: a wait that runs out flags the device
 // status word and the CTA skips the rest of its item.
@@ -48,6 +52,18 @@ struct TesaBwdRows {
   float delta[256];
   int mixed;
 };
+
+// The 8 bf16 values of a 16-byte shared-memory chunk converted to fp16 in place (exact inside the fp16
+// range).  Operands arrive by cp.async (all of an item's copies in flight at once); each thread converts
+// the chunks it copied itself, after its own copies have landed.
+__device__ __forceinline__ void tesa_bwd_to_f16(uint8_t* p) {
+  uint4 v = *reinterpret_cast<const uint4*>(p);
+  float2 f = unpack_bf16x2(v.x); v.x = pack_f16x2_sat(f.x, f.y);
+  f = unpack_bf16x2(v.y); v.y = pack_f16x2_sat(f.x, f.y);
+  f = unpack_bf16x2(v.z); v.z = pack_f16x2_sat(f.x, f.y);
+  f = unpack_bf16x2(v.w); v.w = pack_f16x2_sat(f.x, f.y);
+  *reinterpret_cast<uint4*>(p) = v;
+}
 
 // Row table of an item (all 256 window tokens); returns whether the window mixes wrap regions.
 __device__ __forceinline__ bool tesa_bwd_rows(const TesaBwdParams& p, int item, TesaBwdRows& rt, int& hd) {
@@ -124,13 +140,23 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dq_kernel(const T
   }
   cp_async_commit();
   cp_async_wait<0>();
+  for (int it = threadIdx.x; it < 256 * 16; it += kTesaBwdThreads) {
+    const uint32_t off = sw128_kmajor_offset(it >> 4, (it & 15) * 8, 32768);
+    tesa_bwd_to_f16(sK + off);
+    tesa_bwd_to_f16(sV + off);
+  }
+  for (int it = threadIdx.x; it < 128 * 16; it += kTesaBwdThreads) {
+    const uint32_t off = sw128_kmajor_offset(it >> 4, (it & 15) * 8, 16384);
+    tesa_bwd_to_f16(sQ + off);
+    tesa_bwd_to_f16(sDO + off);
+  }
   fence_proxy_async();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
   const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV), o0 = smem_u32(sDO);
   if (threadIdx.x == 0) {
-    const uint32_t idesc = idesc_bf16_f32(128, 256, 0, 0);
+    const uint32_t idesc = idesc_f16_f32(128, 256, 0, 0);
 #pragma unroll
     for (int s = 0; s < 8; ++s) {   // S = Q K^T and dP = dO V^T, K = 128 dims
       const uint32_t off = (s & 3) * 32;
@@ -181,7 +207,7 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dq_kernel(const T
       const uint32_t* dw = reinterpret_cast<const uint32_t*>(&dv);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 a = unpack_bf16x2(ow[e]), g = unpack_bf16x2(dw[e]);
+        const float2 a = unpack_bf16x2(ow[e]), g = unpack_f16x2(dw[e]);
         dl = fmaf(a.x, g.x, fmaf(a.y, g.y, dl));
       }
     }
@@ -198,7 +224,7 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dq_kernel(const T
       sp[0] = L2;
       sp[1] = delta;
     }
-    // dS = P (dP - delta) in bf16, K-major [128 q][256 keys] in the V buffer (dP has been computed)
+    // dS = P (dP - delta) in fp16, K-major [128 q][256 keys] in the V buffer (dP has been computed)
     for (int c0 = hf * 128; c0 < hf * 128 + 128; c0 += 32) {
       uint32_t s[32], g[32];
       tmem_ld32(trow + c0, s);
@@ -216,7 +242,7 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dq_kernel(const T
             if (rt.code[c0 + u] != myc) p0 = 0.f;
             if (rt.code[c0 + u + 1] != myc) p1 = 0.f;
           }
-          pk[e] = pack_bf16x2(p0 * (__uint_as_float(g[u]) - delta), p1 * (__uint_as_float(g[u + 1]) - delta));
+          pk[e] = pack_f16x2_sat(p0 * (__uint_as_float(g[u]) - delta), p1 * (__uint_as_float(g[u + 1]) - delta));
         }
         *reinterpret_cast<uint4*>(sV + sw128_kmajor_offset(r, c0 + u8, 16384)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
@@ -227,7 +253,7 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dq_kernel(const T
   __syncthreads();
   if (ok && threadIdx.x == 0) {
     tc_fence_after();
-    const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);
+    const uint32_t idesc = idesc_f16_f32(128, 128, 0, 1);
 #pragma unroll
     for (int s = 0; s < 16; ++s)   // dQ = dS K: A = dS K-major, B = K rows read MN-major (N = dims)
       mma_bf16_ss(tmem, desc_sw128(v0 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), desc_sw128(k0 + s * 2048, 32768, 1024),
@@ -325,11 +351,20 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dkdv_kernel(const
     }
     cp_async_commit();
     cp_async_wait<0>();
+    for (int it = threadIdx.x; it < 128 * 16; it += kTesaBwdThreads) {
+      const uint32_t off = sw128_kmajor_offset(it >> 4, (it & 15) * 8, 16384);
+      tesa_bwd_to_f16(sQ + off);
+      tesa_bwd_to_f16(sDO + off);
+      if (t == 0) {   // the key block's K and V (copied by this thread in the same pattern) on the first tile
+        tesa_bwd_to_f16(sK + off);
+        tesa_bwd_to_f16(sV + off);
+      }
+    }
     fence_proxy_async();
     __syncthreads();
     if (threadIdx.x == 0) {
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t idesc = idesc_f16_f32(128, 128, 0, 0);
 #pragma unroll
       for (int s = 0; s < 8; ++s) {   // S = Q_t K_kb^T, dP = dO_t V_kb^T
         const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
@@ -362,8 +397,8 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dkdv_kernel(const
               if (rt.code[kb * 128 + c0 + u] != myc) a0 = 0.f;
               if (rt.code[kb * 128 + c0 + u + 1] != myc) a1 = 0.f;
             }
-            pp[e] = pack_bf16x2(a0, a1);
-            pd[e] = pack_bf16x2(a0 * (__uint_as_float(g[u]) - delta), a1 * (__uint_as_float(g[u + 1]) - delta));
+            pp[e] = pack_f16x2_sat(a0, a1);
+            pd[e] = pack_f16x2_sat(a0 * (__uint_as_float(g[u]) - delta), a1 * (__uint_as_float(g[u + 1]) - delta));
           }
           const uint32_t off = sw128_mnmajor_offset(r, c0 + u8, 16384);
           *reinterpret_cast<uint4*>(sP + off) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
@@ -376,7 +411,7 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dkdv_kernel(const
     __syncthreads();
     if (ok && threadIdx.x == 0) {
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, 128, 1, 1);
+      const uint32_t idesc = idesc_f16_f32(128, 128, 1, 1);
 #pragma unroll
       for (int s = 0; s < 8; ++s) {   // dV += P^T dO_t, dK += dS^T Q_t: K = the tile's 128 queries
         mma_bf16_ss(tmem + 256, desc_sw128(p0 + s * 2048, 16384, 1024), desc_sw128(o0 + s * 2048, 16384, 1024), idesc,
@@ -414,7 +449,6 @@ __global__ void __launch_bounds__(kTesaBwdThreads, 1) tesa_bwd_dkdv_kernel(const
       }
     }
   }
-  cp_async_wait<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

@@ -222,31 +222,36 @@ __global__ void __launch_bounds__(kTesaThreads, 1) tesa_bf16_kernel(const TesaBf
       const int myc = rt.code[i];
       if (__any_sync(0xffffffffu, !mbar_wait(s_full, k & 1))) break;
       tc_fence_after();
+      // two 32-column TMEM loads in flight per wait
       float mx = -INFINITY;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        uint32_t v[32];
+      for (int c0 = 0; c0 < 256; c0 += 64) {
+        uint32_t v[32], w[32];
         tmem_ld32(srow_t + c0, v);
+        tmem_ld32(srow_t + c0 + 32, w);
         tmem_wait_ld();
         if (has_mask) {
 #pragma unroll
-          for (int u = 0; u < 32; ++u)
+          for (int u = 0; u < 32; ++u) {
             if (rt.code[c0 + u] == myc) mx = fmaxf(mx, __uint_as_float(v[u]));
+            if (rt.code[c0 + 32 + u] == myc) mx = fmaxf(mx, __uint_as_float(w[u]));
+          }
         } else {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) mx = fmaxf(mx, __uint_as_float(v[u]));
+          for (int u = 0; u < 32; ++u) mx = fmaxf(mx, fmaxf(__uint_as_float(v[u]), __uint_as_float(w[u])));
         }
       }
       const float mxs = mx * p.scale_log2;
       float sum = 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(srow_t + c0, v);
+      for (int c0 = 0; c0 < 256; c0 += 64) {
+        uint32_t v[64];
+        tmem_ld32(srow_t + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(srow_t + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t pk[32];
 #pragma unroll
-        for (int u = 0; u < 32; u += 2) {
+        for (int u = 0; u < 64; u += 2) {
           float e0 = ex2_approx(fmaf(__uint_as_float(v[u]), p.scale_log2, -mxs));
           float e1 = ex2_approx(fmaf(__uint_as_float(v[u + 1]), p.scale_log2, -mxs));
           if (has_mask) {
@@ -256,7 +261,9 @@ __global__ void __launch_bounds__(kTesaThreads, 1) tesa_bf16_kernel(const TesaBf
           sum += e0 + e1;
           pk[u / 2] = pack_bf16x2(e0, e1);
         }
-        tmem_st16(srow_t + c0 / 2, pk);   // columns [c0 / 2, c0 / 2 + 16) were read already
+        // columns [c0 / 2, c0 / 2 + 32) were read already (they lie below c0 + 64)
+        tmem_st16(srow_t + c0 / 2, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+        tmem_st16(srow_t + c0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -266,13 +273,14 @@ __global__ void __launch_bounds__(kTesaThreads, 1) tesa_bf16_kernel(const TesaBf
       if (__any_sync(0xffffffffu, !mbar_wait(o_full, k & 1))) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(srow_t + 128 + c0, v);
+      for (int c0 = 0; c0 < 128; c0 += 64) {
+        uint32_t v[64];
+        tmem_ld32(srow_t + 128 + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(srow_t + 128 + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
         uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 8; ++q) {
           uint4 pk;
           pk.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]) * inv, __uint_as_float(v[q * 8 + 1]) * inv);
           pk.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]) * inv, __uint_as_float(v[q * 8 + 3]) * inv);

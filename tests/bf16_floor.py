@@ -88,12 +88,15 @@ def _split(a):
 
 # Rounding points of the tensor-core scan, for the error decomposition.  "bf16_states" is the scan as
 # first built (G, the decay-weighted inputs of the chunk states, the chunk states and the carried states
-# all in bf16); "kernel" is the scan as it now runs (G and the weighted inputs in fp16, chunk states in
-# fp32, carried states as a bf16 hi + lo pair); in both the intra-chunk matrix M is a bf16 MMA operand
-# and the output y is stored in bf16.
+# all in bf16); "kernel" is the scan as it now runs on bf16 x (the standalone entry points: G and the
+# weighted inputs in fp16, chunk states in fp32, carried states as a bf16 hi + lo pair, the intra-chunk
+# matrix M a bf16 MMA operand); "kernel_f16x" is the block's scan, whose x rows the in-projection stores
+# in fp16, with M an fp16 operand.  The output y is stored in bf16 in all of them.
+_id = lambda a: a
 SCAN_ROUNDING = {
-    "bf16_states": dict(G=_r, W=_r, S=_r, H=_r),
-    "kernel": dict(G=_h, W=_h, S=lambda a: a, H=_split),
+    "bf16_states": dict(G=_r, W=_r, S=_r, H=_r, M=_r, X=_r),
+    "kernel": dict(G=_h, W=_h, S=_id, H=_split, M=_r, X=_r),
+    "kernel_f16x": dict(G=_h, W=_h, S=_id, H=_split, M=_h, X=_h),
 }
 
 
@@ -143,7 +146,7 @@ def ssd_rounding_emulation(x, Bm, Cm, delta, A, D, R, Q=256, scheme="kernel"):
             j = np.arange(m)[None, :]
             dec = np.where(j < i, np.exp(np.minimum(s[:, None] - s[None, :], 0)),
                            np.where(j > i, np.exp(np.minimum(sx[None, :] - sx[:, None], 0)), 0.0))
-            M = _r(rp["G"](G) * delta[a0:a1, h][None, :] * dec)
+            M = rp["M"](rp["G"](G) * delta[a0:a1, h][None, :] * dec)
             y = M @ x[a0:a1, h] + np.exp(s)[:, None] * (Cm[a0:a1] @ Hf[v].T) + \
                 np.exp(s[-1] - sx)[:, None] * (Cm[a0:a1] @ Hb[v].T)
             y += 2 * (np.diag(G) * delta[a0:a1, h] + D[h])[:, None] * x[a0:a1, h]
@@ -163,7 +166,7 @@ def rounding_emulation_forward(X, w, cfg, layer, scheme="kernel"):
         Rv = _r(O.review_tokens(X3, cfg.R, order))
         S = np.concatenate([Rv, Xp], axis=0)
         x, Bm, Cm, delta = O.in_projection(S, w, cfg)
-        x, Bm, Cm = _r(x), _r(Bm), _r(Cm)
+        x, Bm, Cm = SCAN_ROUNDING[scheme]["X"](x), _r(Bm), _r(Cm)
         A = -np.exp(np.asarray(w["A_log"], np.float64))
         y = ssd_rounding_emulation(x, Bm, Cm, delta, A, np.asarray(w["D"], np.float64), cfg.R, cfg.Q,
                                    scheme).reshape(T * H * W, -1)

@@ -94,7 +94,7 @@ BIG_BYTES = 8 << 20
 
 
 def oracle_cached(key: str, fn, extra=()):
-    """fn() -> np.ndarray, cached on disk (as float32: far below every tolerance) under a key that includes
+    """fn() -> np.ndarray, cached on disk (see store_dtype: far below every tolerance) under a key that includes
     the oracle's source digest (plus the files `extra` names; keys holding "floor" also digest
     tests/bf16_floor.py, which computes the floors).  Small results and large ones are kept in separate
     folders."""
@@ -108,9 +108,19 @@ def oracle_cached(key: str, fn, extra=()):
     d = CACHE_BIG if out.size * 4 > BIG_BYTES else CACHE
     os.makedirs(d, exist_ok=True)
     path = os.path.join(d, name)
-    np.save(path + ".tmp.npy", out.astype(np.float32))
+    np.save(path + ".tmp.npy", out.astype(store_dtype(out)))
     os.replace(path + ".tmp.npy", path)
     return out
+
+
+def store_dtype(a):
+    """Storage type of a cached result: float16 for large arrays (relative rounding 2^-11, forty times below
+    the bf16 tolerances; only bf16 test cases produce arrays this large, and finite values below 65504) and
+    float32 otherwise (the fp32 test cases' results, compared at 1e-4, are all small)."""
+    a = np.asarray(a)
+    if a.size > (1 << 18) and np.isfinite(a).all() and np.abs(a).max() < 6e4:
+        return np.float16
+    return np.float32
 
 
 def gpu_ready():
