@@ -50,7 +50,8 @@ __device__ __forceinline__ void store_vec(T_* p, const float (&f)[V]) {
   }
 }
 
-__device__ __forceinline__ float silu_f(float v) { return v / (1.f + __expf(-v)); }
+// SiLU with the fast divide (a few ulp; for v < -88 the quotient is 0, the value rounded to zero anyway).
+__device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.f + __expf(-v)); }
 
 // Causal depthwise convolution + SiLU.  Sequence position i of sample b reads the source row of s (prefix
 // row rrow(b, i) of s.xr for i < R, else video row vrow(b, i - R) of s.xv, row strides s.ldxr / s.ldxv)
@@ -131,27 +132,44 @@ __global__ void __launch_bounds__(256) conv_silu_tiled_kernel(SeqRows s, int C, 
   T_* tile = reinterpret_cast<T_*>(cv_smem);   // [kCvTP + kConvK - 1][kCvTC]
   constexpr int V = 16 / sizeof(T_);
   constexpr int NV = kCvTC / V;                // vectors per tile row
+  constexpr int RW = kCvTP + kConvK - 1;
+  constexpr int NIT = (RW * NV + 255) / 256;   // tile vectors per thread
+  __shared__ long long s_row[RW];              // source row of each tile row (-1 outside the sequence)
+  __shared__ int s_pre[RW];                    // 1: a review-prefix row
   const int L = s.R + s.n;
   const int t = blockIdx.x;
   const int ct = t % ntc, pt = (t / ntc) % ntp, b = t / (ntc * ntp);
   const int pos0 = pt * kCvTP, ch0 = ct * kCvTC;
-  auto row_of = [&](int i, bool& pre) -> long long {
-    pre = i < s.R;
-    return pre ? s.rrow(b, i) : s.vrow(b, i - s.R);
-  };
-  constexpr int RW = kCvTP + kConvK - 1;
-#pragma unroll 4
-  for (int it = threadIdx.x; it < RW * NV; it += blockDim.x) {
-    const int r = it / NV, cv = it % NV;
-    const int i = pos0 - (kConvK - 1) + r, ch = ch0 + cv * V;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (i >= 0 && i < L && ch < C) {
-      bool pre;
-      const long long row = row_of(i, pre);
-      const T_* src = pre ? static_cast<const T_*>(s.xr) + row * s.ldxr : static_cast<const T_*>(s.xv) + row * s.ldxv;
-      v = __ldg(reinterpret_cast<const uint4*>(src + ch));
+  for (int r = threadIdx.x; r < RW; r += blockDim.x) {
+    const int i = pos0 - (kConvK - 1) + r;
+    long long row = -1;
+    int pre = 0;
+    if (i >= 0 && i < L) {
+      pre = i < s.R;
+      row = pre ? s.rrow(b, i) : s.vrow(b, i - s.R);
     }
-    *reinterpret_cast<uint4*>(tile + r * kCvTC + cv * V) = v;
+    s_row[r] = row;
+    s_pre[r] = pre;
+  }
+  __syncthreads();
+  uint4 v[NIT];
+#pragma unroll
+  for (int k = 0; k < NIT; ++k) {
+    const int it = threadIdx.x + k * 256;
+    const int r = it / NV, cv = it % NV, ch = ch0 + cv * V;
+    v[k] = make_uint4(0, 0, 0, 0);
+    if (it < RW * NV && ch < C) {
+      const long long row = s_row[r];
+      if (row >= 0) {
+        const T_* src = s_pre[r] ? static_cast<const T_*>(s.xr) + row * s.ldxr : static_cast<const T_*>(s.xv) + row * s.ldxv;
+        v[k] = __ldg(reinterpret_cast<const uint4*>(src + ch));
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NIT; ++k) {
+    const int it = threadIdx.x + k * 256;
+    if (it < RW * NV) *reinterpret_cast<uint4*>(tile + (it / NV) * kCvTC + (it % NV) * V) = v[k];
   }
   __syncthreads();
   const int cv = threadIdx.x % NV, ch = ch0 + cv * V;
@@ -181,9 +199,8 @@ __global__ void __launch_bounds__(256) conv_silu_tiled_kernel(SeqRows s, int C, 
     }
 #pragma unroll
     for (int e = 0; e < V; ++e) o[e] = silu_f(o[e]);
-    bool pre;
-    const long long row = row_of(i, pre);
-    store_vec<T_, V>((pre ? out_r : out_v) + row * ldo + ch, o);
+    const long long row = s_row[p + kConvK - 1];
+    store_vec<T_, V>((s_pre[p + kConvK - 1] ? out_r : out_v) + row * ldo + ch, o);
   }
 }
 
@@ -231,11 +248,18 @@ __global__ void __launch_bounds__(256) gate_rmsnorm_reg_kernel(T_* __restrict__ 
     for (int q = 0; q < MAXQ; ++q) {
       const int v = lane + 32 * q;
       if (v < nvec) {
+        // the gated values are formed again (the same operations, so the same values) rather than held
         const T_* a = reinterpret_cast<const T_*>(&yv[q]);
         const T_* c = reinterpret_cast<const T_*>(&zv[q]);
         float o[V];
 #pragma unroll
-        for (int e = 0; e < V; ++e) o[e] = to_f32(a[e]) * silu_f(to_f32(c[e])) * inv * __ldg(norm_w + v * V + e);
+        for (int e = 0; e < V; e += 4) {
+          const float4 wv = __ldg(reinterpret_cast<const float4*>(norm_w + v * V + e));
+          o[e] = to_f32(a[e]) * silu_f(to_f32(c[e])) * inv * wv.x;
+          o[e + 1] = to_f32(a[e + 1]) * silu_f(to_f32(c[e + 1])) * inv * wv.y;
+          o[e + 2] = to_f32(a[e + 2]) * silu_f(to_f32(c[e + 2])) * inv * wv.z;
+          o[e + 3] = to_f32(a[e + 3]) * silu_f(to_f32(c[e + 3])) * inv * wv.w;
+        }
         store_vec<T_, V>(yr + v * V, o);
       }
     }

@@ -392,7 +392,7 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   p.ldy = ldy;
   p.y_bstride = y_bstride;
   const size_t smem_gram = 1024 + 98304 + 2048 + 64;
-  const size_t smem_state = 1024 + 131072 + 2048 + 64 + 2048 + 64;
+  const size_t smem_state = 1024 + kStSmem;
   const size_t smem_out = 1024 + kOutSmem;
   const bool xf16 = rows.x_f16 != 0;
   auto state_k = xf16 ? ssd_state_kernel<true> : ssd_state_kernel<false>;
@@ -402,10 +402,21 @@ mate_status run_ssd(const mate_config* c, const SeqRows& rows, const float* A_lo
   trace_begin(MATE_K_SSD_GRAM, st);
   ssd_gram_kernel<<<dim3(p.nVc, c->B, 2), 128, smem_gram, st>>>(p);
   MATE_LAUNCH_CHECK();
-  int hpc = 1;
-  while (hpc < 16 && c->nh % (hpc * 2) == 0) hpc *= 2;   // heads per CTA (c3: 2: 0.72 ms, 4: 0.63, 8: 0.58, 16: 0.56)
+  SsdStateMaps smp;
+  {
+    const CUtensorMapDataType xt = xf16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const long long rv = (long long)c->B * rows.v_bstride, rr = (long long)c->B * rows.r_bstride;
+    smp.rows_v = static_cast<int>(rv);
+    smp.rows_r = static_cast<int>(rr);
+    if (!make_tmap(&smp.xv, rows.xv, rv, (long long)c->nh * c->P, rows.ldxv, 1, xt)) return MATE_ERR_CUDA;
+    if (p.nRc > 0) {
+      if (!make_tmap(&smp.xr, rows.xr, rr, (long long)c->nh * c->P, rows.ldxr, 1, xt)) return MATE_ERR_CUDA;
+    } else {
+      smp.xr = smp.xv;   // no review chunks: never read
+    }
+  }
   trace_begin(MATE_K_SSD_STATE, st);
-  state_k<<<dim3(p.nRc + p.nVc, c->B, c->nh / hpc), 256, smem_state, st>>>(p, hpc);
+  state_k<<<std::min(c->B * (p.nRc + p.nVc), device_sms()), kStThreads, smem_state, st>>>(p, smp);
   MATE_LAUNCH_CHECK();
   trace_begin(MATE_K_SSD_CARRY, st);
   ssd_carry_kernel<<<dim3(kSsdP * kSsdN / 8 / 128, c->nh, 2 * c->B), 128, 0, st>>>(p);
@@ -581,9 +592,10 @@ mate_status run_gate_norm(const mate_config* c, void* y, int ldy, const void* z,
     auto* yy = static_cast<__nv_bfloat16*>(y);
     const auto* zz = static_cast<const __nv_bfloat16*>(z);
     // rows that fit the registers: each lane holds up to 4 (or 8) 16-byte vectors of y and of z
-    if (vec && C / 8 <= 32 * 4)
+    const bool wvec = aligned16(norm_w);   // the register kernel reads the norm weights as float4
+    if (vec && wvec && C / 8 <= 32 * 4)
       gate_rmsnorm_reg_kernel<__nv_bfloat16, 4><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
-    else if (vec && C / 8 <= 32 * 8)
+    else if (vec && wvec && C / 8 <= 32 * 8)
       gate_rmsnorm_reg_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
     else if (vec) gate_rmsnorm_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);
     else gate_rmsnorm_kernel<__nv_bfloat16, 1><<<blocks, 256, 0, st>>>(yy, ldy, zz, ldz, norm_w, C, nrows);

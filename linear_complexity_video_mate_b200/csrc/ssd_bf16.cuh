@@ -271,219 +271,339 @@ __global__ void __launch_bounds__(128, 1) ssd_gram_kernel(const SsdBf16Params p)
 }
 
 // ---------------------------------------------------------------------------------------------------
-// Chunk-local end states.  grid (nRc + nVc, B, nh / heads_per_cta), 256 threads (thread j = token j).
-// D[n][p] = sum_j B[j][n] * (w_j x[j][p]): A operand = the B tile read MN-major, B operand = the
-// weighted x tile (MN-major), M = N_state = 128, N = P = 64, K = Q = 256; both operands fp16 (the B
-// rows are converted once per chunk, the weighted x per head), states written in fp32.
+// Chunk-local end states, persistent and pipelined.  grid = min(B (nRc + nVc), SMs), kStThreads threads;
+// each CTA walks the chunks w = blockIdx.x, blockIdx.x + gridDim.x, ... (w = b (nRc + nVc) + c) and,
+// inside a chunk, every head.  The roles overlap one head's x loads, MMAs and state stores with the next
+// head's scan and weighting:
+//   warps 0..3   drain: a head's two states from TMEM (lane quadrant = warp, lane = state row n) through
+//                a 4 KB transpose buffer per warp (32 rows x 32 columns at a time) to the fp32 state arrays
+//                as whole 128-byte row segments, then release the accumulator set
+//   warps 4..11  prep (thread j = token j of the chunk): per chunk the B rows (bf16 -> fp16, into the
+//                tile read MN-major as the A operand); per head the decay scan, the output kernel's decay
+//                tables and the decay-weighted x tiles (fp16, MN-major) from the head's x tile
+//   warp 12      MMA issue (lane 0): D[n][p] = sum_j B[j][n] (w_j x[j][p]), M = N_state = 128, N = P = 64,
+//                K = Q = 256, for both directions into one of two TMEM accumulator sets [Sf | Sb]
+//   warp 13      x loader: each head's 256 x rows (64 columns, TMA four-row gathers through the scan-order
+//                row map) into a ring of two tiles, two heads ahead of the weighting
 // ---------------------------------------------------------------------------------------------------
+constexpr int kStPrepWarp0 = 4, kStMmaWarp = 12, kStLoadWarp = 13, kStThreads = 448;
+constexpr uint32_t kStOffX = 65536;                 // weighted x: fwd 32 KB | bwd 32 KB
+constexpr uint32_t kStOffXr = kStOffX + 65536;      // x tiles as loaded, two of 32 KB
+constexpr uint32_t kStOffW = kStOffXr + 65536;      // weights of the current head: fwd [256], bwd [256]
+constexpr uint32_t kStOffRow = kStOffW + 2048;      // source rows of the chunk [256]
+constexpr uint32_t kStOffMisc = kStOffRow + 2048;   // scan warp totals [8], row-block boundaries [8]
+constexpr uint32_t kStOffStage = kStOffMisc + 64;   // drain transpose buffers, 4 KB per drain warp
+constexpr uint32_t kStOffBar = kStOffStage + 4 * 4096;
+constexpr uint32_t kStSmem = kStOffBar + 128;
+static_assert(kStSmem + 1024 <= 232448, "shared memory of the state kernel");
+
+// Inclusive prefix sum of one value per prep thread (j = 0..255) on named barrier `id`.
+__device__ __forceinline__ float prep_scan_256(float v, float* warp_tot, int j, int id) {
+  const int lane = j & 31, w = j >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float u = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += u;
+  }
+  if (lane == 31) warp_tot[w] = v;
+  named_bar_sync(id, 256);
+  float base = 0.f;
+  for (int k = 0; k < w; ++k) base += warp_tot[k];
+  named_bar_sync(id, 256);
+  return v + base;
+}
+
+// x rows of the state kernel: review and video arrays (one-row boxes of 64 columns, for four-row gathers).
+struct SsdStateMaps {
+  CUtensorMap xv, xr;
+  int rows_v, rows_r;   // row extents; gathers of rows past a partial chunk's end use them (zeros)
+};
+
 template <bool XF16>
-__global__ void __launch_bounds__(256, 1) ssd_state_kernel(const SsdBf16Params p, int heads_per_cta) {
+__global__ void __launch_bounds__(kStThreads, 1) ssd_state_kernel(const SsdBf16Params p,
+                                                                  const __grid_constant__ SsdStateMaps mp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sB = smem;                 // [256 j][128 n]
-  uint8_t* sXf = smem + 65536;        // [256 j][64 p]
-  uint8_t* sXb = smem + 98304;
-  float* sWf = reinterpret_cast<float*>(smem + 131072);
-  float* sWb = sWf + 256;
-  float* wtot = sWb + 256;
-  long long* srow = reinterpret_cast<long long*>(wtot + 8);   // [256]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(srow + 256);
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
-  float* bnd = reinterpret_cast<float*>(bar + 2);   // s at the ends of row blocks 0..2, s' at starts of 1..3
-  const int c = blockIdx.x, b = blockIdx.y;
-  const ChunkBase cb = chunk_base(p.s, c, p.nRc);
-  const bool video = c >= p.nRc;
-  const int nC = p.nRc + p.nVc;
+  uint8_t* sB = smem;   // [256 j][128 n] fp16
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStOffBar);
+  uint64_t* x_full = bars;          // weighted x (and, for a chunk's first head, the B tile): 256 prep threads
+  uint64_t* x_empty = bars + 1;     // MMA commit
+  uint64_t* acc_full = bars + 2;    // [2] MMA commit -> drain
+  uint64_t* acc_empty = bars + 4;   // [2] 4 drain warps -> MMA
+  uint64_t* xr_full = bars + 6;     // [2] x tile bytes
+  uint64_t* xr_empty = bars + 8;    // [2] 256 prep threads have read the tile
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bars + 10);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = threadIdx.x;
+  const int nC = p.nRc + p.nVc, nwork = p.B * nC, nh = p.nh;
+  const bool per_dir = p.A_log_b != nullptr;   // backward scan with its own A, D and delta
 
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
+    mbar_init(x_full, 256);
+    mbar_init(x_empty, 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&acc_full[q], 1);
+      mbar_init(&acc_empty[q], 4);
+      mbar_init(&xr_full[q], 1);
+      mbar_init(&xr_empty[q], 256);
+    }
     mbar_fence_init();
   }
-  if (warp == 0) tmem_alloc(slot, 128);
-  fill_chunk_rows(p.s, b, c, p.nRc, srow);
+  if (warp == kStMmaWarp) tmem_alloc(slot, 256);
+  tc_fence_before();
   __syncthreads();
-  {
-    // the chunk's B rows, bf16 -> fp16, into the K-major swizzled tile (zeros past a partial chunk's end)
-    uint4 bv[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int it = threadIdx.x + u * 256;
-      const long long rw = srow[it >> 4];
-      bv[u] = rw >= 0 ? __ldg(reinterpret_cast<const uint4*>(cb.b + rw * cb.ldb) + (it & 15)) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int it = threadIdx.x + u * 256;
-      const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bv[u]);
-      uint4 o;
-      uint32_t* po = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = unpack_bf16x2(bw[e]);
-        po[e] = pack_f16x2_sat(f.x, f.y);
-      }
-      *reinterpret_cast<uint4*>(sB + sw128_kmajor_offset(it >> 4, (it & 15) * 8, 32768)) = o;
-    }
-  }
-  const long long myrw = srow[j];
   tc_fence_after();
   const uint32_t tmem = *slot;
-  uint32_t phase = 0;
 
-  // x rows of this thread's 8 items (row it>>3, 16-byte chunk it&7); the next head's rows are fetched
-  // while the current head's MMAs run
-  uint4 xr[8];
-  auto load_x = [&](int h) {
+  if (warp < kStPrepWarp0) {
+    // ------------------------------------------------------------------------------ drain
+    float4* stage = reinterpret_cast<float4*>(smem + kStOffStage + warp * 4096);
+    int u = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+      const int c = w % nC, b = w / nC;
+      const bool video = c >= p.nRc;
+      for (int h = 0; h < nh; ++h, ++u) {
+        const int acc = u & 1, use = u >> 1;
+        if (!mbar_wait(&acc_full[acc], use & 1)) { ok = false; break; }
+        tc_fence_after();
+        for (int dir = 0; dir < 2; ++dir) {
+          if (dir == 1 && !video && !per_dir) break;
+          float* dst = dir == 0
+              ? p.Sf + ((static_cast<long long>(b) * nC + c) * nh + h) * (kSsdP * kSsdN)
+              : (video ? p.Sb + ((static_cast<long long>(b) * p.nVc + (c - p.nRc)) * nh + h) * (kSsdP * kSsdN)
+                       : p.Srb + ((static_cast<long long>(b) * p.nRc + c) * nh + h) * (kSsdP * kSsdN));
+          // lane = state row n holds 32 p values per load; the warp's 32 rows x 32 columns go through its
+          // transpose buffer (16-byte chunk c of row r at chunk c ^ (r & 7): conflict-free both ways) so
+          // that each store instruction writes four whole 128-byte row segments of the [N][P] state
+          for (int pc = 0; pc < 2; ++pc) {
+            uint32_t r[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * 128 + dir * 64 + pc * 32, r);
+            tmem_wait_ld();
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int it = threadIdx.x + u * 256;
-      const long long rw = srow[it >> 3];
-      xr[u] = rw >= 0 ? __ldg(reinterpret_cast<const uint4*>(cb.x + rw * cb.ldx + h * kSsdP + (it & 7) * 8))
-                      : make_uint4(0, 0, 0, 0);
-    }
-  };
-  const bool per_dir = p.A_log_b != nullptr;   // backward scan with its own A, D and delta
-  load_x(blockIdx.z * heads_per_cta);
-  float dl_next = myrw >= 0 ? cb.d[myrw * cb.ldd + blockIdx.z * heads_per_cta] : 0.f;
-  float dlb_next = per_dir ? (myrw >= 0 ? cb.d[myrw * cb.ldd + p.s.db_off + blockIdx.z * heads_per_cta] : 0.f)
-                           : dl_next;
-
-  for (int hh = 0; hh < heads_per_cta; ++hh) {
-    const int h = blockIdx.z * heads_per_cta + hh;
-    const float A = -__expf(p.A_log[h]);
-    const float dl = dl_next, dlb = dlb_next;
-    const float a = dl * A;
-    const float s = block_scan_256(a, wtot);
-    if (j == 255) wtot[8 - 1] = s;  // reuse slot 7 for s_last after the scan finished with wtot
-    if ((j & 63) == 63 && j < 255) bnd[j >> 6] = s;          // bnd[ib - 1] = s_{64 ib - 1}, ib = 1..3
-    __syncthreads();
-    const float s_last = wtot[7];
-    // backward scan quantities: the same as the forward ones unless the backward parameters differ
-    float ab = a, sbk = s, sb_last = s_last;
-    if (per_dir) {
-      ab = dlb * -__expf(p.A_log_b[h]);
-      __syncthreads();   // every thread has read s_last before the second scan reuses wtot
-      sbk = block_scan_256(ab, wtot);
-      if (j == 255) wtot[8 - 1] = sbk;
-      __syncthreads();
-      sb_last = wtot[7];
-    }
-    const float sx = sbk - ab;   // exclusive backward cumulative sum s'
-    if ((j & 63) == 0 && j > 0) bnd[4 + (j >> 6) - 1] = sx;  // bnd[4 + ib] = s'_{64 ib + 64}, ib = 0..2
-    __syncthreads();
-    if (video) {
-      // decay tables of the output kernel (see kOutTbl); thread j is token j of the chunk
-      const long long cv = static_cast<long long>(b) * p.nVc + (c - p.nRc);
-      if (hh == 0 && blockIdx.z == 0) p.crow[cv * kSsdQ + j] = myrw >= 0 ? static_cast<int>(myrw) : -1;
-      float* T0 = p.tbl + (cv * p.nh + h) * 2 * kOutTbl;
-      float* T = T0 + (j >> 7) * kOutTbl;
-      const int r = j & 127, ib = j >> 6;
-      T[kTUf + r] = ib > 0 ? __expf(s - bnd[ib - 1]) : 0.f;
-      T[kTUb + r] = ib < 3 ? __expf(bnd[4 + ib] - sx) : 0.f;
-      T[kTSi + r] = s * kLog2e;
-      T[kTSx + r] = sx * kLog2e;
-      T[kTEf + r] = __expf(s);
-      T[kTEb + r] = __expf(sb_last - sx);
-      T[kTDl + r] = 0.5f * (dl + dlb);   // the output epilogue's diagonal term uses 2 (D + G_ii dl)
-      const float l2d = dl > 0.f ? __log2f(dl) : -INFINITY;
-      const float l2db = dlb > 0.f ? __log2f(dlb) : -INFINITY;
-      T[kTLf + r] = l2d - s * kLog2e;
-      T[kTLb + r] = l2db + sx * kLog2e;
+            for (int q = 0; q < 8; ++q)
+              stage[lane * 8 + (q ^ (lane & 7))] =
+                  make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                              __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+            __syncwarp();
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {   // column factors of row block q (stored with the tile holding it)
-        const float wfv = (q > 0 && j < 64 * q) ? dl * __expf(bnd[q - 1] - s) : 0.f;
-        const float wbv = (q < 3 && j >= 64 * q + 64) ? dlb * __expf(sx - bnd[4 + q]) : 0.f;
-        if (XF16) {
-          float* Tq = T0 + (q >> 1) * kOutTbl;
-          reinterpret_cast<__half*>(Tq + kTWf)[(q & 1) * 256 + j] = __float2half_rn(wfv);
-          reinterpret_cast<__half*>(Tq + kTWb)[(q & 1) * 256 + j] = __float2half_rn(wbv);
-        } else {
-          float* W = T0 + (q >> 1) * kOutTbl + (q & 1) * 256 + j;
-          W[kTWf] = wfv;
-          W[kTWb] = wbv;
+            for (int k = 0; k < 8; ++k) {
+              const int row = k * 4 + (lane >> 3), q = lane & 7;
+              reinterpret_cast<float4*>(dst + (warp * 32 + row) * kSsdP + pc * 32)[q] = stage[row * 8 + (q ^ (row & 7))];
+            }
+            __syncwarp();
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
+    }
+  } else if (warp < kStMmaWarp) {
+    // ------------------------------------------------------------------------------ prep
+    const int j = threadIdx.x - kStPrepWarp0 * 32;
+    float* sWf = reinterpret_cast<float*>(smem + kStOffW);
+    float* sWb = sWf + 256;
+    long long* srow = reinterpret_cast<long long*>(smem + kStOffRow);
+    float* wtot = reinterpret_cast<float*>(smem + kStOffMisc);
+    float* bnd = wtot + 8;   // s at the ends of row blocks 0..2, s' at the starts of 1..3
+    int u = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+      const int c = w % nC, b = w / nC;
+      const ChunkBase cb = chunk_base(p.s, c, p.nRc);
+      const bool video = c >= p.nRc;
+      named_bar_sync(1, 256);   // every prep thread is done with the previous chunk's rows
+      {
+        const RowRef rr = chunk_row(p.s, b, c, p.nRc, j);
+        srow[j] = rr.valid ? rr.r : -1;
+      }
+      named_bar_sync(1, 256);
+      const long long myrw = srow[j];
+      uint4 bv[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int it = j + e * 256;
+        const long long rw = srow[it >> 4];
+        bv[e] = rw >= 0 ? __ldg(reinterpret_cast<const uint4*>(cb.b + rw * cb.ldb) + (it & 15)) : make_uint4(0, 0, 0, 0);
+      }
+      // the previous chunk's MMAs (all committed before its last head's x_empty) must be done with the B tile
+      if (u > 0) ok = mbar_wait(x_empty, (u - 1) & 1);
+      if (named_bar_any(1, 256, !ok)) { ok = false; break; }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {   // bf16 -> fp16 (zeros past a partial chunk's end)
+        const int it = j + e * 256;
+        const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bv[e]);
+        uint4 o;
+        uint32_t* po = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = unpack_bf16x2(bw[k]);
+          po[k] = pack_f16x2_sat(f.x, f.y);
+        }
+        *reinterpret_cast<uint4*>(sB + sw128_kmajor_offset(it >> 4, (it & 15) * 8, 32768)) = o;
+      }
+      float dl_next = myrw >= 0 ? cb.d[myrw * cb.ldd] : 0.f;
+      float dlb_next = per_dir ? (myrw >= 0 ? cb.d[myrw * cb.ldd + p.s.db_off] : 0.f) : dl_next;
+      float alog_next = p.A_log[0];
+      for (int h = 0; h < nh; ++h, ++u) {
+        const float A = -__expf(alog_next);
+        const float dl = dl_next, dlb = dlb_next;
+        if (h + 1 < nh) {   // the next head's deltas and A: a whole head of work to arrive
+          dl_next = myrw >= 0 ? cb.d[myrw * cb.ldd + h + 1] : 0.f;
+          dlb_next = per_dir ? (myrw >= 0 ? cb.d[myrw * cb.ldd + p.s.db_off + h + 1] : 0.f) : dl_next;
+          alog_next = p.A_log[h + 1];
+        }
+        const float a = dl * A;
+        const float s = prep_scan_256(a, wtot, j, 1);
+        if (j == 255) wtot[8 - 1] = s;   // slot 7 holds s_last once the scan is done with the warp totals
+        if ((j & 63) == 63 && j < 255) bnd[j >> 6] = s;   // bnd[ib - 1] = s_{64 ib - 1}, ib = 1..3
+        named_bar_sync(1, 256);
+        const float s_last = wtot[7];
+        // backward scan quantities: the same as the forward ones unless the backward parameters differ
+        float ab = a, sbk = s, sb_last = s_last;
+        if (per_dir) {
+          ab = dlb * -__expf(p.A_log_b[h]);
+          named_bar_sync(1, 256);   // every thread has read s_last before the second scan reuses wtot
+          sbk = prep_scan_256(ab, wtot, j, 1);
+          if (j == 255) wtot[8 - 1] = sbk;
+          named_bar_sync(1, 256);
+          sb_last = wtot[7];
+        }
+        const float sx = sbk - ab;   // exclusive backward cumulative sum s'
+        if ((j & 63) == 0 && j > 0) bnd[4 + (j >> 6) - 1] = sx;   // bnd[4 + ib] = s'_{64 ib + 64}, ib = 0..2
+        named_bar_sync(1, 256);
+        if (video) {
+          // decay tables of the output kernel (see kOutTbl)
+          const long long cv = static_cast<long long>(b) * p.nVc + (c - p.nRc);
+          if (h == 0) p.crow[cv * kSsdQ + j] = myrw >= 0 ? static_cast<int>(myrw) : -1;
+          float* T0 = p.tbl + (cv * nh + h) * 2 * kOutTbl;
+          float* T = T0 + (j >> 7) * kOutTbl;
+          const int r = j & 127, ib = j >> 6;
+          T[kTUf + r] = ib > 0 ? __expf(s - bnd[ib - 1]) : 0.f;
+          T[kTUb + r] = ib < 3 ? __expf(bnd[4 + ib] - sx) : 0.f;
+          T[kTSi + r] = s * kLog2e;
+          T[kTSx + r] = sx * kLog2e;
+          T[kTEf + r] = __expf(s);
+          T[kTEb + r] = __expf(sb_last - sx);
+          T[kTDl + r] = 0.5f * (dl + dlb);   // the output epilogue's diagonal term uses 2 (D + G_ii dl)
+          const float l2d = dl > 0.f ? __log2f(dl) : -INFINITY;
+          const float l2db = dlb > 0.f ? __log2f(dlb) : -INFINITY;
+          T[kTLf + r] = l2d - s * kLog2e;
+          T[kTLb + r] = l2db + sx * kLog2e;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {   // column factors of row block q (stored with the tile holding it)
+            const float wfv = (q > 0 && j < 64 * q) ? dl * __expf(bnd[q - 1] - s) : 0.f;
+            const float wbv = (q < 3 && j >= 64 * q + 64) ? dlb * __expf(sx - bnd[4 + q]) : 0.f;
+            if (XF16) {
+              float* Tq = T0 + (q >> 1) * kOutTbl;
+              reinterpret_cast<__half*>(Tq + kTWf)[(q & 1) * 256 + j] = __float2half_rn(wfv);
+              reinterpret_cast<__half*>(Tq + kTWb)[(q & 1) * 256 + j] = __float2half_rn(wbv);
+            } else {
+              float* W = T0 + (q >> 1) * kOutTbl + (q & 1) * 256 + j;
+              W[kTWf] = wfv;
+              W[kTWb] = wbv;
+            }
+          }
+        }
+        if (j == 0) {
+          p.gl[(static_cast<long long>(b) * nC + c) * nh + h] = s_last;
+          if (per_dir) p.glb[(static_cast<long long>(b) * nC + c) * nh + h] = sb_last;
+        }
+        sWf[j] = __expf(s_last - s) * dl;
+        // second product: the backward state of a video chunk (decay to its start); for a review chunk
+        // under separate backward parameters, its state at the chunk end under those parameters
+        sWb[j] = (video || !per_dir) ? __expf(sx) * dlb : __expf(sb_last - sbk) * dlb;
+        const int xb = u & 1;
+        // the previous head's MMAs are done with the weighted tiles, and this head's x tile has landed
+        ok = mbar_wait(x_empty, (u & 1) ^ 1) && mbar_wait(&xr_full[xb], (u >> 1) & 1);
+        if (named_bar_any(1, 256, !ok)) { ok = false; break; }
+        uint8_t* sXf = smem + kStOffX;
+        uint8_t* sXb = sXf + 32768;
+        const uint8_t* sXr = smem + kStOffXr + xb * 32768;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {   // weighted x tiles, 8 values (one 16-byte chunk) per item
+          const int it = j + e * 256;
+          const int r = it >> 3, ch = it & 7;
+          const float wf = sWf[r], wb = sWb[r];
+          const uint32_t off = sw128_mnmajor_offset(r, ch * 8, 32768);
+          const uint4 xv = *reinterpret_cast<const uint4*>(sXr + off);
+          const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xv);
+          uint4 of, ob;
+          uint32_t* pf = reinterpret_cast<uint32_t*>(&of);
+          uint32_t* pb = reinterpret_cast<uint32_t*>(&ob);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = XF16 ? unpack_f16x2(xw[k]) : unpack_bf16x2(xw[k]);
+            pf[k] = pack_f16x2_sat(f.x * wf, f.y * wf);
+            pb[k] = pack_f16x2_sat(f.x * wb, f.y * wb);
+          }
+          *reinterpret_cast<uint4*>(sXf + off) = of;
+          *reinterpret_cast<uint4*>(sXb + off) = ob;
+        }
+        fence_proxy_async();
+        mbar_arrive(x_full);
+        mbar_arrive(&xr_empty[xb]);
+      }
+    }
+  } else if (warp == kStMmaWarp) {
+    // ------------------------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      // both directions as one N = 128 product: B = [Xf | Xb], two MN blocks 32 KB apart -> [Sf | Sb];
+      // N = 64 (Xf only) for a review chunk without a backward state
+      const uint32_t idesc2 = idesc_f16_f32(128, 128, 1, 1), idesc1 = idesc_f16_f32(128, 64, 1, 1);
+      const uint32_t ab = smem_u32(sB);
+      int u = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+        const bool two = (w % nC) >= p.nRc || per_dir;   // a backward state for this chunk
+        for (int h = 0; h < nh; ++h, ++u) {
+          const int buf = u & 1, use = u >> 1;
+          if (!mbar_wait(x_full, u & 1) || !mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t xf = smem_u32(smem + kStOffX);
+          const uint32_t d = tmem + buf * 128;
+#pragma unroll 4
+          for (int k = 0; k < 16; ++k)
+            mma_bf16_ss(d, desc_sw128(ab + k * 2048, 32768, 1024), desc_sw128(xf + k * 2048, 32768, 1024),
+                        two ? idesc2 : idesc1, k > 0);
+          mma_commit(x_empty);
+          mma_commit(&acc_full[buf]);
         }
       }
     }
-    if (threadIdx.x == 0 && per_dir) p.glb[(static_cast<long long>(b) * nC + c) * p.nh + h] = sb_last;
-    sWf[j] = __expf(s_last - s) * dl;
-    // second product: the backward state of a video chunk (decay to its start); for a review chunk under
-    // separate backward parameters, its state at the chunk end under those parameters
-    sWb[j] = (video || !per_dir) ? __expf(sx) * dlb : __expf(sb_last - sbk) * dlb;
-    __syncthreads();
-    // weighted x tiles, 8 bf16 (one 16-byte chunk) per item; 8 items per row
+    __syncwarp();
+  } else if (warp == kStLoadWarp) {
+    // ------------------------------------------------------------------------------ x loader
+    // every exit decision is warp-uniform (a lane leaving alone would strand __syncwarp)
+    auto wait_all = [&](uint64_t* bar, unsigned parity) { return !__any_sync(0xffffffffu, !mbar_wait(bar, parity)); };
+    int u = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+      const int c = w % nC, b = w / nC;
+      const bool video = c >= p.nRc;
+      const CUtensorMap* map = video ? &mp.xv : &mp.xr;
+      int id[8];   // chunk rows 8 lane .. 8 lane + 7 (rows past a partial chunk's end: the map's extent)
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int it = threadIdx.x + u * 256;
-      const int r = it >> 3, ch = it & 7;
-      const float wf = sWf[r], wb = sWb[r];
-      const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xr[u]);
-      uint4 of, ob;
-      uint32_t* pf = reinterpret_cast<uint32_t*>(&of);
-      uint32_t* pb = reinterpret_cast<uint32_t*>(&ob);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = XF16 ? unpack_f16x2(xw[e]) : unpack_bf16x2(xw[e]);
-        pf[e] = pack_f16x2_sat(f.x * wf, f.y * wf);
-        pb[e] = pack_f16x2_sat(f.x * wb, f.y * wb);
+      for (int e = 0; e < 8; ++e) {
+        const RowRef rr = chunk_row(p.s, b, c, p.nRc, 8 * lane + e);
+        id[e] = rr.valid ? static_cast<int>(rr.r) : (video ? mp.rows_v : mp.rows_r);
       }
-      const uint32_t off = sw128_mnmajor_offset(r, ch * 8, 32768);
-      *reinterpret_cast<uint4*>(sXf + off) = of;
-      *reinterpret_cast<uint4*>(sXb + off) = ob;
-    }
-    fence_proxy_async();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_f16_f32(128, 64, 1, 1);
-      const uint32_t ab = smem_u32(sB), xf = smem_u32(sXf), xb = smem_u32(sXb);
-#pragma unroll 4
-      for (int k = 0; k < 16; ++k) {
-        const uint64_t ad = desc_sw128(ab + k * 2048, 32768, 1024);
-        mma_bf16_ss(tmem, ad, desc_sw128(xf + k * 2048, 32768, 1024), idesc, k > 0);
-        if (video || per_dir) mma_bf16_ss(tmem + 64, ad, desc_sw128(xb + k * 2048, 32768, 1024), idesc, k > 0);
-      }
-      mma_commit(bar);
-    }
-    if (hh + 1 < heads_per_cta) {
-      load_x(h + 1);
-      dl_next = myrw >= 0 ? cb.d[myrw * cb.ldd + h + 1] : 0.f;
-      dlb_next = per_dir ? (myrw >= 0 ? cb.d[myrw * cb.ldd + p.s.db_off + h + 1] : 0.f) : dl_next;
-    }
-    const bool ok = mbar_wait(bar, phase);
-    phase ^= 1;
-    // a wait that ran out (flagged in the status word) ends the walk for the whole CTA: no read-out, no
-    // further heads; the CTA still frees its TMEM
-    if (__syncthreads_or(!ok)) break;
-    tc_fence_after();
-    const int dir = warp >> 2, quad = warp & 3;
-    const int nidx = quad * 32 + lane;
-    if (dir == 0 || video || per_dir) {
-      float* dst = dir == 0
-          ? p.Sf + ((static_cast<long long>(b) * nC + c) * p.nh + h) * (kSsdP * kSsdN)
-          : (video ? p.Sb + ((static_cast<long long>(b) * p.nVc + (c - p.nRc)) * p.nh + h) * (kSsdP * kSsdN)
-                   : p.Srb + ((static_cast<long long>(b) * p.nRc + c) * p.nh + h) * (kSsdP * kSsdN));
-      // lane = state row n: its 64 p values are one contiguous 256-byte row of the [N][P] fp32 state
-      for (int pc = 0; pc < 2; ++pc) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + dir * 64 + pc * 32, r);
-        tmem_wait_ld();
-        float4* d4 = reinterpret_cast<float4*>(dst + nidx * kSsdP + pc * 32);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          d4[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
-                              __uint_as_float(r[4 * q + 3]));
+      for (int h = 0; h < nh; ++h, ++u) {
+        const int xb = u & 1, use = u >> 1;
+        if (!wait_all(&xr_empty[xb], (use & 1) ^ 1)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(&xr_full[xb], 32768);
+        __syncwarp();
+        uint8_t* dst = smem + kStOffXr + xb * 32768;
+        tma_gather4(map, &xr_full[xb], dst + (2 * lane) * 512, h * kSsdP, id[0], id[1], id[2], id[3]);
+        tma_gather4(map, &xr_full[xb], dst + (2 * lane + 1) * 512, h * kSsdP, id[4], id[5], id[6], id[7]);
       }
     }
-    if (threadIdx.x == 0) p.gl[(static_cast<long long>(b) * nC + c) * p.nh + h] = s_last;
-    tc_fence_before();
-    __syncthreads();
   }
+  tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kStMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -571,15 +691,16 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 //   warp 0       per item: the head's decay tables (one bulk copy) and x rows (all 256 of the chunk,
 //                MN-major, TMA four-row gathers) into one of two x buffers.
 //   warp 1       per group: the tile's C rows (K-major, four-row gathers); per item: the head's incoming
-//                states [Hf | Hb] (MN-major, 2D TMA), first their hi parts, then, once the hi product is
-//                done, their lo parts into the same buffer.
+//                states as four [N = 128][P = 64] blocks, Hf hi, Hb hi, Hf lo, Hb lo (MN-major, 2D TMA),
+//                through a ring of three 16 KB slots, so that up to three are in flight.
 //   warp 2       per group: the tile's rows of G (2D TMA) into four 64-column slots, each refilled once
 //                the last head of the previous group has read it.
 //   warp 3       MMA issue (lane 0 only; an issuing thread stalls while the tensor pipe is busy, so it has
-//                no other work): Yd = M x per K half of M (A from TMEM) and, after each half,
-//                [Yf | Yb] (+)= C [Hf | Hb]^T as one N = 128 product (hi parts, then lo parts), into one of
+//                no other work): Yd = M x per K half of M (A from TMEM) and, after each half, two of the
+//                four N = 64 products Yf (+)= C Hf^T, Yb (+)= C Hb^T (hi parts, then lo parts), into one of
 //                two TMEM accumulator sets.
-//   warps 4..11  transform (two warps per TMEM lane quadrant, alternating 8-column chunks): form
+//   warps 4..11  transform (two warps per TMEM lane quadrant, each taking 16 contiguous TMEM columns of
+//                every 64-element column block, stored with one TMEM store): form
 //                M_ij = G_ij delta_j dec(i, j) (diagonal excluded) from the G slots and store M straight
 //                into TMEM as the A operand of the MMA (two bf16 per 32-bit column), in two K halves.
 //   warps 12..15 epilogue: y_i = Yd + exp(s_i) Yf + exp(s_last - s'_i) Yb + 2 (D + G_ii delta_i) x_i,
@@ -601,15 +722,16 @@ static_assert(kOutFirstXformWarp % 4 == 0 && kOutFirstEpiWarp % 4 == 0, "TMEM la
 
 // shared memory map (offsets from the 1024-aligned base)
 constexpr uint32_t kOutTblBytes = kOutTbl * 4;         // 8704
-constexpr uint32_t kOutXBuf = 41984;                    // x tile (32 KB) + the head's tables, two of them
-constexpr uint32_t kOutOffTbl = 32768;
-constexpr uint32_t kOutOffC = 2 * kOutXBuf;             // C rows of the tile: 2 K blocks of 16 KB
-constexpr uint32_t kOutOffH = kOutOffC + 32768;         // [Hf | Hb] hi or lo: 2 MN blocks of [N = 128][P = 64]
-constexpr uint32_t kOutOffG = kOutOffH + 32768;         // 4 slots of [128 rows][64 cols] K-major
+constexpr uint32_t kOutXBuf = 32768;                    // x tile of one item, two of them
+constexpr uint32_t kOutOffTbl = 2 * kOutXBuf;           // the item's decay tables, two of them
+constexpr uint32_t kOutOffC = kOutOffTbl + 2 * kOutTblBytes;   // C rows of the tile: 2 K blocks of 16 KB
+constexpr uint32_t kOutHSlots = 3;                      // ring of [N = 128][P = 64] state blocks
+constexpr uint32_t kOutOffH = kOutOffC + 32768;
+constexpr uint32_t kOutOffG = kOutOffH + kOutHSlots * 16384;   // 4 slots of [128 rows][64 cols] K-major
 constexpr uint32_t kOutOffBar = kOutOffG + 4 * 16384;
 constexpr uint32_t kOutSmem = kOutOffBar + 256;
-static_assert(kOutOffTbl + kOutTblBytes <= kOutXBuf, "tables overflow the x buffer");
-static_assert(kOutXBuf % 1024 == 0 && kOutOffC % 1024 == 0 && kOutOffG % 1024 == 0, "1024-byte operand tiles");
+static_assert(kOutOffC % 1024 == 0 && kOutOffH % 1024 == 0 && kOutOffG % 1024 == 0, "1024-byte operand tiles");
+static_assert(kOutSmem + 1024 <= 232448, "shared memory of the output kernel");
 
 // Tensor maps of the output kernel: x and C rows of the video arrays (one-row boxes of 64 columns, for
 // four-row gathers), the carried states ([2][N rows][P] hi | lo per chunk and head, 64 x 128 boxes) and G
@@ -626,18 +748,19 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOutOffBar);
   uint64_t* x_full = bars;         // [2] x + table bytes
-  uint64_t* x_empty = bars + 2;    // [2] last Yd MMA commit + 4 epilogue warps
-  uint64_t* h_full = bars + 4;     // Hf + Hb bytes (hi parts, then lo parts: two phases per item)
-  uint64_t* h_empty = bars + 5;    // Yf / Yb MMA commit (one per part)
-  uint64_t* c_full = bars + 6;     // C bytes (per group)
-  uint64_t* c_empty = bars + 7;    // last head's Yf / Yb MMA commit
-  uint64_t* g_full = bars + 8;     // [4] one G slot's bytes (per group)
-  uint64_t* g_empty = bars + 12;   // [4] the 8 transform warps have read the slot for the last head
-  uint64_t* m_full = bars + 16;    // [2] per K half of M: transform -> MMA (count 256)
-  uint64_t* m_empty = bars + 18;   // [2] per K half of M: MMA commit -> transform
-  uint64_t* y_full = bars + 20;    // [2] MMA commit -> epilogue
-  uint64_t* y_empty = bars + 22;   // [2] epilogue warps -> MMA (count 4)
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bars + 24);
+  uint64_t* x_empty = bars + 2;    // [2] last Yd MMA commit (the epilogue reads its x rows and table
+                                   //     entries from global memory, so the buffer never waits for it)
+  uint64_t* h_full = bars + 4;     // [3] one state block's bytes
+  uint64_t* h_empty = bars + 7;    // [3] the Yf / Yb MMA commit that read the slot
+  uint64_t* c_full = bars + 10;    // C bytes (per group)
+  uint64_t* c_empty = bars + 11;   // last head's Yf / Yb MMA commit
+  uint64_t* g_full = bars + 12;    // [4] one G slot's bytes (per group)
+  uint64_t* g_empty = bars + 16;   // [4] the 8 transform warps have read the slot for the last head
+  uint64_t* m_full = bars + 20;    // [2] per K half of M: transform -> MMA (count 256)
+  uint64_t* m_empty = bars + 22;   // [2] per K half of M: MMA commit -> transform
+  uint64_t* y_full = bars + 24;    // [2] MMA commit -> epilogue
+  uint64_t* y_empty = bars + 26;   // [2] epilogue warps -> MMA (count 4)
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bars + 28);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nh = p.nh;
@@ -646,14 +769,16 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
   if (threadIdx.x == 0) {
     for (int q = 0; q < 2; ++q) {
       mbar_init(&x_full[q], 1);
-      mbar_init(&x_empty[q], 5);
+      mbar_init(&x_empty[q], 1);
       mbar_init(&m_full[q], kOutXformWarps * 32);
       mbar_init(&m_empty[q], 1);
       mbar_init(&y_full[q], 1);
       mbar_init(&y_empty[q], kOutEpiWarps);
     }
-    mbar_init(h_full, 1);
-    mbar_init(h_empty, 1);
+    for (int q = 0; q < 3; ++q) {
+      mbar_init(&h_full[q], 1);
+      mbar_init(&h_empty[q], 1);
+    }
     mbar_init(c_full, 1);
     mbar_init(c_empty, 1);
     for (int q = 0; q < 4; ++q) {
@@ -705,7 +830,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
         uint8_t* XB = smem + buf * kOutXBuf;
         if (lane == 0) {
           mbar_arrive_expect_tx(&x_full[buf], 32768 + kOutTblBytes);
-          bulk_load(XB + kOutOffTbl, p.tbl + ((cidx * nh + h) * 2 + t) * kOutTbl, kOutTblBytes, &x_full[buf]);
+          bulk_load(smem + kOutOffTbl + buf * kOutTblBytes, p.tbl + ((cidx * nh + h) * 2 + t) * kOutTbl, kOutTblBytes,
+                    &x_full[buf]);
         }
         __syncwarp();
 #pragma unroll
@@ -737,13 +863,13 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
       for (int kb = 0; kb < 2; ++kb)
         tma_gather4(&mp.c, c_full, smem + kOutOffC + kb * 16384 + lane * 512, kb * 64, id[0], id[1], id[2], id[3]);
       for (int h = 0; h < nh && ok; ++h, ++k) {
-        for (int part = 0; part < 2; ++part) {   // hi parts, then lo parts, through the one H buffer
-          if (!wait_all(h_empty, part ^ 1)) { ok = false; break; }
+        for (int q = 0; q < 4; ++q) {   // Hf hi, Hb hi, Hf lo, Hb lo through the ring of three slots
+          const int u = 4 * k + q, sl = u % 3, use = u / 3;
+          if (!wait_all(&h_empty[sl], (use & 1) ^ 1)) { ok = false; break; }
           if (lane == 0) {
-            mbar_arrive_expect_tx(h_full, 32768);
-            const int hrow = static_cast<int>(((cidx * nh + h) * 2 + part) * kSsdN);
-            tma_load_2d(&mp.hf, h_full, smem + kOutOffH, 0, hrow);
-            tma_load_2d(&mp.hb, h_full, smem + kOutOffH + 16384, 0, hrow);
+            mbar_arrive_expect_tx(&h_full[sl], 16384);
+            const int hrow = static_cast<int>(((cidx * nh + h) * 2 + (q >> 1)) * kSsdN);
+            tma_load_2d((q & 1) ? &mp.hb : &mp.hf, &h_full[sl], smem + kOutOffH + sl * 16384, 0, hrow);
           }
           __syncwarp();
         }
@@ -773,7 +899,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
     if (lane == 0) {
       // Yd: N = P, fp16 operands when x is fp16
       const uint32_t idesc_d = XF16 ? idesc_f16_f32(128, 64, 0, 1) : idesc_bf16_f32(128, 64, 0, 1);
-      const uint32_t idesc_h = idesc_bf16_f32(128, 128, 0, 1);   // [Yf | Yb]: N = 2 P, B = [Hf | Hb]
+      const uint32_t idesc_h = idesc_bf16_f32(128, 64, 0, 1);    // Yf or Yb: N = P, B = one state block
       const uint32_t cbase = smem_u32(smem + kOutOffC), hbase = smem_u32(smem + kOutOffH);
       int k = 0, kg = 0;
       bool ok = true;
@@ -782,6 +908,19 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           const int buf = k & 1, use = k >> 1, acc = k & 1;
           const uint32_t xb = smem_u32(smem + buf * kOutXBuf);
           const uint32_t ybase = tmem + 128 + acc * 192;
+          // Yf (+)= C Hf^T or Yb (+)= C Hb^T from the ring slot of part q (0: Hf hi, 1: Hb hi, 2: Hf lo, 3: Hb lo)
+          auto state_product = [&](int q) -> bool {
+            const int u = 4 * k + q, sl = u % 3, hu = u / 3;
+            if (!mbar_wait(&h_full[sl], hu & 1)) return false;
+            tc_fence_after();
+            const uint32_t hs = hbase + sl * 16384;
+#pragma unroll
+            for (int kq = 0; kq < 8; ++kq)   // K = N_state = 128
+              mma_bf16_ss(ybase + 64 + (q & 1) * 64, desc_sw128(cbase + (kq >> 2) * 16384 + (kq & 3) * 32, 16, 1024),
+                          desc_sw128(hs + kq * 2048, 16384, 1024), idesc_h, (q >> 1) != 0 || kq > 0);
+            mma_commit(&h_empty[sl]);
+            return true;
+          };
           ok = mbar_wait(&y_empty[acc], (use & 1) ^ 1) && mbar_wait(&m_full[0], k & 1);
           if (!ok) break;
           tc_fence_after();
@@ -789,14 +928,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           for (int q = 0; q < 8; ++q)   // Yd = M x, first K half (M in TMEM, 8 columns per 16 elements)
             mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, q > 0);
           mma_commit(&m_empty[0]);
-          ok = mbar_wait(h_full, 0) && (h > 0 || mbar_wait(c_full, kg & 1));
+          ok = (h > 0 || mbar_wait(c_full, kg & 1)) && state_product(0) && state_product(1);
           if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int q = 0; q < 8; ++q)   // [Yf | Yb] = C [Hf | Hb]_hi^T, K = N_state = 128
-            mma_bf16_ss(ybase + 64, desc_sw128(cbase + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
-                        desc_sw128(hbase + q * 2048, 16384, 1024), idesc_h, q > 0);
-          mma_commit(h_empty);
           ok = mbar_wait(&m_full[1], k & 1);
           if (!ok) break;
           tc_fence_after();
@@ -805,14 +938,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
             mma_bf16_ts(ybase, tmem + q * 8, desc_sw128(xb + q * 2048, 32768, 1024), idesc_d, true);
           mma_commit(&m_empty[1]);
           mma_commit(&x_empty[buf]);
-          ok = mbar_wait(h_full, 1);
+          ok = state_product(2) && state_product(3);
           if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int q = 0; q < 8; ++q)   // [Yf | Yb] += C [Hf | Hb]_lo^T
-            mma_bf16_ss(ybase + 64, desc_sw128(cbase + (q >> 2) * 16384 + (q & 3) * 32, 16, 1024),
-                        desc_sw128(hbase + q * 2048, 16384, 1024), idesc_h, true);
-          mma_commit(h_empty);
           if (h == nh - 1) mma_commit(c_empty);
           mma_commit(&y_full[acc]);
         }
@@ -824,7 +951,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
     const int xw = warp - kOutFirstXformWarp;
     const int quad = warp & 3, half = xw >> 2;
     const int r = quad * 32 + lane;
-    const uint32_t tm_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 4;
+    const uint32_t tm_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 16;
     int k = 0, kg = 0;
     bool ok = true;
     for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x, ++kg) {
@@ -833,7 +960,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
       for (int h = 0; h < nh && ok; ++h, ++k) {
         const int buf = k & 1, use = k >> 1;
         if (!wait_all(&x_full[buf], use & 1)) { ok = false; break; }
-        const float* tb = reinterpret_cast<const float*>(smem + buf * kOutXBuf + kOutOffTbl);
+        const float* tb = reinterpret_cast<const float*>(smem + kOutOffTbl + buf * kOutTblBytes);
         const float ufi = tb[kTUf + r], ubi = tb[kTUb + r];
         const float si2 = tb[kTSi + r], sxi2 = tb[kTSx + r];
         const float* wfr = tb + kTWf + (ib - 2 * t) * 256;
@@ -847,37 +974,44 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           }
           if (h == 0 && !wait_all(&g_full[cb], kg & 1)) { ok = false; break; }
           const uint8_t* grow = smem + kOutOffG + cb * 16384 + r * 128;
+          // this warp's 4 consecutive 16-byte chunks of the row (32 elements, 16 contiguous TMEM columns),
+          // stored with one 16-column TMEM store
           const uint32_t tcol = tm_row + cb * 32;
+          uint32_t pk[16];
           if (cb != ib && XF16) {
             // M = (G w) u in packed fp16: two multiplies per element pair
             const uint32_t uu = pack_f16x2_sat(cb < ib ? ufi : ubi, cb < ib ? ufi : ubi);
             const __half* wh = reinterpret_cast<const __half*>(tb + (cb < ib ? kTWf : kTWb)) + (ib - 2 * t) * 256 +
-                               cb * 64 + half * 8;
+                               cb * 64 + half * 32;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const int ch = 2 * qq + half;
+            for (int c = 0; c < 4; ++c) {
+              const int ch = 4 * half + c;
               const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
-              const uint4 wv = *reinterpret_cast<const uint4*>(wh + qq * 16);
-              tmem_st4(tcol + qq * 8, mul_f16x2(mul_f16x2(gc.x, wv.x), uu), mul_f16x2(mul_f16x2(gc.y, wv.y), uu),
-                       mul_f16x2(mul_f16x2(gc.z, wv.z), uu), mul_f16x2(mul_f16x2(gc.w, wv.w), uu));
+              const uint4 wv = *reinterpret_cast<const uint4*>(wh + c * 8);
+              pk[4 * c + 0] = mul_f16x2(mul_f16x2(gc.x, wv.x), uu);
+              pk[4 * c + 1] = mul_f16x2(mul_f16x2(gc.y, wv.y), uu);
+              pk[4 * c + 2] = mul_f16x2(mul_f16x2(gc.z, wv.z), uu);
+              pk[4 * c + 3] = mul_f16x2(mul_f16x2(gc.w, wv.w), uu);
             }
           } else if (cb != ib) {
             const float u = cb < ib ? ufi : ubi;
             const float2 uu = make_float2(u, u);
-            const float* w = (cb < ib ? wfr : wbr) + cb * 64 + half * 8;
+            const float* w = (cb < ib ? wfr : wbr) + cb * 64 + half * 32;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const int ch = 2 * qq + half;
+            for (int c = 0; c < 4; ++c) {
+              const int ch = 4 * half + c;
               const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
-              const float4 wa = *reinterpret_cast<const float4*>(w + qq * 16);
-              const float4 wc = *reinterpret_cast<const float4*>(w + qq * 16 + 4);
+              const float4 wa = *reinterpret_cast<const float4*>(w + c * 8);
+              const float4 wc = *reinterpret_cast<const float4*>(w + c * 8 + 4);
               // the same products as g * (u * w) elementwise, two per instruction
               const float2 m0 = mul_f32x2(unpack_f16x2(gc.x), mul_f32x2(uu, make_float2(wa.x, wa.y)));
               const float2 m1 = mul_f32x2(unpack_f16x2(gc.y), mul_f32x2(uu, make_float2(wa.z, wa.w)));
               const float2 m2 = mul_f32x2(unpack_f16x2(gc.z), mul_f32x2(uu, make_float2(wc.x, wc.y)));
               const float2 m3 = mul_f32x2(unpack_f16x2(gc.w), mul_f32x2(uu, make_float2(wc.z, wc.w)));
-              tmem_st4(tcol + qq * 8, pack_bf16x2(m0.x, m0.y), pack_bf16x2(m1.x, m1.y), pack_bf16x2(m2.x, m2.y),
-                       pack_bf16x2(m3.x, m3.y));
+              pk[4 * c + 0] = pack_bf16x2(m0.x, m0.y);
+              pk[4 * c + 1] = pack_bf16x2(m1.x, m1.y);
+              pk[4 * c + 2] = pack_bf16x2(m2.x, m2.y);
+              pk[4 * c + 3] = pack_bf16x2(m3.x, m3.y);
             }
           } else {
             // one exponential per element in the log2 domain; the diagonal itself is added in fp32 in
@@ -885,8 +1019,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
             const float* lfr = tb + kTLf - 128 * t;
             const float* lbr = tb + kTLb - 128 * t;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const int ch = 2 * qq + half;
+            for (int c = 0; c < 4; ++c) {
+              const int ch = 4 * half + c;
               const int j0 = cb * 64 + ch * 8;
               const uint4 gc = *reinterpret_cast<const uint4*>(grow + ((ch ^ (r & 7)) << 4));
               const float4 f0 = *reinterpret_cast<const float4*>(lfr + j0);
@@ -903,19 +1037,18 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
                 const float wv = ex2_approx(jj < i ? si2 + lf8[e] : lb8[e] - sxi2);
                 m[e] = jj == i ? 0.f : wv;
               }
-              uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 if (XF16) {
-                  pk[e] = mul_f16x2(gu[e], pack_f16x2_sat(m[2 * e], m[2 * e + 1]));
+                  pk[4 * c + e] = mul_f16x2(gu[e], pack_f16x2_sat(m[2 * e], m[2 * e + 1]));
                 } else {
                   const float2 gm = mul_f32x2(unpack_f16x2(gu[e]), make_float2(m[2 * e], m[2 * e + 1]));
-                  pk[e] = pack_bf16x2(gm.x, gm.y);
+                  pk[4 * c + e] = pack_bf16x2(gm.x, gm.y);
                 }
               }
-              tmem_st4(tcol + qq * 8, pk[0], pk[1], pk[2], pk[3]);
             }
           }
+          tmem_st16(tcol, pk);
           if (h == nh - 1) {   // the group's last head has read this G slot
             __syncwarp();
             if (lane == 0) mbar_arrive(&g_empty[cb]);
@@ -940,26 +1073,34 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
       const int i = t * 128 + r;
       const int len = min(kSsdQ, p.s.n - v * kSsdQ);
       const bool valid = i < len;
-      const float gdi = p.Gd[(static_cast<long long>(b) * p.nVc + v) * kSsdQ + i];
+      const long long cidx = static_cast<long long>(b) * p.nVc + v;
+      const float gdi = p.Gd[cidx * kSsdQ + i];
       const long long yrow = b * p.y_bstride + p.s.map(v * kSsdQ + (valid ? i : 0));
+      // this token's x row (source row from the chunk's row table) and its decay-table entries are read
+      // from global memory (L2), issued before the accumulators are ready, so that the x / table buffer
+      // is released by the MMAs alone
+      const int xsrc = valid ? p.crow[cidx * kSsdQ + i] : 0;
+      const uint8_t* xrow = static_cast<const uint8_t*>(p.s.xv) + static_cast<long long>(xsrc) * p.s.ldxv * 2;
       for (int h = 0; h < nh; ++h, ++k) {
-        const int buf = k & 1, acc = k & 1, use = k >> 1;
+        const int acc = k & 1, use = k >> 1;
         const float Dh = p.Dp_b != nullptr ? 0.5f * (p.Dp[h] + p.Dp_b[h]) : p.Dp[h];
+        const float* tg = p.tbl + ((cidx * nh + h) * 2 + t) * kOutTbl;
+        const float ef = tg[kTEf + r], eb = tg[kTEb + r], dli = tg[kTDl + r];
+        // x row of this token (packed bf16 or fp16 pairs) for the skip and diagonal terms
+        uint32_t xw[32];
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xrow + h * kSsdP * 2) + q);
+            xw[q * 4 + 0] = xv.x; xw[q * 4 + 1] = xv.y; xw[q * 4 + 2] = xv.z; xw[q * 4 + 3] = xv.w;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) xw[q] = 0u;
+        }
         if (!wait_all(&y_full[acc], use & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint8_t* XB = smem + buf * kOutXBuf;
-        const float* tb = reinterpret_cast<const float*>(XB + kOutOffTbl);
-        const float ef = tb[kTEf + r], eb = tb[kTEb + r], dli = tb[kTDl + r];
         const float D2 = 2.f * (Dh + (valid ? gdi * dli : 0.f));
-        // x row of this token (packed bf16 pairs) for the skip and diagonal terms
-        uint32_t xw[32];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(XB + sw128_mnmajor_offset(i, q * 8, 32768));
-          xw[q * 4 + 0] = xv.x; xw[q * 4 + 1] = xv.y; xw[q * 4 + 2] = xv.z; xw[q * 4 + 3] = xv.w;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&x_empty[buf]);
         __nv_bfloat16* ydst = p.y + yrow * p.ldy + h * kSsdP;
         const uint32_t ybase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128 + acc * 192;
 #pragma unroll
