@@ -30,7 +30,9 @@ Readings taken where the pages are silent (each is also listed in the design not
 
 Pins: every function here is checked by tests/test_oracle_pins.py against closed forms, brute force,
 textbook reshapes and hand-derived fixtures (tests/golden/).  The composed block (mate_forward) is pinned
-only through its pinned parts: parity unpinned beyond that composition (the pages print no worked example).
+as a whole by a per-token closed form (every step forgetting its state, one-token attention windows: the
+block reduces to [2 (delta (B . C) + D) x] W_out^T + v W_o^T on every scan order, review prefix included)
+and by the sum-of-branches identity; the pages print no worked example of the block.
 """
 from __future__ import annotations
 

@@ -326,6 +326,35 @@ def test_block_is_sum_of_branches():
                                    + O.mate_forward(w["X"], w_te, cfg, layer), rtol=1e-12, atol=1e-12)
 
 
+def test_block_fast_decay_one_token_windows_closed_form():
+    """The whole block, review prefix and all four scan orders included, in the special case where every
+    step forgets its state (delta A <= -60, so exp(delta A) < 1e-26) and every attention window holds one
+    token.  Then, per token t and straight from the definitions (Mamba2 recurrence in both directions, each
+    contributing delta_t (B_t . C_t) x_t + D x_t; attention over a single key returns its value):
+        Out_t = [2 (delta_t (B_t . C_t) + D) x_t] W_out^T + v_t W_o^T,
+    with x | B | C | dt the columns of X_t W_in^T, delta = softplus(dt + dt_bias), v the last third of
+    X_t W_qkv^T.  A permutation that does not return each token's result to its own row, a dropped
+    direction, a misplaced column block or a wrong softplus argument fails it."""
+    import dataclasses
+    cfg = dataclasses.replace(_small_cfg(T=4, H=8, W=8, R=16, B=2), wt=1, wh=1, ww=1, st=0, sh=0, sw=0)
+    w = make_inputs(cfg, dt_bias=60.0, a_log_range=(0.5, 1.0))   # delta > 60, |A| >= e^0.5
+    X = np.asarray(w["X"], np.float64).reshape(-1, cfg.d)
+    Z = X @ np.asarray(w["W_in"], np.float64).T
+    nP = cfg.nh * cfg.P
+    x = Z[:, :nP].reshape(-1, cfg.nh, cfg.P)
+    bc = np.sum(Z[:, nP:nP + cfg.N] * Z[:, nP + cfg.N:nP + 2 * cfg.N], axis=1)           # B_t . C_t
+    dtv = Z[:, nP + 2 * cfg.N:nP + 2 * cfg.N + cfg.nh] + np.asarray(w["dt_bias"], np.float64)
+    delta = np.log1p(np.exp(dtv))
+    assert (delta * np.exp(np.asarray(w["A_log"], np.float64))).min() > 60.0
+    y = 2.0 * (delta * bc[:, None] + np.asarray(w["D"], np.float64)[None, :])[:, :, None] * x
+    a = cfg.th * cfg.tp
+    v = (X @ np.asarray(w["W_qkv"], np.float64).T)[:, 2 * a:3 * a]
+    want = y.reshape(-1, nP) @ np.asarray(w["W_out"], np.float64).T + v @ np.asarray(w["W_o"], np.float64).T
+    for layer in range(4):
+        got = O.mate_forward(w["X"], w, cfg, layer).reshape(-1, cfg.d)
+        np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-9 * np.abs(want).max())
+
+
 def test_ma_branch_without_prefix_is_scan_of_reordered_tokens():
     # R = 0, D = 0, W_out = identity on d_inner = d: MA(X) = unpermute(bidir-scan(in_proj(permute(X))))
     cfg = MateConfig("t", 1, 2, 4, 4, 8, 2, 4, 3, 8, 0, 1, 8, 2, 4, 4, 1, 2, 2, "f32", 0)
