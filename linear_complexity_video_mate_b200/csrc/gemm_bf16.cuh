@@ -12,7 +12,8 @@
 //   warps 2..9  epilogue: tcgen05.ld the finished accumulator, convert, store; the other accumulator
 //               is being filled meanwhile.  Two warps per TMEM lane quadrant, one column half each, so
 //               that a tile's epilogue (bias, GELU, residual, 256 columns) keeps up with a short
-//               (K = 1024) main loop.
+//               (K = 1024) main loop.  Each warp's 32 rows x 32 columns go through a 2 KB transpose
+//               buffer, so that every store instruction writes eight whole 64-byte row segments.
 // Optional epilogue side output: columns [dt_col0, dt_col0 + dt_cols) also produce
 // delta = softplus(acc + dt_bias) in fp32 (the Mamba2 step size).  Optional epilogue transforms
 // (GemmEpilogue) serve the DiT block around MATE: bias + GELU for the MLP's first layer, bias and a gated
@@ -83,6 +84,7 @@ __device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log
 // the accumulator (two buffers of up to 256 columns) and each CTA runs its own epilogue.
 // ---------------------------------------------------------------------------------------------------
 __host__ __device__ inline uint32_t gemm_pair_stage_bytes(int bn) { return 128 * 128 + (bn / 2) * 128; }
+constexpr uint32_t kGemmStageOut = kGemmEpiWarps * 2048;   // epilogue transpose buffers, after the barriers
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -190,9 +192,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t acc_par = (it >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_par)) break;
       tc_fence_after();
-      const int row = mb * 256 + rank * 128 + quad * 32 + lane;
+      const int row0 = mb * 256 + rank * 128 + quad * 32;   // this warp's first row
+      const int row = row0 + lane;
       const bool row_ok = row < p.M;
       __nv_bfloat16* crow = p.C + static_cast<size_t>(row) * p.ldc;
+      // 32 rows x 16-byte chunks c at position c ^ ((row >> 1) & 3): conflict-free writes and reads
+      uint4* stg = reinterpret_cast<uint4*>(smem + p.stages * stage_bytes + 256) + (warp - 2) * 128;
       const int col_end = min(p.N, nb * p.bn + p.bn);
       const int c_hi = min(col_end - nb * p.bn, chalf * 128 + 128);
       for (int c0 = chalf * 128; c0 < c_hi; c0 += 32) {
@@ -200,11 +205,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256 + c0, r);
         tmem_wait_ld();
         const int col0 = nb * p.bn + c0;
-        if (!row_ok || col0 >= col_end) continue;
+        if (col0 >= col_end) continue;                 // the same for the whole warp
+        const bool full32 = col0 + 32 <= col_end;      // the same for the whole warp
+        // a full slice is stored by the whole warp together (rows past M are dropped at the store);
+        // a ragged one row by row
+        if (!full32 && !row_ok) continue;
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        const bool full32 = col0 + 32 <= col_end;
         if (has_ep) {
           const GemmEpilogue& e = p.ep;
           if (e.bias != nullptr) {
@@ -224,7 +232,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_f<true>(v[j]);
           }
-          if (e.resid != nullptr) {
+          if (e.resid != nullptr && row_ok) {
             const __nv_bfloat16* rr = static_cast<const __nv_bfloat16*>(e.resid) + row * e.ld_resid + col0;
             const float* g = e.gate != nullptr ? e.gate + static_cast<long long>(row / e.gate_rows) * e.ld_gate + col0
                                                : nullptr;
@@ -256,7 +264,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         const bool f16 = col0 < p.f16_cols;   // the 32-column slice lies wholly on one side
         if (full32) {
-          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 pk;
@@ -271,8 +278,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               pk.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
               pk.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
             }
-            dst[q] = pk;
+            stg[lane * 4 + (q ^ ((lane >> 1) & 3))] = pk;
           }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {   // rows 8 i .. 8 i + 7 of the warp, four lanes per 64-byte segment
+            const int rr = i * 8 + (lane >> 2), q = lane & 3;
+            if (row0 + rr < p.M)
+              reinterpret_cast<uint4*>(p.C + static_cast<size_t>(row0 + rr) * p.ldc + col0)[q] =
+                  stg[rr * 4 + (q ^ ((rr >> 1) & 3))];
+          }
+          __syncwarp();
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -285,7 +301,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               }
             }
         }
-        if (p.delta != nullptr && col0 < p.dt_col0 + p.dt_cols && col0 + 32 > p.dt_col0) {
+        if (p.delta != nullptr && row_ok && col0 < p.dt_col0 + p.dt_cols && col0 + 32 > p.dt_col0) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int c = col0 + j - p.dt_col0;

@@ -288,10 +288,10 @@ mate_status gemm_bf16(int kid, const void* A, int lda, long long M, int K, const
   // 256-row tiles computed by 2-CTA clusters (tcgen05 cta_group::2)
   p.num_tiles = ceil_div(M, 256) * p.num_n_tiles;
   const uint32_t psb = gemm_pair_stage_bytes(p.bn);
-  p.stages = std::min<int>(8, static_cast<int>((kSmemLimit - 1024 - 256) / psb));
+  p.stages = std::min<int>(8, static_cast<int>((kSmemLimit - 1024 - 256 - kGemmStageOut) / psb));
   CUtensorMap ta, tb;
   if (!make_tmap(&ta, A, M, K, lda, 128) || !make_tmap(&tb, Bw, N, K, ldb, p.bn / 2)) return MATE_ERR_CUDA;
-  const size_t smem = 1024 + (size_t)p.stages * psb + 256;
+  const size_t smem = 1024 + (size_t)p.stages * psb + 256 + kGemmStageOut;
   if (!set_smem(gemm_bf16_pair_kernel, smem)) return MATE_ERR_CUDA;
   const int pairs = std::min(p.num_tiles, device_sms() / 2);
   trace_begin(kid, st);
