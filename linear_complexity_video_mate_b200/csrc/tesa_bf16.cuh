@@ -13,7 +13,9 @@
 //   warps 5..12  softmax and output, one warp per (TMEM lane quadrant, query tile), one thread per query
 //                row: exact row softmax over all 256 keys (region mask only in windows that hold several
 //                wrap regions), P written in bf16 back into the row's own S columns ([256 t, 256 t + 128),
-//                two keys per column, each column written after it was read); then O / rowsum to global.
+//                two keys per column, each column written after it was read); then O / rowsum to global,
+//                32 columns at a time through a 2 KB transpose buffer per warp, so that each store
+//                instruction writes eight whole 64-byte row segments.
 // P never touches shared memory, so Q / K / V buffers are refilled while the softmax and P V of the
 // current item run.
 #pragma once
@@ -45,7 +47,9 @@ struct TesaRows {   // per item, two of them
 };
 constexpr uint32_t kTesaOffQ = 0, kTesaOffK = 65536, kTesaOffV = 131072, kTesaOffRows = 196608;
 constexpr uint32_t kTesaOffBar = kTesaOffRows + 2 * 3328;
-constexpr uint32_t kTesaSmem = kTesaOffBar + 256;
+constexpr uint32_t kTesaOffStage = kTesaOffBar + 256;   // output transpose buffers, 2 KB per softmax warp
+constexpr uint32_t kTesaSmem = kTesaOffStage + kTesaSoftWarps * 2048;
+static_assert(kTesaSmem + 1024 <= 232448, "shared memory of the TESA kernel");
 static_assert(sizeof(TesaRows) <= 3328, "row table size");
 
 __global__ void __launch_bounds__(kTesaThreads, 1) tesa_bf16_kernel(const TesaBf16Params p) {
@@ -269,25 +273,34 @@ __global__ void __launch_bounds__(kTesaThreads, 1) tesa_bf16_kernel(const TesaBf
       tc_fence_before();
       mbar_arrive(p_full);
       const float inv = 1.f / sum;
-      __nv_bfloat16* orow = p.O + rt.srow[i] * p.ldo + p.ocol + hd * 128;
       if (__any_sync(0xffffffffu, !mbar_wait(o_full, k & 1))) break;
       tc_fence_after();
+      // this warp's 32 rows x 32 columns at a time: 16-byte chunk c of row r at position c ^ ((r >> 1) & 3)
+      // (conflict-free writes and reads), then four lanes per row segment
+      uint4* stg = reinterpret_cast<uint4*>(smem + kTesaOffStage + sw * 2048);
+      const long long* srw = rt.srow + t * 128 + quad * 32;
+      __nv_bfloat16* ob = p.O + p.ocol + hd * 128;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 64) {
-        uint32_t v[64];
-        tmem_ld32(srow_t + 128 + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(srow_t + 128 + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(srow_t + 128 + c0, v);
         tmem_wait_ld();
-        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < 4; ++q) {
           uint4 pk;
           pk.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]) * inv, __uint_as_float(v[q * 8 + 1]) * inv);
           pk.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]) * inv, __uint_as_float(v[q * 8 + 3]) * inv);
           pk.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]) * inv, __uint_as_float(v[q * 8 + 5]) * inv);
           pk.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]) * inv, __uint_as_float(v[q * 8 + 7]) * inv);
-          dst[q] = pk;
+          stg[lane * 4 + (q ^ ((lane >> 1) & 3))] = pk;
         }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int rr = u * 8 + (lane >> 2), q = lane & 3;
+          reinterpret_cast<uint4*>(ob + srw[rr] * p.ldo + c0)[q] = stg[rr * 4 + (q ^ ((rr >> 1) & 3))];
+        }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
