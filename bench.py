@@ -128,8 +128,8 @@ def tensor_peak(peaks, region_s, clocks):
 # DRAM bytes per launch measured with ncu (dram__bytes_read.sum + dram__bytes_write.sum), scaled to the
 # bench workload as the profile summary explains; valid only while the kernel source is the one captured.
 MEASURED_TRAFFIC = {
-    "in_projection": {"bytes": 2.667e9, "source": "linear_complexity_video_mate_b200/csrc/gemm_bf16.cuh",
-                      "sha1": "f990f6124c1825c1e17d95057c35d90b97ebb559",
+    "in_projection": {"bytes": 2.675e9, "source": "linear_complexity_video_mate_b200/csrc/gemm_bf16.cuh",
+                      "sha1": "8631257f47be87c82d568522e3bc0b600917d489",
                       "profile": "profiles/gemm_bf16_pair_in_projection_bf16_64x32x32.md",
                       "workload": "bf16_256x32x32"},
 }

@@ -692,7 +692,7 @@ __global__ void __launch_bounds__(128) ssd_carry_kernel(const SsdBf16Params p) {
 //                MN-major, TMA four-row gathers) into one of two x buffers.
 //   warp 1       per group: the tile's C rows (K-major, four-row gathers); per item: the head's incoming
 //                states as four [N = 128][P = 64] blocks, Hf hi, Hb hi, Hf lo, Hb lo (MN-major, 2D TMA),
-//                through a ring of two 16 KB slots.
+//                through a ring of three 16 KB slots, so that up to three are in flight.
 //   warp 2       per group: the tile's rows of G (2D TMA) into four 64-column slots, each refilled once
 //                the last head of the previous group has read it.
 //   warp 3       MMA issue (lane 0 only; an issuing thread stalls while the tensor pipe is busy, so it has
@@ -725,12 +725,11 @@ constexpr uint32_t kOutTblBytes = kOutTbl * 4;         // 8704
 constexpr uint32_t kOutXBuf = 32768;                    // x tile of one item, two of them
 constexpr uint32_t kOutOffTbl = 2 * kOutXBuf;           // the item's decay tables, two of them
 constexpr uint32_t kOutOffC = kOutOffTbl + 2 * kOutTblBytes;   // C rows of the tile: 2 K blocks of 16 KB
-constexpr uint32_t kOutHSlots = 2;                      // ring of [N = 128][P = 64] state blocks
+constexpr uint32_t kOutHSlots = 3;                      // ring of [N = 128][P = 64] state blocks
 constexpr uint32_t kOutOffH = kOutOffC + 32768;
 constexpr uint32_t kOutOffG = kOutOffH + kOutHSlots * 16384;   // 4 slots of [128 rows][64 cols] K-major
 constexpr uint32_t kOutOffBar = kOutOffG + 4 * 16384;
-constexpr uint32_t kOutOffStage = kOutOffBar + 256;     // epilogue transpose buffers, 4 KB per epilogue warp
-constexpr uint32_t kOutSmem = kOutOffStage + kOutEpiWarps * 4096;
+constexpr uint32_t kOutSmem = kOutOffBar + 256;
 static_assert(kOutOffC % 1024 == 0 && kOutOffH % 1024 == 0 && kOutOffG % 1024 == 0, "1024-byte operand tiles");
 static_assert(kOutSmem + 1024 <= 232448, "shared memory of the output kernel");
 
@@ -751,8 +750,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
   uint64_t* x_full = bars;         // [2] x + table bytes
   uint64_t* x_empty = bars + 2;    // [2] last Yd MMA commit (the epilogue reads its x rows and table
                                    //     entries from global memory, so the buffer never waits for it)
-  uint64_t* h_full = bars + 4;     // [kOutHSlots <= 3] one state block's bytes
-  uint64_t* h_empty = bars + 7;    // [kOutHSlots <= 3] the Yf / Yb MMA commit that read the slot
+  uint64_t* h_full = bars + 4;     // [3] one state block's bytes
+  uint64_t* h_empty = bars + 7;    // [3] the Yf / Yb MMA commit that read the slot
   uint64_t* c_full = bars + 10;    // C bytes (per group)
   uint64_t* c_empty = bars + 11;   // last head's Yf / Yb MMA commit
   uint64_t* g_full = bars + 12;    // [4] one G slot's bytes (per group)
@@ -776,7 +775,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
       mbar_init(&y_full[q], 1);
       mbar_init(&y_empty[q], kOutEpiWarps);
     }
-    for (int q = 0; q < static_cast<int>(kOutHSlots); ++q) {
+    for (int q = 0; q < 3; ++q) {
       mbar_init(&h_full[q], 1);
       mbar_init(&h_empty[q], 1);
     }
@@ -864,8 +863,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
       for (int kb = 0; kb < 2; ++kb)
         tma_gather4(&mp.c, c_full, smem + kOutOffC + kb * 16384 + lane * 512, kb * 64, id[0], id[1], id[2], id[3]);
       for (int h = 0; h < nh && ok; ++h, ++k) {
-        for (int q = 0; q < 4; ++q) {   // Hf hi, Hb hi, Hf lo, Hb lo through the ring of slots
-          const int u = 4 * k + q, sl = u % kOutHSlots, use = u / kOutHSlots;
+        for (int q = 0; q < 4; ++q) {   // Hf hi, Hb hi, Hf lo, Hb lo through the ring of three slots
+          const int u = 4 * k + q, sl = u % 3, use = u / 3;
           if (!wait_all(&h_empty[sl], (use & 1) ^ 1)) { ok = false; break; }
           if (lane == 0) {
             mbar_arrive_expect_tx(&h_full[sl], 16384);
@@ -911,7 +910,7 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           const uint32_t ybase = tmem + 128 + acc * 192;
           // Yf (+)= C Hf^T or Yb (+)= C Hb^T from the ring slot of part q (0: Hf hi, 1: Hb hi, 2: Hf lo, 3: Hb lo)
           auto state_product = [&](int q) -> bool {
-            const int u = 4 * k + q, sl = u % kOutHSlots, hu = u / kOutHSlots;
+            const int u = 4 * k + q, sl = u % 3, hu = u / 3;
             if (!mbar_wait(&h_full[sl], hu & 1)) return false;
             tc_fence_after();
             const uint32_t hs = hbase + sl * 16384;
@@ -1102,10 +1101,8 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
         if (!wait_all(&y_full[acc], use & 1)) { ok = false; break; }
         tc_fence_after();
         const float D2 = 2.f * (Dh + (valid ? gdi * dli : 0.f));
+        __nv_bfloat16* ydst = p.y + yrow * p.ldy + h * kSsdP;
         const uint32_t ybase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128 + acc * 192;
-        // the warp's 32 rows x 64 columns go through its transpose buffer (16-byte chunk c of row r at
-        // position c ^ (r & 7): conflict-free writes and reads), then out as whole 128-byte row segments
-        uint4* stg = reinterpret_cast<uint4*>(smem + kOutOffStage + (warp - kOutFirstEpiWarp) * 4096);
 #pragma unroll
         for (int pc = 0; pc < 4; ++pc) {   // 16 columns at a time
           uint32_t yd[16], yf[16], yb[16];
@@ -1113,31 +1110,26 @@ __global__ void __launch_bounds__(kSsdOutThreads, 1) ssd_output_kernel(const Ssd
           tmem_ld16(ybase + 64 + pc * 16, yf);
           tmem_ld16(ybase + 128 + pc * 16, yb);
           tmem_wait_ld();
-          uint32_t ou[8];
+          if (valid) {
+            uint32_t ou[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 xf = XF16 ? unpack_f16x2(xw[pc * 8 + e]) : unpack_bf16x2(xw[pc * 8 + e]);
-            const int k0 = 2 * e;
-            const float y0 = __uint_as_float(yd[k0]) + ef * __uint_as_float(yf[k0]) +
-                             eb * __uint_as_float(yb[k0]) + D2 * xf.x;
-            const float y1 = __uint_as_float(yd[k0 + 1]) + ef * __uint_as_float(yf[k0 + 1]) +
-                             eb * __uint_as_float(yb[k0 + 1]) + D2 * xf.y;
-            ou[e] = pack_bf16x2(y0, y1);
+            for (int e = 0; e < 8; ++e) {
+              const float2 xf = XF16 ? unpack_f16x2(xw[pc * 8 + e]) : unpack_bf16x2(xw[pc * 8 + e]);
+              const int k0 = 2 * e;
+              const float y0 = __uint_as_float(yd[k0]) + ef * __uint_as_float(yf[k0]) +
+                               eb * __uint_as_float(yb[k0]) + D2 * xf.x;
+              const float y1 = __uint_as_float(yd[k0 + 1]) + ef * __uint_as_float(yf[k0 + 1]) +
+                               eb * __uint_as_float(yb[k0 + 1]) + D2 * xf.y;
+              ou[e] = pack_bf16x2(y0, y1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(ydst + pc * 16);
+            dst[0] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+            dst[1] = make_uint4(ou[4], ou[5], ou[6], ou[7]);
           }
-          stg[lane * 8 + ((2 * pc) ^ (lane & 7))] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
-          stg[lane * 8 + ((2 * pc + 1) ^ (lane & 7))] = make_uint4(ou[4], ou[5], ou[6], ou[7]);
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&y_empty[acc]);   // the accumulators are read: the MMAs may reuse them
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {   // rows 4 u .. 4 u + 3 of the warp, eight lanes per row segment
-          const int rr = u * 4 + (lane >> 3), q = lane & 7;
-          const long long yr = __shfl_sync(0xffffffffu, yrow, rr);
-          const int vr = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr);
-          if (vr) reinterpret_cast<uint4*>(p.y + yr * p.ldy + h * kSsdP)[q] = stg[rr * 8 + (q ^ (rr & 7))];
-        }
-        __syncwarp();   // the buffer is read before the next item writes it
+        if (lane == 0) mbar_arrive(&y_empty[acc]);
       }
     }
   }
