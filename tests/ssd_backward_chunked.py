@@ -27,13 +27,14 @@ def _chunks(L: int, Q: int):
     return [(c0, min(c0 + Q, L)) for c0 in range(0, L, Q)]
 
 
-def ssd_backward_chunked(x, Bm, Cm, delta, A, D, dy, Q: int):
+def ssd_backward_chunked(x, Bm, Cm, delta, A, D, dy, Q: int, chunks=None):
     """Gradients of the one-direction recurrence (same outputs as oracle.backward.ssd_recurrence_backward)
-    computed chunk by chunk.  x [L, nh, P], Bm / Cm [L, N], delta [L, nh], A / D [nh], dy [L, nh, P]."""
+    computed chunk by chunk.  x [L, nh, P], Bm / Cm [L, N], delta [L, nh], A / D [nh], dy [L, nh, P].
+    `chunks` (a list of [c0, c1) covering 0..L in order) overrides the uniform cut into Q rows."""
     x, Bm, Cm, delta, A, D, dy = (np.asarray(v, np.float64) for v in (x, Bm, Cm, delta, A, D, dy))
     L, nh, P = x.shape
     N = Bm.shape[1]
-    chunks = _chunks(L, Q)
+    chunks = _chunks(L, Q) if chunks is None else list(chunks)
     dx, dB, dC = np.zeros_like(x), np.zeros_like(Bm), np.zeros_like(Cm)
     ddelta, dA, dD = np.zeros_like(delta), np.zeros(nh), np.zeros(nh)
     for h in range(nh):
@@ -79,3 +80,41 @@ def ssd_backward_chunked(x, Bm, Cm, delta, A, D, dy, Q: int):
             ddelta[c0:c1, h] = np.sum(xs * gB, axis=1) + A[h] * da
             dA[h] += np.sum(dl * da)
     return dx, dB, dC, ddelta, dA, dD
+
+
+def kernel_chunks(R: int, n: int, Q: int, backward: bool):
+    """The chunk boundaries the tensor-core scan uses over [review rows; video rows]: ceil(R/Q) review
+    chunks, then the video rows cut at multiples of Q of the scan position.  The backward traversal runs
+    over [review rows; video rows reversed] and visits the same video chunks in reverse order, so in its
+    own coordinates a partial last video chunk comes first."""
+    out = [(c0, min(c0 + Q, R)) for c0 in range(0, R, Q)]
+    video = [(v0, min(v0 + Q, n)) for v0 in range(0, n, Q)]
+    if backward:
+        video = [(n - v1, n - v0) for v0, v1 in reversed(video)]
+    return out + [(R + a, R + b) for a, b in video]
+
+
+def ssd_bidirectional_backward_chunked(x, Bm, Cm, delta, A, D, R: int, dy, Q: int):
+    """Gradients of the bidirectional scan with a prefix (the same outputs as
+    oracle.backward.ssd_bidirectional_backward), each direction computed chunk by chunk on the chunks the
+    forward kernels use: the forward direction over [prefix; video], the backward direction over [prefix;
+    video reversed] with its per-row gradients mapped back through the flip."""
+    x = np.asarray(x, np.float64)
+    L, nh, P = x.shape
+    n = L - R
+    dy = np.asarray(dy, np.float64)
+    dyf = np.zeros((L, nh, P))
+    dyf[R:] = dy
+    gf = ssd_backward_chunked(x, Bm, Cm, delta, A, D, dyf, Q, kernel_chunks(R, n, Q, False))
+    flip = np.concatenate([np.arange(R), np.arange(L - 1, R - 1, -1)])
+    dyb = np.zeros((L, nh, P))
+    dyb[R:] = dy[::-1]
+    Bm, Cm, delta = (np.asarray(v, np.float64) for v in (Bm, Cm, delta))
+    gb = ssd_backward_chunked(x[flip], Bm[flip], Cm[flip], delta[flip], A, D, dyb, Q, kernel_chunks(R, n, Q, True))
+    out = []
+    for f, b in zip(gf[:4], gb[:4]):
+        g = f.copy()
+        g[flip] += b
+        out.append(g)
+    return out[0], out[1], out[2], out[3], gf[4] + gb[4], gf[5] + gb[5]
+
